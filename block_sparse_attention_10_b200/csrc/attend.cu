@@ -1,0 +1,319 @@
+// attend.cu — exact softmax attention over the selected NVFP4 blocks (decode).
+//
+// "Main attention then runs exactly, but only over the top 16 blocks ... That
+// caps each query at 2,048 keys" ("vLLM Adds Day-0 Support for
+// MiniMax-M3.1-Flash", ainewsbites.com, "A model built for efficient
+// inference").  Query head h reads KV head h / (Hq/Hkv); keys j > pos are
+// masked; K and V are NVFP4 and dequantised in registers.
+//
+// Design (B200): one thread-block cluster of 4 CTAs x 4 warps per
+// (sequence, query token, KV head): each of the 16 warps takes one selected
+// block (split-K over the <= 16 blocks), so the whole gather of <= 2,048 keys
+// is in flight at once.  Per 16 keys a warp computes
+//   S   = Q K^T    mma m16n8k16: A = the G query heads of this KV head
+//                  (zero-padded to 16 rows), B = dequantised K (exact f16);
+//   P   = online softmax of S in the exp2 domain (fp32);
+//   O^T += V^T P^T mma m16n8k16: A = dequantised V (exact f16), B = P as
+//                  fp16 taken straight from S's accumulator layout, so the
+//                  output tile [128 dims x 8 heads] wastes no rows.
+// The partial (m, l, O) of the 4 warps are merged in shared memory, then the 4
+// CTAs of the cluster merge through distributed shared memory (each CTA
+// finalises 32 of the 128 dims).  No global scratch, no second launch, a
+// fixed merge order (bitwise deterministic).  K/V tiles are double-buffered
+// in registers (128-bit loads for K, 64-bit for V; both fully coalesced).
+#include <cooperative_groups.h>
+
+#include "internal.h"
+
+namespace msa {
+namespace {
+
+namespace cg = cooperative_groups;
+
+constexpr int kAttWarps = 4;
+constexpr int kAttCluster = 4;
+constexpr int kAttThreads = 32 * kAttWarps;
+constexpr int kD = 128;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+struct KVTile {
+    uint4 k[2];      // keys base+g, base+8+g: bytes [16c, 16c+16) of the key's 64-byte row
+    uint32_t ks[2];  // their E4M3 scales of groups 2c, 2c+1 (16 bits)
+    uint2 v[4];      // keys base+{2c, 2c+1, 2c+8, 2c+9}: bytes [8g, 8g+8) (dims 16g..16g+15)
+    uint32_t vs[4];  // their E4M3 scale of group g
+};
+
+__device__ __forceinline__ void load_tile(KVTile& T, const uint8_t* kd, const uint8_t* ksc, const uint8_t* vd,
+                                          const uint8_t* vsc, int base, int nk, int g, int c) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int key = base + 8 * h + g;
+        if (key < nk) {
+            T.k[h] = ldg_nc_v4(kd + key * 64 + c * 16);
+            T.ks[h] = ldg_nc_u16(ksc + key * 8 + c * 2);
+        } else {
+            T.k[h] = make_uint4(0u, 0u, 0u, 0u);
+            T.ks[h] = 0u;
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int key = base + 2 * c + (i & 1) + 8 * (i >> 1);
+        if (key < nk) {
+            T.v[i] = ldg_nc_v2(vd + key * 64 + g * 8);
+            T.vs[i] = ldg_nc_u8(vsc + key * 8 + g);
+        } else {
+            T.v[i] = make_uint2(0u, 0u);
+            T.vs[i] = 0u;
+        }
+    }
+}
+
+template <int G>
+__global__ void __cluster_dims__(kAttCluster, 1, 1) __launch_bounds__(kAttThreads, 3)
+    attend_kernel(const Problem p, const int32_t* __restrict__ sel, float* __restrict__ out,
+                  float* __restrict__ lse) {
+    __shared__ __align__(16) float sO[kAttWarps][8][kD];
+    __shared__ float sM[kAttWarps][8], sL[kAttWarps][8];
+    __shared__ float cM[8], cL[8];
+
+    pdl_wait();
+    pdl_launch_dependents();
+
+    cg::cluster_group cluster = cg::this_cluster();
+    const int crank = (int)cluster.block_rank();
+    const int64_t unit = blockIdx.x / kAttCluster;  // ((b * Tq) + t) * Hkv + kvh
+    const int kvh = (int)(unit % p.Hkv);
+    const int64_t bt = unit / p.Hkv;
+    const int b = (int)(bt / p.Tq), t = (int)(bt % p.Tq);
+    const int64_t L = clamp_len(p.seq_lens[b], p.Tq, p.lmax, nullptr);
+    const int64_t pos = L - p.Tq + t;
+    const int64_t nvis = pos / kBlock + 1;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, c = lane & 3;
+    const int gw = crank * kAttWarps + warp;
+
+    // Q rows (query heads kvh*G + g), dims [32c, 32c+32) as 16 f16x2 pairs
+    uint32_t qa[8][2];
+    if (g < G) {
+        const __nv_bfloat16* qrow = p.q + ((bt * p.Hq) + (int64_t)kvh * G + g) * kD + c * 32;
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            const uint4 w4 = *reinterpret_cast<const uint4*>(qrow + 8 * v);
+            qa[2 * v][0] = bf16x2_to_f16x2(w4.x);
+            qa[2 * v][1] = bf16x2_to_f16x2(w4.y);
+            qa[2 * v + 1][0] = bf16x2_to_f16x2(w4.z);
+            qa[2 * v + 1][1] = bf16x2_to_f16x2(w4.w);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) qa[i][0] = qa[i][1] = 0u;
+    }
+
+    const float sc_log2 = p.softmax_scale * p.k.s_t * kLog2e;
+    float m_run = -INFINITY, l_run = 0.0f;
+    float o[8][4];
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.0f;
+
+    const int32_t* srow = sel + bt * kTopK;
+    for (int si = gw; si < kTopK; si += kAttCluster * kAttWarps) {
+        const int blk = srow[si];
+        if (blk < 0) continue;
+        if (blk >= nvis) {
+            if (lane == 0) set_status(p.status, MSA_STATUS_SELECT);
+            continue;
+        }
+        const int64_t kbase = (int64_t)blk * kBlock;
+        const int nk = (int)min64(kBlock, pos + 1 - kbase);
+        const int64_t vec0 = ((int64_t)b * p.Hkv + kvh) * p.lmax + kbase;
+        const uint8_t* kd = p.k.data + vec0 * 64;
+        const uint8_t* ksc = p.k.scale + vec0 * 8;
+        const uint8_t* vd = p.v.data + vec0 * 64;
+        const uint8_t* vsc = p.v.scale + vec0 * 8;
+        const int ntiles = (nk + 15) >> 4;
+
+        KVTile cur, nxt;
+        load_tile(cur, kd, ksc, vd, vsc, 0, nk, g, c);
+        for (int kt = 0; kt < ntiles; ++kt) {
+            if (kt + 1 < ntiles) load_tile(nxt, kd, ksc, vd, vsc, (kt + 1) * 16, nk, g, c);
+            // ---- S = Q K^T over 16 keys (two n-tiles of 8 keys)
+            float sacc[2][4];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                sacc[h][0] = sacc[h][1] = sacc[h][2] = sacc[h][3] = 0.0f;
+                uint32_t kh[16];
+                e2m1x8_to_f16x8(cur.k[h].x, kh[0], kh[1], kh[2], kh[3]);
+                e2m1x8_to_f16x8(cur.k[h].y, kh[4], kh[5], kh[6], kh[7]);
+                e2m1x8_to_f16x8(cur.k[h].z, kh[8], kh[9], kh[10], kh[11]);
+                e2m1x8_to_f16x8(cur.k[h].w, kh[12], kh[13], kh[14], kh[15]);
+                const uint32_t slo = e4m3_bcast_f16x2(cur.ks[h]), shi = e4m3_bcast_f16x2(cur.ks[h] >> 8);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const uint32_t sc = i < 4 ? slo : shi;
+                    mma16816(sacc[h], qa[i][0], 0u, qa[i][1], 0u, hmul2(kh[2 * i], sc), hmul2(kh[2 * i + 1], sc));
+                }
+            }
+            // ---- online softmax for query row g (exp2 domain)
+            float x[4];
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int key = kt * 16 + 8 * h + 2 * c + e;
+                    x[2 * h + e] = key < nk ? sacc[h][e] * sc_log2 : -INFINITY;
+                }
+            float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            const float m_new = fmaxf(m_run, mx);
+            const float corr = exp2f(m_run - m_new);
+            float pr[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) pr[e] = exp2f(x[e] - m_new);
+            l_run = l_run * corr + (pr[0] + pr[1]) + (pr[2] + pr[3]);
+            m_run = m_new;
+            const uint32_t pb0 = pack_f16x2(pr[0], pr[1]), pb1 = pack_f16x2(pr[2], pr[3]);
+            // rescale O^T columns: this thread holds query rows 2c and 2c+1
+            const float c0 = __shfl_sync(0xffffffffu, corr, 8 * c), c1 = __shfl_sync(0xffffffffu, corr, 8 * c + 4);
+            // ---- O^T += V^T P^T
+            uint32_t vh[4][8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                e2m1x8_to_f16x8(cur.v[i].x, vh[i][0], vh[i][1], vh[i][2], vh[i][3]);
+                e2m1x8_to_f16x8(cur.v[i].y, vh[i][4], vh[i][5], vh[i][6], vh[i][7]);
+                const uint32_t sc = e4m3_bcast_f16x2(cur.vs[i]);
+#pragma unroll
+                for (int m = 0; m < 8; ++m) vh[i][m] = hmul2(vh[i][m], sc);
+            }
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                o[mt][0] *= c0;
+                o[mt][1] *= c1;
+                o[mt][2] *= c0;
+                o[mt][3] *= c1;
+                const uint32_t a0 = prmt(vh[0][mt], vh[1][mt], 0x5410u);
+                const uint32_t a1 = prmt(vh[0][mt], vh[1][mt], 0x7632u);
+                const uint32_t a2 = prmt(vh[2][mt], vh[3][mt], 0x5410u);
+                const uint32_t a3 = prmt(vh[2][mt], vh[3][mt], 0x7632u);
+                mma16816(o[mt], a0, a1, a2, a3, pb0, pb1);
+            }
+            cur = nxt;
+        }
+    }
+
+    // ---- merge the 4 warps of this CTA
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+    l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+    if (c == 0) {
+        sM[warp][g] = m_run;
+        sL[warp][g] = l_run;
+    }
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+        const int d = 16 * g + 2 * mt;
+        sO[warp][2 * c][d] = o[mt][0];
+        sO[warp][2 * c + 1][d] = o[mt][1];
+        sO[warp][2 * c][d + 1] = o[mt][2];
+        sO[warp][2 * c + 1][d + 1] = o[mt][3];
+    }
+    __syncthreads();
+    {
+        const int q = threadIdx.x >> 4, d0 = (threadIdx.x & 15) * 8;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kAttWarps; ++w) M = fmaxf(M, sM[w][q]);
+        float f[kAttWarps], Lc = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kAttWarps; ++w) {
+            f[w] = sM[w][q] == -INFINITY ? 0.0f : exp2f(sM[w][q] - M);
+            Lc += f[w] * sL[w][q];
+        }
+        float acc[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kAttWarps; ++w)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[j] += f[w] * sO[w][q][d0 + j];
+        // all warps' reads of this (q, d0..d0+7) slice happen in this thread: safe to overwrite
+#pragma unroll
+        for (int j = 0; j < 8; ++j) sO[0][q][d0 + j] = acc[j];
+        if ((threadIdx.x & 15) == 0) {
+            cM[q] = M;
+            cL[q] = Lc;
+        }
+    }
+    cluster.sync();
+
+    // ---- merge the 4 CTAs of the cluster: CTA r finalises dims [32r, 32r + 32)
+    {
+        const int q = threadIdx.x >> 4, d = 32 * crank + (threadIdx.x & 15) * 2;
+        float Mr[kAttCluster], Lr[kAttCluster], O0[kAttCluster], O1[kAttCluster];
+#pragma unroll
+        for (int r = 0; r < kAttCluster; ++r) {
+            const float* pm = cluster.map_shared_rank(&cM[0], r);
+            const float* pl = cluster.map_shared_rank(&cL[0], r);
+            const float* po = cluster.map_shared_rank(&sO[0][0][0], r);
+            Mr[r] = pm[q];
+            Lr[r] = pl[q];
+            const float2 v2 = *reinterpret_cast<const float2*>(po + q * kD + d);
+            O0[r] = v2.x;
+            O1[r] = v2.y;
+        }
+        float M = -INFINITY;
+#pragma unroll
+        for (int r = 0; r < kAttCluster; ++r) M = fmaxf(M, Mr[r]);
+        float Lt = 0.0f, a0 = 0.0f, a1 = 0.0f;
+#pragma unroll
+        for (int r = 0; r < kAttCluster; ++r) {
+            const float f = Mr[r] == -INFINITY ? 0.0f : exp2f(Mr[r] - M);
+            Lt += f * Lr[r];
+            a0 += f * O0[r];
+            a1 += f * O1[r];
+        }
+        if (q < G) {
+            const float inv = Lt > 0.0f ? p.v.s_t / Lt : 0.0f;
+            float* orow = out + ((bt * p.Hq) + (int64_t)kvh * G + q) * kD;
+            *reinterpret_cast<float2*>(orow + d) = make_float2(a0 * inv, a1 * inv);
+            if (lse != nullptr && crank == 0 && (threadIdx.x & 15) == 0)
+                lse[bt * p.Hq + (int64_t)kvh * G + q] = Lt > 0.0f ? (M + log2f(Lt)) * kLn2 : -INFINITY;
+        }
+    }
+    cluster.sync();  // keep this CTA's shared memory alive until every peer has read it
+}
+
+template <int G>
+int launch_g(const Problem& p, const int32_t* sel, float* out, float* lse, bool pdl, cudaStream_t st) {
+    const int64_t units = (int64_t)p.B * p.Tq * p.Hkv;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(units * kAttCluster));
+    cfg.blockDim = dim3(kAttThreads);
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, attend_kernel<G>, p, sel, out, lse) != cudaSuccess) return MSA_ECUDA;
+    return MSA_OK;
+}
+
+}  // namespace
+
+int launch_attend(const Problem& p, const int32_t* sel, float* out, float* lse, bool pdl, cudaStream_t st) {
+    if (p.D != kD) return MSA_EUNSUPPORTED;
+    const int64_t units = (int64_t)p.B * p.Tq * p.Hkv;
+    if (units * kAttCluster > 0x7FFFFFFFll) return MSA_EUNSUPPORTED;
+    switch (p.Hq / p.Hkv) {
+        case 1: return launch_g<1>(p, sel, out, lse, pdl, st);
+        case 2: return launch_g<2>(p, sel, out, lse, pdl, st);
+        case 4: return launch_g<4>(p, sel, out, lse, pdl, st);
+        case 8: return launch_g<8>(p, sel, out, lse, pdl, st);
+        default: return MSA_EUNSUPPORTED;
+    }
+}
+
+}  // namespace msa

@@ -1,0 +1,418 @@
+// index_decode.cu — MSA indexer + per-block pooling for decode (Tq * HI <= 32).
+//
+// Method ("vLLM Adds Day-0 Support for MiniMax-M3.1-Flash", ainewsbites.com,
+// "A model built for efficient inference"): a lightweight indexer scores every
+// key of the context and the scores are pooled into one score per 128-token
+// block.  Reading taken here: s_j = sum_h w_h * max(0, q_h . k_j) with one
+// NVFP4 index key per token; pooled = mean (or max) over visible tokens.
+//
+// Design (B200): the kernel is HBM-bound — it must stream every index key
+// (DI/2 + DI/16 bytes per token) exactly once for all Tq query tokens.
+//   * Persistent grid, 2 CTAs per SM.  Each CTA owns a contiguous range of
+//     (sequence, block) units; one producer lane streams each unit's NVFP4
+//     nibbles and scales (one 128-token block: 9 KB at DI = 128) into a ring
+//     of shared-memory stages with untiled bulk copies (cp.async.bulk, no
+//     multicast), signalled through mbarriers; 8 consumer warps take units
+//     round-robin.
+//   * Consumers dequantise in registers with the sm_100a converters
+//     (E2M1x2 -> f16x2, E4M3 -> f16; e2m1*e4m3 is exact in f16) and run the
+//     [16 keys x DI] x [DI x 8 queries] products on tensor cores
+//     (mma.sync m16n8k16, f32 accumulate).  The per-tensor fp32 scale is
+//     applied once, after pooling (ReLU and both pools commute with a
+//     positive scale).
+//   * Each thread reads the 16 (DI = 128) or 8 (DI = 64) contiguous bytes of
+//     a key that its A-fragment needs: the head dim is permuted identically
+//     on the key and query side (a dot product does not depend on the order
+//     of its terms), which makes every shared-memory read a 128/64-bit
+//     conflict-free load.
+//   * Epilogue in registers: ReLU, head weights, sum over heads with warp
+//     shuffles, causal / length masking, block pooling, one store per
+//     (token, block).
+#include "internal.h"
+
+namespace msa {
+namespace {
+
+constexpr int kIdxConsumers = 8;
+constexpr int kIdxThreads = 32 * (kIdxConsumers + 1);
+constexpr int kMaxB = 4096;
+
+template <int DI>
+struct IdxGeom {
+    static constexpr int kRowBytes = DI / 2;
+    static constexpr int kSclBytes = DI / 16;
+    static constexpr int kDataBytes = kBlock * kRowBytes;
+    static constexpr int kStageBytes = kBlock * (kRowBytes + kSclBytes);
+    static constexpr int kStages = DI == 128 ? 10 : 20;
+    static constexpr int kKSteps = DI / 16;
+    static constexpr int kPairs = DI / 8;  // f16x2 pairs of q per thread
+};
+
+template <int DI>
+constexpr size_t idx_smem_bytes(int B) {
+    return (size_t)IdxGeom<DI>::kStages * IdxGeom<DI>::kStageBytes + 2 * IdxGeom<DI>::kStages * sizeof(uint64_t) +
+           (size_t)(2 * B + 2) * sizeof(int);
+}
+
+template <int HI>
+__device__ __forceinline__ int token_of(int nt, int c, int e) {
+    if constexpr (HI == 1) return 8 * nt + 2 * c + e;
+    else if constexpr (HI == 2) return 4 * nt + c;
+    else if constexpr (HI == 4) return 2 * nt + (c >> 1);
+    else return nt;
+}
+template <int HI>
+__device__ __forceinline__ bool token_owner(int c) {
+    if constexpr (HI <= 2) return true;
+    else if constexpr (HI == 4) return (c & 1) == 0;
+    else return c == 0;
+}
+
+template <int DI, int HI, int NT>
+__global__ void __launch_bounds__(kIdxThreads, 2)
+    index_decode_kernel(const Problem p, float* __restrict__ block_scores, float* __restrict__ token_scores) {
+    using G = IdxGeom<DI>;
+    constexpr int S = G::kStages;
+    constexpr int KS = G::kKSteps;
+    constexpr int TPN = HI == 1 ? 2 : 1;  // tokens per thread per n-tile
+
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * G::kStageBytes);
+    uint64_t* empty = full + S;
+    int* prefix = reinterpret_cast<int*>(empty + S);  // [B + 1] units before sequence b
+    int* lens = prefix + (p.B + 1);                   // [B] clamped lengths
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int B = p.B, Tq = p.Tq;
+    const int NQ = Tq * HI;
+
+    pdl_wait();
+
+    if (warp == 0) {
+        int carry = 0;
+        if (lane == 0) prefix[0] = 0;
+        for (int b0 = 0; b0 < B; b0 += 32) {
+            const int b = b0 + lane;
+            int nb = 0;
+            if (b < B) {
+                const int64_t L = clamp_len(p.seq_lens[b], Tq, p.lmax, blockIdx.x == 0 ? p.status : nullptr);
+                lens[b] = (int)L;
+                nb = (int)((L + kBlock - 1) / kBlock);
+            }
+            int x = nb;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, x, o);
+                if (lane >= o) x += y;
+            }
+            if (b < B) prefix[b + 1] = carry + x;
+            carry += __shfl_sync(0xffffffffu, x, 31);
+        }
+        if (lane == 0) {
+            for (int s = 0; s < S; ++s) {
+                mbar_init(&full[s], 1);
+                mbar_init(&empty[s], 1);
+            }
+            fence_mbar_init();
+        }
+    }
+    __syncthreads();
+    pdl_launch_dependents();
+
+    const int64_t U = prefix[B];
+    const int64_t u_begin = U * blockIdx.x / gridDim.x;
+    const int nu = (int)(U * (blockIdx.x + 1) / gridDim.x - u_begin);
+
+    if (warp == 0) {
+        // ------------------------------------------------------------------ producer
+        if (lane == 0) {
+            int b = 0;
+            int k = 0;
+            bool ok = true;
+            for (; k < nu; ++k) {
+                const int s = k % S;
+                const uint32_t round = (uint32_t)(k / S);
+                if (round > 0 && !mbar_wait(&empty[s], (round - 1) & 1u)) {
+                    set_status(p.status, MSA_STATUS_TIMEOUT);
+                    ok = false;
+                    break;
+                }
+                const int64_t u = u_begin + k;
+                while (prefix[b + 1] <= u) ++b;
+                const int64_t n = u - prefix[b];
+                const int valid = (int)min64(kBlock, lens[b] - n * kBlock);
+                const int rows = (valid + 15) & ~15;
+                const uint32_t db = (uint32_t)(rows * G::kRowBytes), sb = (uint32_t)(rows * G::kSclBytes);
+                const int64_t row0 = (int64_t)b * p.lmax + n * kBlock;
+                uint8_t* st = smem + (size_t)s * G::kStageBytes;
+                mbar_arrive_expect_tx(&full[s], db + sb);
+                bulk_g2s(st, p.ik.data + row0 * G::kRowBytes, db, &full[s]);
+                bulk_g2s(st + G::kDataBytes, p.ik.scale + row0 * G::kSclBytes, sb, &full[s]);
+            }
+            // drain: never leave with copies in flight into this CTA's shared memory
+            const int issued = k;
+            for (int j = max(0, issued - S); j < issued; ++j) {
+                if (!mbar_wait(&full[j % S], (uint32_t)(j / S) & 1u)) {
+                    set_status(p.status, MSA_STATUS_TIMEOUT);
+                    break;
+                }
+            }
+            (void)ok;
+        }
+        return;
+    }
+
+    // ---------------------------------------------------------------------- consumers
+    const int cw = warp - 1;
+    const int g = lane >> 2, c = lane & 3;
+    const float s_t = p.ik.s_t;
+
+    // blocks past a sequence's length score -inf (no unit covers them)
+    {
+        const int64_t total = (int64_t)B * Tq * p.nbmax;
+        const int64_t stride = (int64_t)gridDim.x * kIdxConsumers * 32;
+        for (int64_t i = (int64_t)blockIdx.x * kIdxConsumers * 32 + cw * 32 + lane; i < total; i += stride) {
+            const int64_t n = i % p.nbmax;
+            const int b = (int)(i / (p.nbmax * Tq));
+            if (n >= prefix[b + 1] - prefix[b]) block_scores[i] = -INFINITY;
+        }
+    }
+
+    uint32_t qf[NT][KS][2];
+    float wq[NT][2];
+    int cur_b = -1;
+    int b = 0;
+
+    for (int k = cw; k < nu; k += kIdxConsumers) {
+        const int s = k % S;
+        if (!mbar_wait(&full[s], (uint32_t)(k / S) & 1u)) {
+            set_status(p.status, MSA_STATUS_TIMEOUT);
+            break;
+        }
+        const int64_t u = u_begin + k;
+        while (prefix[b + 1] <= u) ++b;
+        const int64_t n = u - prefix[b];
+        const int L = lens[b];
+        const int valid = (int)min64(kBlock, L - n * kBlock);
+        const int64_t kbase = n * kBlock;
+
+        if (b != cur_b) {
+            cur_b = b;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                const int qn = 8 * nt + g;
+                uint32_t pr[G::kPairs];
+                if (qn < NQ) {
+                    const __nv_bfloat16* row = p.q_idx + ((int64_t)b * Tq * HI + qn) * DI + c * (DI / 4);
+#pragma unroll
+                    for (int v = 0; v < G::kPairs / 4; ++v) {
+                        const uint4 w4 = *reinterpret_cast<const uint4*>(row + 8 * v);
+                        pr[4 * v + 0] = bf16x2_to_f16x2(w4.x);
+                        pr[4 * v + 1] = bf16x2_to_f16x2(w4.y);
+                        pr[4 * v + 2] = bf16x2_to_f16x2(w4.z);
+                        pr[4 * v + 3] = bf16x2_to_f16x2(w4.w);
+                    }
+                } else {
+#pragma unroll
+                    for (int v = 0; v < G::kPairs; ++v) pr[v] = 0u;
+                }
+#pragma unroll
+                for (int i = 0; i < KS; ++i) {
+                    qf[nt][i][0] = pr[2 * i];
+                    qf[nt][i][1] = pr[2 * i + 1];
+                }
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    const int qq = 8 * nt + 2 * c + e;
+                    wq[nt][e] = qq < NQ ? (p.w_idx ? p.w_idx[(int64_t)b * Tq * HI + qq] : 1.0f) : 0.0f;
+                }
+            }
+        }
+
+        const uint8_t* sd = smem + (size_t)s * G::kStageBytes;
+        const uint8_t* ss = sd + G::kDataBytes;
+        float pool[NT][TPN];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < TPN; ++e) pool[nt][e] = p.pool_mode == 1 ? -INFINITY : 0.0f;
+
+        const int ntiles = (valid + 15) >> 4;
+        for (int ti = 0; ti < ntiles; ++ti) {
+            const int r0 = ti * 16 + g, r1 = r0 + 8;
+            uint32_t h0[2 * KS], h1[2 * KS];  // f16x2 pairs of rows r0 / r1 (unscaled E2M1)
+            uint32_t s0[KS], s1[KS];          // per k-step E4M3 scale, broadcast f16x2
+            if constexpr (DI == 128) {
+                const uint4 w0 = lds_v4(sd + r0 * 64 + c * 16);
+                const uint4 w1 = lds_v4(sd + r1 * 64 + c * 16);
+                const uint32_t sc0 = lds_u16(ss + r0 * 8 + c * 2);
+                const uint32_t sc1 = lds_u16(ss + r1 * 8 + c * 2);
+                e2m1x8_to_f16x8(w0.x, h0[0], h0[1], h0[2], h0[3]);
+                e2m1x8_to_f16x8(w0.y, h0[4], h0[5], h0[6], h0[7]);
+                e2m1x8_to_f16x8(w0.z, h0[8], h0[9], h0[10], h0[11]);
+                e2m1x8_to_f16x8(w0.w, h0[12], h0[13], h0[14], h0[15]);
+                e2m1x8_to_f16x8(w1.x, h1[0], h1[1], h1[2], h1[3]);
+                e2m1x8_to_f16x8(w1.y, h1[4], h1[5], h1[6], h1[7]);
+                e2m1x8_to_f16x8(w1.z, h1[8], h1[9], h1[10], h1[11]);
+                e2m1x8_to_f16x8(w1.w, h1[12], h1[13], h1[14], h1[15]);
+                const uint32_t a0 = e4m3_bcast_f16x2(sc0), a1 = e4m3_bcast_f16x2(sc0 >> 8);
+                const uint32_t b0 = e4m3_bcast_f16x2(sc1), b1 = e4m3_bcast_f16x2(sc1 >> 8);
+#pragma unroll
+                for (int i = 0; i < KS; ++i) {
+                    s0[i] = i < 4 ? a0 : a1;
+                    s1[i] = i < 4 ? b0 : b1;
+                }
+            } else {
+                const uint2 w0 = lds_v2(sd + r0 * 32 + c * 8);
+                const uint2 w1 = lds_v2(sd + r1 * 32 + c * 8);
+                const uint32_t sc0 = lds_u8(ss + r0 * 4 + c);
+                const uint32_t sc1 = lds_u8(ss + r1 * 4 + c);
+                e2m1x8_to_f16x8(w0.x, h0[0], h0[1], h0[2], h0[3]);
+                e2m1x8_to_f16x8(w0.y, h0[4], h0[5], h0[6], h0[7]);
+                e2m1x8_to_f16x8(w1.x, h1[0], h1[1], h1[2], h1[3]);
+                e2m1x8_to_f16x8(w1.y, h1[4], h1[5], h1[6], h1[7]);
+                const uint32_t a0 = e4m3_bcast_f16x2(sc0), b0 = e4m3_bcast_f16x2(sc1);
+#pragma unroll
+                for (int i = 0; i < KS; ++i) {
+                    s0[i] = a0;
+                    s1[i] = b0;
+                }
+            }
+            float acc[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
+#pragma unroll
+            for (int i = 0; i < KS; ++i) {
+                const uint32_t ra0 = hmul2(h0[2 * i], s0[i]), ra2 = hmul2(h0[2 * i + 1], s0[i]);
+                const uint32_t ra1 = hmul2(h1[2 * i], s1[i]), ra3 = hmul2(h1[2 * i + 1], s1[i]);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) mma16816(acc[nt], ra0, ra1, ra2, ra3, qf[nt][i][0], qf[nt][i][1]);
+            }
+            // epilogue: ReLU * w, sum over heads, mask, pool
+            const int64_t j0 = kbase + r0, j1 = kbase + r1;
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                float v[2][2];  // [row][col]
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    v[0][e] = fmaxf(acc[nt][e], 0.0f) * wq[nt][e];
+                    v[1][e] = fmaxf(acc[nt][2 + e], 0.0f) * wq[nt][e];
+                }
+                float tsum[2][TPN];
+#pragma unroll
+                for (int rr = 0; rr < 2; ++rr) {
+                    if constexpr (HI == 1) {
+                        tsum[rr][0] = v[rr][0];
+                        tsum[rr][TPN - 1] = v[rr][1];
+                    } else {
+                        float x = v[rr][0] + v[rr][1];
+                        if constexpr (HI >= 4) x += __shfl_xor_sync(0xffffffffu, x, 1);
+                        if constexpr (HI >= 8) x += __shfl_xor_sync(0xffffffffu, x, 2);
+                        tsum[rr][0] = x;
+                    }
+                }
+#pragma unroll
+                for (int e = 0; e < TPN; ++e) {
+                    const int t = token_of<HI>(nt, c, e);
+                    const int64_t pos = (int64_t)L - Tq + t;
+                    const bool vis0 = t < Tq && j0 <= pos, vis1 = t < Tq && j1 <= pos;
+                    const float x0 = vis0 ? tsum[0][e] : 0.0f, x1 = vis1 ? tsum[1][e] : 0.0f;
+                    if (p.pool_mode == 1) {
+                        if (vis0) pool[nt][e] = fmaxf(pool[nt][e], x0);
+                        if (vis1) pool[nt][e] = fmaxf(pool[nt][e], x1);
+                    } else {
+                        pool[nt][e] += x0 + x1;
+                    }
+                    if (token_scores != nullptr && token_owner<HI>(c)) {
+                        float* ts = token_scores + ((int64_t)b * Tq + t) * p.lmax;
+                        if (vis0) ts[j0] = x0 * s_t;
+                        if (vis1) ts[j1] = x1 * s_t;
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+
+        // pool across the 8 row groups and store one score per (token, block)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+            for (int e = 0; e < TPN; ++e) {
+                float x = pool[nt][e];
+#pragma unroll
+                for (int o = 4; o < 32; o <<= 1) {
+                    const float y = __shfl_xor_sync(0xffffffffu, x, o);
+                    x = p.pool_mode == 1 ? fmaxf(x, y) : x + y;
+                }
+                const int t = token_of<HI>(nt, c, e);
+                if (g == 0 && token_owner<HI>(c) && t < Tq) {
+                    const int64_t pos = (int64_t)L - Tq + t;
+                    const int64_t cnt = min64(kBlock, max64(0, pos + 1 - kbase));
+                    float outv = -INFINITY;
+                    if (cnt > 0) outv = p.pool_mode == 1 ? x * s_t : (x / (float)cnt) * s_t;
+                    block_scores[((int64_t)b * Tq + t) * p.nbmax + n] = outv;
+                }
+            }
+        }
+    }
+}
+
+template <int DI, int HI, int NT>
+int launch_t(const Problem& p, float* bs, float* ts, bool pdl, cudaStream_t st) {
+    auto kern = index_decode_kernel<DI, HI, NT>;
+    const size_t smem = idx_smem_bytes<DI>(p.B);
+    static int configured_dev = -1;
+    const DeviceInfo& di = device_info();
+    if (configured_dev != di.device) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)idx_smem_bytes<DI>(kMaxB)) != cudaSuccess)
+            return MSA_ECUDA;
+        configured_dev = di.device;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * di.num_sms));
+    cfg.blockDim = dim3(kIdxThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, p, bs, ts) != cudaSuccess) return MSA_ECUDA;
+    return MSA_OK;
+}
+
+template <int DI, int HI>
+int launch_nt(const Problem& p, float* bs, float* ts, bool pdl, cudaStream_t st) {
+    const int nq = p.Tq * HI;
+    if (nq <= 8) return launch_t<DI, HI, 1>(p, bs, ts, pdl, st);
+    if (nq <= 16) return launch_t<DI, HI, 2>(p, bs, ts, pdl, st);
+    if (nq <= 24) return launch_t<DI, HI, 3>(p, bs, ts, pdl, st);
+    return launch_t<DI, HI, 4>(p, bs, ts, pdl, st);
+}
+
+template <int DI>
+int launch_hi(const Problem& p, float* bs, float* ts, bool pdl, cudaStream_t st) {
+    switch (p.HI) {
+        case 1: return launch_nt<DI, 1>(p, bs, ts, pdl, st);
+        case 2: return launch_nt<DI, 2>(p, bs, ts, pdl, st);
+        case 4: return launch_nt<DI, 4>(p, bs, ts, pdl, st);
+        case 8: return launch_nt<DI, 8>(p, bs, ts, pdl, st);
+        default: return MSA_EUNSUPPORTED;
+    }
+}
+
+}  // namespace
+
+int index_decode_max_batch() { return kMaxB; }
+
+int launch_index_decode(const Problem& p, float* block_scores, float* token_scores, bool pdl, cudaStream_t st) {
+    if (p.B > kMaxB || p.Tq * p.HI > 32) return MSA_EUNSUPPORTED;
+    if (p.DI == 128) return launch_hi<128>(p, block_scores, token_scores, pdl, st);
+    if (p.DI == 64) return launch_hi<64>(p, block_scores, token_scores, pdl, st);
+    return MSA_EUNSUPPORTED;
+}
+
+}  // namespace msa

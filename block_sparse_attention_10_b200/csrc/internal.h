@@ -1,0 +1,58 @@
+// internal.h — launchers and argument blocks shared between the entry points
+// (msa_api.cu) and the kernels.  Not part of the public ABI.
+#pragma once
+
+#include <cstdint>
+
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "msa.h"
+
+namespace msa {
+
+struct DeviceInfo {
+    int device = -1;
+    int num_sms = 0;
+    size_t smem_optin = 0;
+};
+// Cached per current device (queried once per device).
+const DeviceInfo& device_info();
+
+// Kernel-side view of an NVFP4 cache.
+struct Cache {
+    const uint8_t* data;
+    const uint8_t* scale;
+    float s_t;
+};
+
+// Arguments shared by the decode kernels.
+struct Problem {
+    int B, Tq, Hq, Hkv, D, HI, DI;
+    int64_t lmax;
+    int64_t nbmax;  // lmax / 128
+    const int32_t* seq_lens;
+    Cache k, v, ik;
+    const __nv_bfloat16* q;
+    const __nv_bfloat16* q_idx;
+    const float* w_idx;
+    float softmax_scale;
+    int pool_mode;
+    uint32_t* status;
+};
+
+int launch_nvfp4_encode(const float* x, int64_t nvec, int dim, float s_t, uint8_t* data, uint8_t* scale,
+                        cudaStream_t st);
+int launch_nvfp4_decode(const uint8_t* data, const uint8_t* scale, int64_t nvec, int dim, float s_t, float* out,
+                        cudaStream_t st);
+int launch_nvfp4_amax(const float* x, int64_t n, float* amax_out, cudaStream_t st);
+
+// Indexer + pooling over every visible key (decode: Tq * HI <= 32).
+int launch_index_decode(const Problem& p, float* block_scores, float* token_scores, bool pdl, cudaStream_t st);
+// Top-16 selection, recent block forced.
+int launch_select(const Problem& p, const float* block_scores, int32_t* sel, int32_t* sel_copy, bool pdl,
+                  cudaStream_t st);
+// Sparse attention over the selected blocks.
+int launch_attend(const Problem& p, const int32_t* sel, float* out, float* lse, bool pdl, cudaStream_t st);
+
+}  // namespace msa

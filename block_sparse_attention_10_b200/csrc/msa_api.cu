@@ -1,0 +1,192 @@
+// msa_api.cu — the C ABI of libmsa.so (see include/msa.h): host-side argument
+// checks, then the kernel launches.  No allocation, no host synchronisation.
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "internal.h"
+
+namespace msa {
+
+const DeviceInfo& device_info() {
+    static thread_local DeviceInfo cache[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+    DeviceInfo& di = cache[dev];
+    if (di.device != dev) {
+        cudaDeviceProp prop;
+        if (cudaGetDeviceProperties(&prop, dev) == cudaSuccess) {
+            di.num_sms = prop.multiProcessorCount;
+            di.smem_optin = prop.sharedMemPerBlockOptin;
+        } else {
+            di.num_sms = 148;
+            di.smem_optin = 227 * 1024;
+        }
+        di.device = dev;
+    }
+    return di;
+}
+
+namespace {
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+bool good_scale(float s) { return std::isfinite(s) && s > 0.0f; }
+
+int check_cache(const msa_nvfp4_cache_t& c) {
+    if (!c.data || !c.scale) return MSA_EINVAL;
+    if (!good_scale(c.tensor_scale)) return MSA_EINVAL;
+    if (!aligned16(c.data) || !aligned16(c.scale)) return MSA_EALIGN;
+    return MSA_OK;
+}
+
+bool is_pow2_le8(int x) { return x == 1 || x == 2 || x == 4 || x == 8; }
+
+// Checks shared by the MSA steps; `need_*` selects which inputs the step reads.
+int check_params(const msa_params_t* p, bool need_index, bool need_attend) {
+    if (!p) return MSA_EINVAL;
+    if (p->B <= 0 || p->Tq <= 0 || p->lmax <= 0 || !p->seq_lens) return MSA_EINVAL;
+    if (p->lmax % MSA_BLOCK_TOKENS != 0) return MSA_EINVAL;
+    if (p->lmax > (int64_t(1) << 31)) return MSA_EUNSUPPORTED;
+    if (p->Tq > p->lmax) return MSA_EINVAL;
+    if (p->pool_mode != 0 && p->pool_mode != 1) return MSA_EINVAL;
+    if (need_index) {
+        if (p->HI <= 0 || p->DI <= 0 || !p->q_idx) return MSA_EINVAL;
+        if (int r = check_cache(p->ik)) return r;
+        if (!aligned16(p->q_idx)) return MSA_EALIGN;
+        if (p->DI != 64 && p->DI != 128) return MSA_EUNSUPPORTED;
+        if (!is_pow2_le8(p->HI)) return MSA_EUNSUPPORTED;
+        if ((int64_t)p->Tq * p->HI > 32) return MSA_EUNSUPPORTED;
+        if (p->B > 4096) return MSA_EUNSUPPORTED;
+    }
+    if (need_attend) {
+        if (p->Hq <= 0 || p->Hkv <= 0 || p->D <= 0 || !p->q) return MSA_EINVAL;
+        if (p->Hq % p->Hkv != 0) return MSA_EINVAL;
+        if (int r = check_cache(p->k)) return r;
+        if (int r = check_cache(p->v)) return r;
+        if (!aligned16(p->q)) return MSA_EALIGN;
+        if (p->D != 128) return MSA_EUNSUPPORTED;
+        if (!is_pow2_le8(p->Hq / p->Hkv)) return MSA_EUNSUPPORTED;
+        if (!(std::isfinite(p->softmax_scale) && p->softmax_scale >= 0.0f)) return MSA_EINVAL;
+    }
+    return MSA_OK;
+}
+
+Problem to_problem(const msa_params_t* p) {
+    Problem q;
+    q.B = p->B;
+    q.Tq = p->Tq;
+    q.Hq = p->Hq;
+    q.Hkv = p->Hkv;
+    q.D = p->D;
+    q.HI = p->HI;
+    q.DI = p->DI;
+    q.lmax = p->lmax;
+    q.nbmax = p->lmax / MSA_BLOCK_TOKENS;
+    q.seq_lens = p->seq_lens;
+    q.k = Cache{p->k.data, p->k.scale, p->k.tensor_scale};
+    q.v = Cache{p->v.data, p->v.scale, p->v.tensor_scale};
+    q.ik = Cache{p->ik.data, p->ik.scale, p->ik.tensor_scale};
+    q.q = static_cast<const __nv_bfloat16*>(p->q);
+    q.q_idx = static_cast<const __nv_bfloat16*>(p->q_idx);
+    q.w_idx = p->w_idx;
+    q.softmax_scale = p->softmax_scale > 0.0f ? p->softmax_scale : 1.0f / sqrtf((float)p->D);
+    q.pool_mode = p->pool_mode;
+    q.status = p->status;
+    return q;
+}
+
+constexpr size_t kAlign = 256;
+size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+size_t ws_block_scores_bytes(const msa_params_t* p) {
+    return round_up((size_t)p->B * p->Tq * (size_t)(p->lmax / MSA_BLOCK_TOKENS) * sizeof(float));
+}
+size_t ws_sel_bytes(const msa_params_t* p) {
+    return round_up((size_t)p->B * p->Tq * MSA_TOPK_BLOCKS * sizeof(int32_t));
+}
+
+}  // namespace
+}  // namespace msa
+
+using namespace msa;
+
+extern "C" {
+
+const char* msa_status_string(int code) {
+    switch (code) {
+        case MSA_OK: return "MSA_OK";
+        case MSA_EINVAL: return "MSA_EINVAL: invalid argument";
+        case MSA_EUNSUPPORTED: return "MSA_EUNSUPPORTED: shape not supported by the kernels";
+        case MSA_EALIGN: return "MSA_EALIGN: pointer not 16-byte aligned";
+        case MSA_EWORKSPACE: return "MSA_EWORKSPACE: workspace missing or too small";
+        case MSA_ECUDA: return "MSA_ECUDA: CUDA launch error";
+        default: return "MSA: unknown status";
+    }
+}
+
+const char* msa_version(void) { return "libmsa 0.1 (sm_100a)"; }
+
+int msa_nvfp4_encode(const float* x, int64_t nvec, int dim, float tensor_scale, uint8_t* data, uint8_t* scale,
+                     cudaStream_t stream) {
+    if (nvec < 0 || dim <= 0 || dim % 16 != 0) return MSA_EINVAL;
+    if (nvec == 0) return MSA_OK;
+    if (!x || !data || !scale || !good_scale(tensor_scale)) return MSA_EINVAL;
+    if (!aligned16(x) || !aligned16(data)) return MSA_EALIGN;
+    return launch_nvfp4_encode(x, nvec, dim, tensor_scale, data, scale, stream);
+}
+
+int msa_nvfp4_decode(const uint8_t* data, const uint8_t* scale, int64_t nvec, int dim, float tensor_scale,
+                     float* out, cudaStream_t stream) {
+    if (nvec < 0 || dim <= 0 || dim % 16 != 0) return MSA_EINVAL;
+    if (nvec == 0) return MSA_OK;
+    if (!out || !data || !scale || !good_scale(tensor_scale)) return MSA_EINVAL;
+    if (!aligned16(out) || !aligned16(data)) return MSA_EALIGN;
+    return launch_nvfp4_decode(data, scale, nvec, dim, tensor_scale, out, stream);
+}
+
+int msa_nvfp4_amax(const float* x, int64_t n, float* amax_out, cudaStream_t stream) {
+    if (n < 0 || !amax_out || (n > 0 && !x)) return MSA_EINVAL;
+    return launch_nvfp4_amax(x, n, amax_out, stream);
+}
+
+size_t msa_workspace_size(const msa_params_t* p) {
+    if (check_params(p, true, true) != MSA_OK) return 0;
+    return ws_block_scores_bytes(p) + ws_sel_bytes(p);
+}
+
+int msa_index(const msa_params_t* p, float* block_scores, float* token_scores, cudaStream_t stream) {
+    if (int r = check_params(p, true, false)) return r;
+    if (!block_scores) return MSA_EINVAL;
+    return launch_index_decode(to_problem(p), block_scores, token_scores, false, stream);
+}
+
+int msa_select(const msa_params_t* p, const float* block_scores, int32_t* sel, cudaStream_t stream) {
+    if (int r = check_params(p, false, false)) return r;
+    if (!block_scores || !sel) return MSA_EINVAL;
+    return launch_select(to_problem(p), block_scores, sel, nullptr, false, stream);
+}
+
+int msa_attend(const msa_params_t* p, const int32_t* sel, float* out, float* lse, cudaStream_t stream) {
+    if (int r = check_params(p, false, true)) return r;
+    if (!sel || !out) return MSA_EINVAL;
+    if (!aligned16(out)) return MSA_EALIGN;
+    return launch_attend(to_problem(p), sel, out, lse, false, stream);
+}
+
+int msa_decode(const msa_params_t* p, void* ws, size_t ws_bytes, float* out, float* lse, int32_t* sel_out,
+               cudaStream_t stream) {
+    if (int r = check_params(p, true, true)) return r;
+    if (!out) return MSA_EINVAL;
+    if (!aligned16(out)) return MSA_EALIGN;
+    const size_t need = ws_block_scores_bytes(p) + ws_sel_bytes(p);
+    if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return MSA_EWORKSPACE;
+    float* bs = static_cast<float*>(ws);
+    int32_t* sel = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + ws_block_scores_bytes(p));
+    const Problem q = to_problem(p);
+    if (int r = launch_index_decode(q, bs, nullptr, true, stream)) return r;
+    if (int r = launch_select(q, bs, sel, sel_out, true, stream)) return r;
+    return launch_attend(q, sel, out, lse, true, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,182 @@
+/*
+ * msa.h — C ABI of libmsa.so: MiniMax-Sparse-Attention (MSA) decode over an
+ * NVFP4 KV cache, hand-written CUDA for NVIDIA B200 (sm_100a).
+ *
+ * The method (source: "vLLM Adds Day-0 Support for MiniMax-M3.1-Flash on
+ * NVIDIA and AMD GPUs", ainewsbites.com, section "A model built for efficient
+ * inference"): the KV cache is cut into blocks of 128 tokens; a lightweight
+ * indexer scores every key of the context and the scores are pooled into one
+ * score per block; exact attention then runs over the top 16 blocks only,
+ * the most recent block always kept, so a query sees at most 2,048 keys.
+ * Keys, values and indexer keys are stored as NVFP4 ("vLLM delivers day-0
+ * support for MiniMax-M3.1-Flash", readmex.ai, TL;DR).
+ *
+ * Readings this library fixes where the pages are silent:
+ *   indexer   s_j = sum_h w_h * max(0, q_idx[h] . k_idx[j]); one index key per
+ *             token, shared by the HI indexer heads; w_h = 1 when w_idx = NULL.
+ *   pooling   mean (pool_mode 0) or max (pool_mode 1) of s_j over the block's
+ *             visible tokens; a block with no visible token scores -inf.
+ *   selection the query's own block r = pos div 128, plus the best
+ *             min(15, r) other blocks by (score desc, block index asc);
+ *             written ascending, padded with -1 to 16 entries.
+ *   attention o = softmax(scale * q.K^T) V over the selected keys j <= pos;
+ *             query head h reads KV head h / (Hq / Hkv).
+ *   positions sequence b holds L_b = seq_lens[b] tokens, its Tq query tokens
+ *             last; query t sits at pos = L_b - Tq + t and sees keys 0..pos.
+ *
+ * NVFP4 layout (one cache = two planes + one fp32):
+ *   data  [B][heads][lmax][dim/2]  uint8, E2M1 codes, element 2i in the low
+ *                                   nibble of byte i, element 2i+1 in the high;
+ *   scale [B][heads][lmax][dim/16] uint8, E4M3 (OCP "FN", bias 7, max 448),
+ *                                   one per 16 consecutive elements;
+ *   tensor_scale                    fp32 > 0, one per cache tensor.
+ *   value = fp32(e2m1 * e4m3) * tensor_scale.   9/16 byte per element.
+ *
+ * Conventions for every entry point:
+ *   - pointers are DEVICE pointers owned by the caller (except where stated);
+ *     nothing is allocated, nothing is freed, the host never synchronises;
+ *   - work is enqueued on `stream` (0 = legacy default stream) and is
+ *     asynchronous; results are bitwise identical from run to run;
+ *   - return 0 (MSA_OK) or an msa_status code; argument errors are detected
+ *     on the host before anything is enqueued; MSA_ECUDA reports a launch error;
+ *   - values that live on the device (seq_lens, selected block ids) cannot be
+ *     checked on the host: kernels clamp or skip them and set a bit in the
+ *     optional device status word (msa_params_t.status).
+ */
+#ifndef MSA_H
+#define MSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MSA_BLOCK_TOKENS 128 /* tokens per MSA block */
+#define MSA_TOPK_BLOCKS 16   /* blocks attended per query */
+
+typedef enum msa_status {
+    MSA_OK = 0,
+    MSA_EINVAL = 1,       /* null pointer, non-positive size, bad tensor scale, lmax % 128 != 0 */
+    MSA_EUNSUPPORTED = 2, /* shape outside what the kernels are built for (see msa_params_t) */
+    MSA_EALIGN = 3,       /* a pointer is not 16-byte aligned */
+    MSA_EWORKSPACE = 4,   /* workspace too small or NULL */
+    MSA_ECUDA = 5         /* the CUDA runtime reported an error when launching */
+} msa_status;
+
+/* Bits of the optional device status word. */
+#define MSA_STATUS_SEQLEN 1u   /* some seq_lens[b] < Tq or > lmax: clamped */
+#define MSA_STATUS_SELECT 2u   /* a selected block id >= the visible block count: skipped */
+#define MSA_STATUS_TIMEOUT 4u  /* a bounded wait inside a kernel gave up (results invalid) */
+
+/* One NVFP4 cache tensor (K, V or index-K); the layout is given above. */
+typedef struct msa_nvfp4_cache {
+    const uint8_t* data;  /* [B][heads][lmax][dim/2], 16-byte aligned */
+    const uint8_t* scale; /* [B][heads][lmax][dim/16], 16-byte aligned */
+    float tensor_scale;   /* > 0, finite */
+} msa_nvfp4_cache_t;
+
+/*
+ * Problem description shared by every MSA entry point.
+ *   B, Tq     sequences and query tokens per sequence (Tq >= 1)
+ *   Hq, Hkv   attention query / KV heads; Hq / Hkv in {1, 2, 4, 8}
+ *   D         attention head dim; 128
+ *   HI, DI    indexer heads / dim; HI in {1, 2, 4, 8}, DI in {64, 128},
+ *             Tq * HI <= 32 (decode indexer)
+ *   lmax      cache capacity in tokens, a multiple of 128
+ *   seq_lens  device int32 [B], Tq <= L_b <= lmax
+ *   k, v      caches with Hkv heads of dim D; ik: 1 head of dim DI
+ *   q         device bf16 [B][Tq][Hq][D]; q_idx: bf16 [B][Tq][HI][DI].  The
+ *             kernels use queries as fp16: |q| must stay below 65504, and bf16
+ *             values below 2^-14 in magnitude keep 11 significant bits at most
+ *   w_idx     device fp32 [B][Tq][HI] indexer head weights, or NULL (all 1)
+ *   softmax_scale  0 means 1/sqrt(D)
+ *   pool_mode 0 = mean, 1 = max
+ *   status    device uint32 status word (bits MSA_STATUS_*), or NULL; kernels
+ *             only OR bits into it, the caller clears it
+ */
+typedef struct msa_params {
+    int B, Tq, Hq, Hkv, D, HI, DI;
+    int64_t lmax;
+    const int32_t* seq_lens;
+    msa_nvfp4_cache_t k, v, ik;
+    const void* q;
+    const void* q_idx;
+    const float* w_idx;
+    float softmax_scale;
+    int pool_mode;
+    uint32_t* status;
+} msa_params_t;
+
+/* Human-readable name of an msa_status code (static string, never NULL). */
+const char* msa_status_string(int code);
+
+/* Number of SMs etc. are queried once per device; this returns the library
+ * build identification (static string). */
+const char* msa_version(void);
+
+/* ---------------------------------------------------------------------------
+ * NVFP4 codec (the format of the readmex.ai TL;DR, "NVFP4 KV cache for both
+ * the indexer and the attention path"; layout as above).
+ * ------------------------------------------------------------------------- */
+
+/* Quantise x (fp32 [nvec][dim], dim % 16 == 0) into NVFP4 planes:
+ * per 16 elements s = E4M3_rne_sat(amax / fp32(6 * tensor_scale)),
+ * code_i = E2M1_rne_sat(x_i / fp32(s * tensor_scale)) (all codes 0 when that
+ * denominator is 0).  Inputs must be finite.  This is the cache write
+ * ("KV-insert") that precedes the MSA path. */
+int msa_nvfp4_encode(const float* x, int64_t nvec, int dim, float tensor_scale,
+                     uint8_t* data, uint8_t* scale, cudaStream_t stream);
+
+/* Dequantise NVFP4 planes into fp32 [nvec][dim]: fp32(e2m1 * e4m3) * tensor_scale. */
+int msa_nvfp4_decode(const uint8_t* data, const uint8_t* scale, int64_t nvec, int dim,
+                     float tensor_scale, float* out, cudaStream_t stream);
+
+/* amax = max |x_i| over n fp32 values, written to *amax_out (device fp32).
+ * A tensor scale for msa_nvfp4_encode is amax / (6 * 448). */
+int msa_nvfp4_amax(const float* x, int64_t n, float* amax_out, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * MSA steps ("A model built for efficient inference", ainewsbites.com)
+ * ------------------------------------------------------------------------- */
+
+/* Bytes of scratch msa_decode needs for this problem (0 on invalid params). */
+size_t msa_workspace_size(const msa_params_t* p);
+
+/* Indexer + block pooling: streams every visible NVFP4 index key once.
+ *   block_scores  fp32 [B][Tq][ceil(lmax/128)]: pooled score of each block,
+ *                 -inf for blocks with no visible key
+ *   token_scores  fp32 [B][Tq][lmax] or NULL: s_j for every visible key j
+ *                 (entries of invisible keys are left untouched) */
+int msa_index(const msa_params_t* p, float* block_scores, float* token_scores,
+              cudaStream_t stream);
+
+/* Top-16 block selection with the recent block forced:
+ *   block_scores  fp32 [B][Tq][ceil(lmax/128)] as written by msa_index
+ *   sel           int32 [B][Tq][16]: selected block ids ascending, -1 padded */
+int msa_select(const msa_params_t* p, const float* block_scores, int32_t* sel,
+               cudaStream_t stream);
+
+/* Exact softmax attention over the selected blocks (split over the blocks,
+ * combined in on-chip memory):
+ *   sel  int32 [B][Tq][16] (ids < 0 are skipped)
+ *   out  fp32 [B][Tq][Hq][D]; lse fp32 [B][Tq][Hq] (natural log of the
+ *        softmax denominator of the scaled scores) or NULL */
+int msa_attend(const msa_params_t* p, const int32_t* sel, float* out, float* lse,
+               cudaStream_t stream);
+
+/* The whole MSA decode step: msa_index -> msa_select -> msa_attend.
+ *   ws, ws_bytes  device scratch of at least msa_workspace_size(p) bytes,
+ *                 256-byte aligned; contents on entry are ignored
+ *   out, lse      as for msa_attend
+ *   sel_out       int32 [B][Tq][16] copy of the selection, or NULL */
+int msa_decode(const msa_params_t* p, void* ws, size_t ws_bytes, float* out, float* lse,
+               int32_t* sel_out, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MSA_H */

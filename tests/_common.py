@@ -40,3 +40,53 @@ def oracle_decode_inputs(inp, pool_mode=0):
     res = oracle.decode(bf16_values(inp.q), bf16_values(inp.q_idx), k, v, ik, inp.seq_lens, w, pool_mode)
     res["caches"] = (k, v, ik)
     return res
+
+
+# ----------------------------------------------------------------------------- parity helpers
+
+SEL_EXEMPT_REL = 1e-4     # selection: blocks within 1e-4 relative of the cutoff are exempt
+ATT_MAX_ABS = 5e-3        # attention: max-abs vs the oracle
+ATT_REL_L2 = 1e-3         # attention: relative L2 vs the oracle
+
+
+def check_selection(gpu_sel, ora_sel, ora_scores, seq_lens, Tq):
+    """GPU selection == oracle selection except for blocks whose oracle pooled score lies
+    within SEL_EXEMPT_REL (relative) of the cutoff (lowest selected non-forced oracle score).
+    Returns the number of exempted differences."""
+    gpu_sel = np.asarray(gpu_sel)
+    ora_sel = np.asarray(ora_sel)
+    B = gpu_sel.shape[0]
+    exempt = 0
+    for b in range(B):
+        for t in range(Tq):
+            pos = seq_lens[b] - Tq + t
+            r = pos // 128
+            nvis = r + 1
+            gs = [int(x) for x in gpu_sel[b, t] if x >= 0]
+            os_ = [int(x) for x in ora_sel[b, t] if x >= 0]
+            assert gs == sorted(gs) and len(set(gs)) == len(gs), (b, t, gs)
+            assert r in gs, (b, t, "recent block missing")
+            assert len(gs) == min(16, nvis), (b, t, len(gs))
+            assert all(0 <= x < nvis for x in gs)
+            assert list(gpu_sel[b, t, len(gs):]) == [-1] * (16 - len(gs))
+            diff = set(gs) ^ set(os_)
+            if not diff:
+                continue
+            s = ora_scores[b, t]
+            others = [x for x in os_ if x != r]
+            cut = min(s[x] for x in others)
+            for n in diff:
+                assert abs(s[n] - cut) <= SEL_EXEMPT_REL * abs(cut), (b, t, n, s[n], cut)
+                exempt += 1
+    return exempt
+
+
+def check_attention(gpu_out, ora_out):
+    g = np.asarray(gpu_out, dtype=np.float64)
+    o = np.asarray(ora_out, dtype=np.float64)
+    assert np.isfinite(g).all()
+    max_abs = np.abs(g - o).max()
+    rel = np.linalg.norm(g - o) / max(np.linalg.norm(o), 1e-30)
+    assert max_abs <= ATT_MAX_ABS, max_abs
+    assert rel <= ATT_REL_L2, rel
+    return max_abs, rel

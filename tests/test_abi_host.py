@@ -1,0 +1,95 @@
+"""The C ABI without a GPU: the library loads, exports every function include/msa.h
+declares, and rejects bad arguments on the host before anything is enqueued."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_sparse_attention_10_b200 import build, msa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    build.build()
+    return msa.lib()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "msa.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w]+\**\s+\**(msa_\w+)\s*\(", src, re.M)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = _declared()
+    assert "msa_decode" in names and "msa_nvfp4_encode" in names
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(msa.EXPORTS)
+
+
+def test_status_strings(L):
+    for code in range(6):
+        assert msa.status_string(code).startswith("MSA_")
+    assert "unknown" in msa.status_string(99)
+
+
+def _params(**kw):
+    base = dict(B=2, Tq=1, Hq=8, Hkv=1, D=128, HI=4, DI=64, lmax=4096, seq_lens=0x1000,
+                k=msa._Cache(0x2000, 0x3000, 0.01), v=msa._Cache(0x4000, 0x5000, 0.01),
+                ik=msa._Cache(0x6000, 0x7000, 0.01), q=0x8000, q_idx=0x9000, w_idx=None,
+                softmax_scale=0.0, pool_mode=0, status=None)
+    base.update(kw)
+    return msa._Params(**base)
+
+
+def test_workspace_size_host_only(L):
+    p = _params()
+    n = L.msa_workspace_size(ctypes.byref(p))
+    nb = 4096 // 128
+    assert n == ((2 * 1 * nb * 4 + 255) // 256) * 256 + ((2 * 16 * 4 + 255) // 256) * 256
+    assert L.msa_workspace_size(None) == 0
+    bad = _params(lmax=4000)
+    assert L.msa_workspace_size(ctypes.byref(bad)) == 0
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("lmax", 4000, 1), ("B", 0, 1), ("Tq", 0, 1), ("seq_lens", None, 1), ("pool_mode", 2, 1),
+    ("D", 64, 2), ("DI", 96, 2), ("HI", 3, 2), ("Hq", 24, 2), ("Tq", 9, 2),
+    ("q", 0x8001, 3), ("q_idx", 0x9008, 3),
+])
+def test_decode_rejects_bad_params(L, field, value, code):
+    p = _params(**{field: value})
+    ws = ctypes.c_void_p(0x10000)
+    r = L.msa_decode(ctypes.byref(p), ws, 1 << 20, ctypes.c_void_p(0x20000), None, None, None)
+    assert r == code, (field, r)
+
+
+def test_bad_cache_and_workspace(L):
+    p = _params(k=msa._Cache(0x2000, 0x3000, 0.0))
+    assert L.msa_decode(ctypes.byref(p), ctypes.c_void_p(0x10000), 1 << 20, ctypes.c_void_p(0x20000), None, None,
+                        None) == 1
+    p = _params(v=msa._Cache(0x4004, 0x5000, 0.01))
+    assert L.msa_attend(ctypes.byref(p), ctypes.c_void_p(0x100), ctypes.c_void_p(0x200), None, None) == 3
+    p = _params()
+    assert L.msa_decode(ctypes.byref(p), ctypes.c_void_p(0x10000), 16, ctypes.c_void_p(0x20000), None, None,
+                        None) == 4
+    assert L.msa_decode(ctypes.byref(p), None, 1 << 20, ctypes.c_void_p(0x20000), None, None, None) == 4
+    assert L.msa_decode(ctypes.byref(p), ctypes.c_void_p(0x10010), 1 << 20, ctypes.c_void_p(0x20000), None, None,
+                        None) == 4
+    assert L.msa_index(ctypes.byref(p), None, None, None) == 1
+    assert L.msa_select(ctypes.byref(p), None, None, None) == 1
+
+
+def test_codec_rejects_bad_args(L):
+    assert L.msa_nvfp4_encode(ctypes.c_void_p(0x100), 4, 24, ctypes.c_float(1.0), ctypes.c_void_p(0x200),
+                              ctypes.c_void_p(0x300), None) == 1
+    assert L.msa_nvfp4_encode(ctypes.c_void_p(0x100), 4, 32, ctypes.c_float(-1.0), ctypes.c_void_p(0x200),
+                              ctypes.c_void_p(0x300), None) == 1
+    assert L.msa_nvfp4_encode(ctypes.c_void_p(0x104), 4, 32, ctypes.c_float(1.0), ctypes.c_void_p(0x200),
+                              ctypes.c_void_p(0x300), None) == 3
+    assert L.msa_nvfp4_encode(None, 0, 32, ctypes.c_float(1.0), None, None, None) == 0  # empty: no-op
+    assert L.msa_nvfp4_decode(ctypes.c_void_p(0x100), ctypes.c_void_p(0x100), 4, 32, ctypes.c_float(1.0), None,
+                              None) == 1
