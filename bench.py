@@ -1,0 +1,433 @@
+#!/usr/bin/env python3
+"""MSA decode benchmark: query-tokens/s per layer and achieved HBM GB/s on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload (one GPU): 32 sequences x 64K-token context, 1 query token each,
+GQA 32 query / 4 KV heads, head dim 128, indexer 8 heads x 128, NVFP4 K/V and
+index keys (synthetic N(0,1) with 8 needle blocks per sequence), bf16 queries,
+top-16 blocks of 128 tokens with the recent block forced.  A step is one
+msa_decode call (indexer -> select -> attention) over the whole batch.
+
+Timed region: K steps replayed from a CUDA graph on one stream, CUDA events,
+barrier + synchronize on both sides; two replicas of the caches alternate
+(each step reads ~189 MB, more than the 126 MB L2, and the caches themselves
+are 1.36 GB per replica).  Multi-GPU (torchrun): every rank runs its own 32
+sequences (weak scaling, no data-path collective); the time is the max over
+ranks.  ``--impl reference`` times the CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from block_sparse_attention_10_b200 import configs, synth  # noqa: E402
+
+WORKLOAD = configs.DECODE_B32_64K
+METRIC = "MSA decode query-tokens/s per layer; achieved HBM GB/s vs 8 TB/s roofline"
+UNIT = "query-tokens/s"
+CONTRACT_HBM_GBS = 8000.0
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def _algorithmic_bytes(w, seq_lens):
+    """Per step: every visible index key once (DI/2 + DI/16 bytes) + K and V (2 x (D/2 + D/16)
+    bytes per KV head) of the keys in the <= 16 selected blocks (Tq = 1: the forced last block
+    holds L - 128 (NB - 1) keys, the 15 others are full)."""
+    idx = sum(seq_lens) * (w.DI // 2 + w.DI // 16)
+    kv_per_key = 2 * (w.D // 2 + w.D // 16)
+    att = 0
+    for L in seq_lens:
+        nb = (L + 127) // 128
+        keys = L if nb <= 16 else 15 * 128 + (L - 128 * (nb - 1))
+        att += keys * kv_per_key * w.Hkv
+    return idx, att
+
+
+def _measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def _profile_traffic(kernel_file, workload_name):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel source is unchanged."""
+    src = os.path.join(ROOT, "block_sparse_attention_10_b200", "csrc", kernel_file)
+    prof = os.path.join(ROOT, "profiles", f"index_decode_{workload_name}.md")
+    if not (os.path.exists(src) and os.path.exists(prof)):
+        return None
+    digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    vals = {}
+    for line in open(prof):
+        if ":" in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    if vals.get("source_sha256_16") != digest:
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+    def __init__(self, index, period=0.002):
+        self.index, self.period = index, period
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        except Exception as e:  # pragma: no cover - no NVML
+            self.err = str(e)
+        return self
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and bit != 0x1:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t:
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def build_problem(w, batch_ids, seed_offset, device):
+    """GPU-resident NVFP4 caches (encoded by the library) + queries for `batch_ids`."""
+    from block_sparse_attention_10_b200 import msa
+    ww = synth.Workload(**{**w.__dict__, "seed": w.seed + seed_offset})
+    inp = synth.make_inputs(ww, batch_ids=batch_ids, device=device)
+    k = msa.encode_cache(inp.k, inp.s_k)
+    v = msa.encode_cache(inp.v, inp.s_v)
+    ik = msa.encode_cache(inp.ik, inp.s_ik)
+    torch.cuda.synchronize()
+    p = msa.MsaProblem(seq_lens=torch.tensor(inp.seq_lens, dtype=torch.int32, device=device), k=k, v=v, ik=ik,
+                       q=inp.q.contiguous(), q_idx=inp.q_idx.contiguous(), w_idx=None,
+                       status=torch.zeros(1, dtype=torch.int32, device=device))
+    del inp
+    return p
+
+
+def clone_problem(p):
+    from block_sparse_attention_10_b200 import msa
+    c = lambda x: msa.Nvfp4Cache(x.data.clone(), x.scale.clone(), x.tensor_scale)  # noqa: E731
+    return msa.MsaProblem(seq_lens=p.seq_lens.clone(), k=c(p.k), v=c(p.v), ik=c(p.ik), q=p.q.clone(),
+                          q_idx=p.q_idx.clone(), w_idx=None, status=p.status)
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def oracle_sample(w, n_seq, seed_offset=0, device="cuda", key_frac=1.0, heads=None):
+    """Host inputs for the oracle: fp32 values from the same generator (evaluated on the GPU,
+    identical bits by construction), NVFP4-encoded by the oracle's own encoder."""
+    import oracle
+    ww = synth.Workload(**{**w.__dict__, "seed": w.seed + seed_offset})
+    out = []
+    for b in range(n_seq):
+        inp = synth.make_inputs(ww, batch_ids=[b], device=device if torch.cuda.is_available() else "cpu")
+        L = inp.seq_lens[0]
+        Ls = max(128, int(L * key_frac)) if key_frac < 1.0 else L
+        k = oracle.nvfp4_encode(inp.k[:, :, :Ls].cpu().numpy(), inp.s_k)
+        v = oracle.nvfp4_encode(inp.v[:, :, :Ls].cpu().numpy(), inp.s_v)
+        ik = oracle.nvfp4_encode(inp.ik[:, :, :Ls].cpu().numpy(), inp.s_ik)
+        q = inp.q.float().cpu().numpy()
+        qi = inp.q_idx.float().cpu().numpy()
+        if heads is not None:
+            q = np.ascontiguousarray(q[:, :, :heads])
+            g = w.Hq // w.Hkv
+            kvh = max(1, heads // g)
+            k = oracle.Nvfp4(k.data[:, :kvh], k.scale[:, :kvh], k.tensor_scale)
+            v = oracle.Nvfp4(v.data[:, :kvh], v.scale[:, :kvh], v.tensor_scale)
+        out.append((q, qi, k, v, ik, [Ls]))
+        del inp
+    return out
+
+
+def time_oracle(samples):
+    import oracle
+    t0 = time.perf_counter()
+    for q, qi, k, v, ik, lens in samples:
+        oracle.decode(q, qi, k, v, ik, lens)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(w, n_seq=16):
+    import oracle
+    oracle.build()
+    # 16 sequences at a time is about 10-15 s of CPU work: all 8 indexer heads over
+    # 64K keys per sequence plus attention of 32 heads over 2,048 keys
+    samples = oracle_sample(w, n_seq)
+    # the oracle parallelises over (sequence, token[, head]): run all sampled sequences in one call
+    import oracle as O
+    qs = np.concatenate([s[0] for s in samples])
+    qis = np.concatenate([s[1] for s in samples])
+    cat = lambda i: O.Nvfp4(np.concatenate([s[i].data for s in samples]),  # noqa: E731
+                            np.concatenate([s[i].scale for s in samples]), samples[0][i].tensor_scale)
+    k, v, ik = cat(2), cat(3), cat(4)
+    lens = [s[5][0] for s in samples]
+    t0 = time.perf_counter()
+    O.decode(qs, qis, k, v, ik, lens)
+    dt = time.perf_counter() - t0
+    return {"value": n_seq * w.Tq / dt, "unit": UNIT, "cores": O.num_threads(), "kind": "oracle",
+            "sample": f"{n_seq} of the 32 sequences (full 64K context, 1 query token each), "
+                      f"oracle decode (index, pool, select, attend) in one call, {dt:.2f} s wall"}
+
+
+def run_reference(args):
+    ws, rank, _ = _dist()
+    if ws > 1 and rank != 0:
+        return
+    import oracle
+    oracle.build()
+    w = WORKLOAD
+    # per-step sample: one query token of one sequence; if K+W full tokens would not fit in
+    # about 150 s, each step takes the same fraction of one token's work (context prefix of
+    # that fraction for the indexer, that fraction of the query heads for attention)
+    probe = oracle_sample(w, 1)
+    t1 = time_oracle(probe)
+    total = args.steps + args.warmup
+    frac = min(1.0, 150.0 / max(1e-9, total * t1))
+    heads = None
+    if frac < 1.0:
+        heads = max(w.Hq // w.Hkv, int(round(w.Hq * frac)) // (w.Hq // w.Hkv) * (w.Hq // w.Hkv))
+        samples = oracle_sample(w, 1, key_frac=frac, heads=heads)
+    else:
+        samples = probe
+    for _ in range(args.warmup):
+        time_oracle(samples)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        time_oracle(samples)
+    dt = time.perf_counter() - t0
+    value = args.steps * frac / dt
+    sample = ("one query token of sequence 0 per step (full 64K context, 32 heads)" if frac >= 1.0 else
+              f"per step {frac:.4f} of one query token's work: indexer over the first {frac:.4f} of the "
+              f"64K context, attention for {heads} of the 32 query heads; value counts {frac:.4f} token/step")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "global_batch": w.B, "seq_len": w.seq_len, "query_tokens": w.Tq},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def run_ours(args):
+    from block_sparse_attention_10_b200 import msa
+    msa.lib()
+    ws_n, rank, local = _dist()
+    if ws_n > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    w = WORKLOAD
+
+    # each rank owns its own 32 sequences (weak scaling): seed offset by rank
+    p0 = build_problem(w, list(range(w.B)), seed_offset=1000 * rank, device=dev)
+    reps = [p0] + [clone_problem(p0) for _ in range(args.replicas - 1)]
+    ws_t = msa.alloc_workspace(p0)
+    out, lse, sel = msa.outputs(p0)
+    stream = torch.cuda.Stream()
+    torch.cuda.synchronize()
+
+    def step(i, s):
+        msa.msa_decode(reps[i % len(reps)], ws_t, out, lse, None, stream=s)
+
+    with torch.cuda.stream(stream):
+        for i in range(max(3, args.warmup)):
+            step(i, stream)
+    torch.cuda.synchronize()
+    # capture G steps in one graph (launch overhead off the host); replays cover K steps
+    G = math.gcd(args.steps, 50) if args.steps % 50 else 50
+    G = max(1, min(G, args.steps))
+    if args.steps % G:
+        G = 1
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(G):
+            step(i, stream)
+    torch.cuda.synchronize()
+    for _ in range(2):
+        graph.replay()
+    torch.cuda.synchronize()
+    if ws_n > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(args.steps // G):
+                graph.replay()
+            e1.record(stream)
+        e1.synchronize()
+    torch.cuda.synchronize()
+    if ws_n > 1:
+        torch.distributed.barrier()
+    ms = e0.elapsed_time(e1) / args.steps
+    if ws_n > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = t.item()
+    status = int(p0.status.item())
+    assert status == 0, f"device status word {status}"
+
+    # dominant kernel (indexer): per-launch CUDA events on its stream
+    nb_i = min(args.steps, 200)
+    bs = torch.empty(w.B, w.Tq, p0.nbmax, dtype=torch.float32, device=dev)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nb_i)]
+    with torch.cuda.stream(stream):
+        for i in range(5):
+            msa.msa_index(reps[i % len(reps)], bs, None, stream=stream)
+        for i, (a, b) in enumerate(evs):
+            a.record(stream)
+            msa.msa_index(reps[i % len(reps)], bs, None, stream=stream)
+            b.record(stream)
+    torch.cuda.synchronize()
+    idx_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    lens = [int(x) for x in p0.seq_lens.tolist()]
+    idx_bytes, att_bytes = _algorithmic_bytes(w, lens)
+    peak, peak_kind = _measured_peaks()
+    achieved = idx_bytes / (idx_ms * 1e-3) / 1e9
+
+    # end to end through the public API: pinned host queries -> device, decode, output -> host
+    n_e2e = min(args.steps, 200)
+    hq = torch.empty_like(p0.q, device="cpu").pin_memory()
+    hqi = torch.empty_like(p0.q_idx, device="cpu").pin_memory()
+    hq.copy_(p0.q.cpu())
+    hqi.copy_(p0.q_idx.cpu())
+    hout = torch.empty_like(out, device="cpu").pin_memory()
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    with torch.cuda.stream(stream):
+        for i in range(n_e2e):
+            r = reps[i % len(reps)]
+            r.q.copy_(hq, non_blocking=True)
+            r.q_idx.copy_(hqi, non_blocking=True)
+            msa.msa_decode(r, ws_t, out, lse, None, stream=stream)
+            hout.copy_(out, non_blocking=True)
+            stream.synchronize()
+    e2e_s = (time.perf_counter() - t0) / n_e2e
+    h2d = hq.numel() * hq.element_size() + hqi.numel() * hqi.element_size()
+    d2h = hout.numel() * hout.element_size()
+    if ws_n > 1:
+        t = torch.tensor([e2e_s], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_s = t.item()
+
+    cpu = None
+    if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w)
+
+    if rank == 0:
+        tokens = w.B * w.Tq * ws_n
+        value = tokens / (ms * 1e-3)
+        step_bytes = idx_bytes + att_bytes
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws_n, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "nvfp4 caches, f16 tensor-core math, f32 accumulate/output",
+            "data": "synthetic",
+            "config": {"workload": w.name, "global_batch": w.B * ws_n, "seq_len": w.seq_len, "query_tokens": w.Tq,
+                       "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "HI": w.HI, "DI": w.DI, "top_blocks": 16,
+                       "block_tokens": 128, "parallelism": f"replicas x{ws_n} (own sequences per GPU)",
+                       "l2": f"inputs larger than L2: {step_bytes / 1e6:.0f} MB read per step, "
+                             f"{args.replicas} rotating cache replicas of "
+                             f"{(p0.k.data.numel() + p0.k.scale.numel()) * 2 / 1e9 + (p0.ik.data.numel() + p0.ik.scale.numel()) / 1e9:.2f} GB"},
+            "step_gbs": step_bytes / (ms * 1e-3) / 1e9,
+            "step_frac_of_8tbs": step_bytes / (ms * 1e-3) / 1e9 / CONTRACT_HBM_GBS,
+            "roofline": {"kernel": "index_decode", "bound": "hbm", "achieved": achieved, "peak": peak,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                         "frac_of_8tbs": achieved / CONTRACT_HBM_GBS,
+                         "algorithmic_bytes_per_launch": idx_bytes, "launch_ms": idx_ms,
+                         "traffic": _profile_traffic("index_decode.cu", w.name)},
+            "cpu_baseline": cpu,
+            "e2e": {"value": w.B * w.Tq * ws_n / e2e_s, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": 3 * args.steps,
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    del graph
+    if ws_n > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--replicas", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -19,8 +19,11 @@
 // The partial (m, l, O) of the 4 warps are merged in shared memory, then the 4
 // CTAs of the cluster merge through distributed shared memory (each CTA
 // finalises 32 of the 128 dims).  No global scratch, no second launch, a
-// fixed merge order (bitwise deterministic).  K/V tiles are double-buffered
-// in registers (128-bit loads for K, 64-bit for V; both fully coalesced).
+// fixed merge order (bitwise deterministic).  Each warp brings its whole
+// block (K and V nibbles + scales of up to 128 keys, 18 KB) into its own
+// shared-memory stage with four untiled bulk copies (cp.async.bulk, no
+// multicast) on one mbarrier, so every selected byte is requested at kernel
+// start; the math then reads shared memory only.
 #include <cooperative_groups.h>
 
 #include "internal.h"
@@ -37,46 +40,29 @@ constexpr int kD = 128;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-struct KVTile {
-    uint4 k[2];      // keys base+g, base+8+g: bytes [16c, 16c+16) of the key's 64-byte row
-    uint32_t ks[2];  // their E4M3 scales of groups 2c, 2c+1 (16 bits)
-    uint2 v[4];      // keys base+{2c, 2c+1, 2c+8, 2c+9}: bytes [8g, 8g+8) (dims 16g..16g+15)
-    uint32_t vs[4];  // their E4M3 scale of group g
-};
-
-__device__ __forceinline__ void load_tile(KVTile& T, const uint8_t* kd, const uint8_t* ksc, const uint8_t* vd,
-                                          const uint8_t* vsc, int base, int nk, int g, int c) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int key = base + 8 * h + g;
-        if (key < nk) {
-            T.k[h] = ldg_nc_v4(kd + key * 64 + c * 16);
-            T.ks[h] = ldg_nc_u16(ksc + key * 8 + c * 2);
-        } else {
-            T.k[h] = make_uint4(0u, 0u, 0u, 0u);
-            T.ks[h] = 0u;
-        }
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int key = base + 2 * c + (i & 1) + 8 * (i >> 1);
-        if (key < nk) {
-            T.v[i] = ldg_nc_v2(vd + key * 64 + g * 8);
-            T.vs[i] = ldg_nc_u8(vsc + key * 8 + g);
-        } else {
-            T.v[i] = make_uint2(0u, 0u);
-            T.vs[i] = 0u;
-        }
-    }
-}
+// Per-warp shared-memory stage: one 128-key block of one KV head.
+constexpr int kKData = kBlock * 64, kKScale = kBlock * 8;
+constexpr int kStage = 2 * (kKData + kKScale);  // 18 KB
+constexpr size_t kAttSmem = (size_t)kAttWarps * kStage + kAttWarps * sizeof(uint64_t) + 2 * 8 * sizeof(float);
 
 template <int G>
 __global__ void __cluster_dims__(kAttCluster, 1, 1) __launch_bounds__(kAttThreads, 3)
     attend_kernel(const Problem p, const int32_t* __restrict__ sel, float* __restrict__ out,
                   float* __restrict__ lse) {
-    __shared__ __align__(16) float sO[kAttWarps][8][kD];
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kAttWarps * kStage);
+    float* cM = reinterpret_cast<float*>(bars + kAttWarps);
+    float* cL = cM + 8;
     __shared__ float sM[kAttWarps][8], sL[kAttWarps][8];
-    __shared__ float cM[8], cL[8];
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, c = lane & 3;
+    uint8_t* stage = smem + warp * kStage;
+    if (lane == 0) {
+        mbar_init(&bars[warp], 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
 
     pdl_wait();
     pdl_launch_dependents();
@@ -90,10 +76,28 @@ __global__ void __cluster_dims__(kAttCluster, 1, 1) __launch_bounds__(kAttThread
     const int64_t L = clamp_len(p.seq_lens[b], p.Tq, p.lmax, nullptr);
     const int64_t pos = L - p.Tq + t;
     const int64_t nvis = pos / kBlock + 1;
-
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = lane >> 2, c = lane & 3;
     const int gw = crank * kAttWarps + warp;
+
+    // this warp's block: issue its bulk copies first, then read Q while they fly
+    int blk = gw < kTopK ? sel[bt * kTopK + gw] : -1;
+    if (blk >= nvis) {
+        if (lane == 0) set_status(p.status, MSA_STATUS_SELECT);
+        blk = -1;
+    }
+    int nk = 0;
+    if (blk >= 0) {
+        const int64_t kbase = (int64_t)blk * kBlock;
+        nk = (int)min64(kBlock, pos + 1 - kbase);
+        if (lane == 0) {
+            const int rows = (nk + 15) & ~15;
+            const int64_t vec0 = ((int64_t)b * p.Hkv + kvh) * p.lmax + kbase;
+            mbar_arrive_expect_tx(&bars[warp], (uint32_t)(2 * rows * (64 + 8)));
+            bulk_g2s(stage, p.k.data + vec0 * 64, (uint32_t)(rows * 64), &bars[warp]);
+            bulk_g2s(stage + kKData, p.k.scale + vec0 * 8, (uint32_t)(rows * 8), &bars[warp]);
+            bulk_g2s(stage + kKData + kKScale, p.v.data + vec0 * 64, (uint32_t)(rows * 64), &bars[warp]);
+            bulk_g2s(stage + 2 * kKData + kKScale, p.v.scale + vec0 * 8, (uint32_t)(rows * 8), &bars[warp]);
+        }
+    }
 
     // Q rows (query heads kvh*G + g), dims [32c, 32c+32) as 16 f16x2 pairs
     uint32_t qa[8][2];
@@ -118,38 +122,32 @@ __global__ void __cluster_dims__(kAttCluster, 1, 1) __launch_bounds__(kAttThread
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.0f;
 
-    const int32_t* srow = sel + bt * kTopK;
-    for (int si = gw; si < kTopK; si += kAttCluster * kAttWarps) {
-        const int blk = srow[si];
-        if (blk < 0) continue;
-        if (blk >= nvis) {
-            if (lane == 0) set_status(p.status, MSA_STATUS_SELECT);
-            continue;
-        }
-        const int64_t kbase = (int64_t)blk * kBlock;
-        const int nk = (int)min64(kBlock, pos + 1 - kbase);
-        const int64_t vec0 = ((int64_t)b * p.Hkv + kvh) * p.lmax + kbase;
-        const uint8_t* kd = p.k.data + vec0 * 64;
-        const uint8_t* ksc = p.k.scale + vec0 * 8;
-        const uint8_t* vd = p.v.data + vec0 * 64;
-        const uint8_t* vsc = p.v.scale + vec0 * 8;
+    if (blk >= 0 && !mbar_wait(&bars[warp], 0)) {
+        if (lane == 0) set_status(p.status, MSA_STATUS_TIMEOUT);
+        mbar_wait(&bars[warp], 0);  // one more bounded wait for the copies before the stage is reused
+        blk = -1;
+    }
+    if (blk >= 0) {
+        const uint8_t* kd = stage;
+        const uint8_t* ksc = stage + kKData;
+        const uint8_t* vd = stage + kKData + kKScale;
+        const uint8_t* vsc = stage + 2 * kKData + kKScale;
         const int ntiles = (nk + 15) >> 4;
-
-        KVTile cur, nxt;
-        load_tile(cur, kd, ksc, vd, vsc, 0, nk, g, c);
         for (int kt = 0; kt < ntiles; ++kt) {
-            if (kt + 1 < ntiles) load_tile(nxt, kd, ksc, vd, vsc, (kt + 1) * 16, nk, g, c);
             // ---- S = Q K^T over 16 keys (two n-tiles of 8 keys)
             float sacc[2][4];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
+                const int key = kt * 16 + 8 * h + g;
+                const uint4 kw = lds_v4(kd + key * 64 + c * 16);
+                const uint32_t ks = e4m3x2_to_f16x2(lds_u16(ksc + key * 8 + c * 2));
                 sacc[h][0] = sacc[h][1] = sacc[h][2] = sacc[h][3] = 0.0f;
                 uint32_t kh[16];
-                e2m1x8_to_f16x8(cur.k[h].x, kh[0], kh[1], kh[2], kh[3]);
-                e2m1x8_to_f16x8(cur.k[h].y, kh[4], kh[5], kh[6], kh[7]);
-                e2m1x8_to_f16x8(cur.k[h].z, kh[8], kh[9], kh[10], kh[11]);
-                e2m1x8_to_f16x8(cur.k[h].w, kh[12], kh[13], kh[14], kh[15]);
-                const uint32_t slo = e4m3_bcast_f16x2(cur.ks[h]), shi = e4m3_bcast_f16x2(cur.ks[h] >> 8);
+                e2m1x8_to_f16x8(kw.x, kh[0], kh[1], kh[2], kh[3]);
+                e2m1x8_to_f16x8(kw.y, kh[4], kh[5], kh[6], kh[7]);
+                e2m1x8_to_f16x8(kw.z, kh[8], kh[9], kh[10], kh[11]);
+                e2m1x8_to_f16x8(kw.w, kh[12], kh[13], kh[14], kh[15]);
+                const uint32_t slo = prmt(ks, ks, 0x1010u), shi = prmt(ks, ks, 0x3232u);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const uint32_t sc = i < 4 ? slo : shi;
@@ -178,13 +176,20 @@ __global__ void __cluster_dims__(kAttCluster, 1, 1) __launch_bounds__(kAttThread
             const uint32_t pb0 = pack_f16x2(pr[0], pr[1]), pb1 = pack_f16x2(pr[2], pr[3]);
             // rescale O^T columns: this thread holds query rows 2c and 2c+1
             const float c0 = __shfl_sync(0xffffffffu, corr, 8 * c), c1 = __shfl_sync(0xffffffffu, corr, 8 * c + 4);
-            // ---- O^T += V^T P^T
+            // ---- O^T += V^T P^T; V of keys 2c, 2c+1, 2c+8, 2c+9 (masked keys read as 0)
             uint32_t vh[4][8];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                e2m1x8_to_f16x8(cur.v[i].x, vh[i][0], vh[i][1], vh[i][2], vh[i][3]);
-                e2m1x8_to_f16x8(cur.v[i].y, vh[i][4], vh[i][5], vh[i][6], vh[i][7]);
-                const uint32_t sc = e4m3_bcast_f16x2(cur.vs[i]);
+                const int key = kt * 16 + 2 * c + (i & 1) + 8 * (i >> 1);
+                uint2 vw = make_uint2(0u, 0u);
+                uint32_t vs = 0u;
+                if (key < nk) {
+                    vw = lds_v2(vd + key * 64 + g * 8);
+                    vs = lds_u8(vsc + key * 8 + g);
+                }
+                e2m1x8_to_f16x8(vw.x, vh[i][0], vh[i][1], vh[i][2], vh[i][3]);
+                e2m1x8_to_f16x8(vw.y, vh[i][4], vh[i][5], vh[i][6], vh[i][7]);
+                const uint32_t sc = e4m3_bcast_f16x2(vs);
 #pragma unroll
                 for (int m = 0; m < 8; ++m) vh[i][m] = hmul2(vh[i][m], sc);
             }
@@ -200,26 +205,28 @@ __global__ void __cluster_dims__(kAttCluster, 1, 1) __launch_bounds__(kAttThread
                 const uint32_t a3 = prmt(vh[2][mt], vh[3][mt], 0x7632u);
                 mma16816(o[mt], a0, a1, a2, a3, pb0, pb1);
             }
-            cur = nxt;
         }
     }
 
-    // ---- merge the 4 warps of this CTA
+    // ---- merge the 4 warps of this CTA (each warp's partial O goes into its own stage)
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
     l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
     if (c == 0) {
         sM[warp][g] = m_run;
         sL[warp][g] = l_run;
     }
+    __syncwarp();
+    float* sOw = reinterpret_cast<float*>(stage);  // [8][kD]
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) {
         const int d = 16 * g + 2 * mt;
-        sO[warp][2 * c][d] = o[mt][0];
-        sO[warp][2 * c + 1][d] = o[mt][1];
-        sO[warp][2 * c][d + 1] = o[mt][2];
-        sO[warp][2 * c + 1][d + 1] = o[mt][3];
+        sOw[(2 * c) * kD + d] = o[mt][0];
+        sOw[(2 * c + 1) * kD + d] = o[mt][1];
+        sOw[(2 * c) * kD + d + 1] = o[mt][2];
+        sOw[(2 * c + 1) * kD + d + 1] = o[mt][3];
     }
     __syncthreads();
+    float* sO0 = reinterpret_cast<float*>(smem);  // the CTA's merged partial, in warp 0's stage
     {
         const int q = threadIdx.x >> 4, d0 = (threadIdx.x & 15) * 8;
         float M = -INFINITY;
@@ -235,12 +242,14 @@ __global__ void __cluster_dims__(kAttCluster, 1, 1) __launch_bounds__(kAttThread
 #pragma unroll
         for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
 #pragma unroll
-        for (int w = 0; w < kAttWarps; ++w)
+        for (int w = 0; w < kAttWarps; ++w) {
+            const float* src = reinterpret_cast<const float*>(smem + w * kStage) + q * kD + d0;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) acc[j] += f[w] * sO[w][q][d0 + j];
-        // all warps' reads of this (q, d0..d0+7) slice happen in this thread: safe to overwrite
+            for (int j = 0; j < 8; ++j) acc[j] += f[w] * src[j];
+        }
+        // every read of this (q, d0..d0+7) slice happened in this thread: safe to overwrite
 #pragma unroll
-        for (int j = 0; j < 8; ++j) sO[0][q][d0 + j] = acc[j];
+        for (int j = 0; j < 8; ++j) sO0[q * kD + d0 + j] = acc[j];
         if ((threadIdx.x & 15) == 0) {
             cM[q] = M;
             cL[q] = Lc;
@@ -254,9 +263,9 @@ __global__ void __cluster_dims__(kAttCluster, 1, 1) __launch_bounds__(kAttThread
         float Mr[kAttCluster], Lr[kAttCluster], O0[kAttCluster], O1[kAttCluster];
 #pragma unroll
         for (int r = 0; r < kAttCluster; ++r) {
-            const float* pm = cluster.map_shared_rank(&cM[0], r);
-            const float* pl = cluster.map_shared_rank(&cL[0], r);
-            const float* po = cluster.map_shared_rank(&sO[0][0][0], r);
+            const float* pm = cluster.map_shared_rank(cM, r);
+            const float* pl = cluster.map_shared_rank(cL, r);
+            const float* po = cluster.map_shared_rank(sO0, r);
             Mr[r] = pm[q];
             Lr[r] = pl[q];
             const float2 v2 = *reinterpret_cast<const float2*>(po + q * kD + d);
@@ -288,9 +297,18 @@ __global__ void __cluster_dims__(kAttCluster, 1, 1) __launch_bounds__(kAttThread
 template <int G>
 int launch_g(const Problem& p, const int32_t* sel, float* out, float* lse, bool pdl, cudaStream_t st) {
     const int64_t units = (int64_t)p.B * p.Tq * p.Hkv;
+    static int configured_dev = -1;
+    const DeviceInfo& di = device_info();
+    if (configured_dev != di.device) {
+        if (cudaFuncSetAttribute(attend_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttSmem) !=
+            cudaSuccess)
+            return MSA_ECUDA;
+        configured_dev = di.device;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(units * kAttCluster));
     cfg.blockDim = dim3(kAttThreads);
+    cfg.dynamicSmemBytes = kAttSmem;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;

@@ -68,6 +68,61 @@ __device__ __forceinline__ bool token_owner(int c) {
     else return c == 0;
 }
 
+// One 16-key tile: rows r0 and r0 + 8 of the stage, dequantised (E2M1 * E4M3, exact in
+// f16) into A fragments, times the resident query fragments; acc = [NT n-tiles][c0..c3].
+template <int DI, int NT>
+__device__ __forceinline__ void tile_mma(const uint8_t* sd, const uint8_t* ss, int r0, int c,
+                                         const uint32_t (&qf)[NT][DI / 16][2], float (&acc)[NT][4]) {
+    constexpr int KS = DI / 16;
+    const int r1 = r0 + 8;
+    uint32_t h0[2 * KS], h1[2 * KS];
+    uint32_t s0[KS], s1[KS];
+    if constexpr (DI == 128) {
+        const uint4 w0 = lds_v4(sd + r0 * 64 + c * 16);
+        const uint4 w1 = lds_v4(sd + r1 * 64 + c * 16);
+        const uint32_t sc0 = e4m3x2_to_f16x2(lds_u16(ss + r0 * 8 + c * 2));
+        const uint32_t sc1 = e4m3x2_to_f16x2(lds_u16(ss + r1 * 8 + c * 2));
+        e2m1x8_to_f16x8(w0.x, h0[0], h0[1], h0[2], h0[3]);
+        e2m1x8_to_f16x8(w0.y, h0[4], h0[5], h0[6], h0[7]);
+        e2m1x8_to_f16x8(w0.z, h0[8], h0[9], h0[10], h0[11]);
+        e2m1x8_to_f16x8(w0.w, h0[12], h0[13], h0[14], h0[15]);
+        e2m1x8_to_f16x8(w1.x, h1[0], h1[1], h1[2], h1[3]);
+        e2m1x8_to_f16x8(w1.y, h1[4], h1[5], h1[6], h1[7]);
+        e2m1x8_to_f16x8(w1.z, h1[8], h1[9], h1[10], h1[11]);
+        e2m1x8_to_f16x8(w1.w, h1[12], h1[13], h1[14], h1[15]);
+        const uint32_t a0 = prmt(sc0, sc0, 0x1010u), a1 = prmt(sc0, sc0, 0x3232u);
+        const uint32_t b0 = prmt(sc1, sc1, 0x1010u), b1 = prmt(sc1, sc1, 0x3232u);
+#pragma unroll
+        for (int i = 0; i < KS; ++i) {
+            s0[i] = i < 4 ? a0 : a1;
+            s1[i] = i < 4 ? b0 : b1;
+        }
+    } else {
+        const uint2 w0 = lds_v2(sd + r0 * 32 + c * 8);
+        const uint2 w1 = lds_v2(sd + r1 * 32 + c * 8);
+        const uint32_t a0 = e4m3_bcast_f16x2(lds_u8(ss + r0 * 4 + c));
+        const uint32_t b0 = e4m3_bcast_f16x2(lds_u8(ss + r1 * 4 + c));
+        e2m1x8_to_f16x8(w0.x, h0[0], h0[1], h0[2], h0[3]);
+        e2m1x8_to_f16x8(w0.y, h0[4], h0[5], h0[6], h0[7]);
+        e2m1x8_to_f16x8(w1.x, h1[0], h1[1], h1[2], h1[3]);
+        e2m1x8_to_f16x8(w1.y, h1[4], h1[5], h1[6], h1[7]);
+#pragma unroll
+        for (int i = 0; i < KS; ++i) {
+            s0[i] = a0;
+            s1[i] = b0;
+        }
+    }
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
+#pragma unroll
+    for (int i = 0; i < KS; ++i) {
+        const uint32_t ra0 = hmul2(h0[2 * i], s0[i]), ra2 = hmul2(h0[2 * i + 1], s0[i]);
+        const uint32_t ra1 = hmul2(h1[2 * i], s1[i]), ra3 = hmul2(h1[2 * i + 1], s1[i]);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) mma16816(acc[nt], ra0, ra1, ra2, ra3, qf[nt][i][0], qf[nt][i][1]);
+    }
+}
+
 template <int DI, int HI, int NT>
 __global__ void __launch_bounds__(kIdxThreads, 2)
     index_decode_kernel(const Problem p, float* __restrict__ block_scores, float* __restrict__ token_scores) {
@@ -231,6 +286,54 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
 
         const uint8_t* sd = smem + (size_t)s * G::kStageBytes;
         const uint8_t* ss = sd + G::kDataBytes;
+        // fast path: a full block that every query token sees entirely, mean pooling, no
+        // per-token output.  The pooled mean is linear, so ReLU'd products are summed per
+        // accumulator element over all tiles and reduced over heads and rows once per block.
+        const bool fast = valid == kBlock && kbase + (kBlock - 1) <= (int64_t)L - Tq && p.pool_mode == 0 &&
+                          token_scores == nullptr;
+        if (fast) {
+            float colsum[NT][4];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) colsum[nt][0] = colsum[nt][1] = colsum[nt][2] = colsum[nt][3] = 0.0f;
+#pragma unroll 2
+            for (int ti = 0; ti < kBlock / 16; ++ti) {
+                float acc[NT][4];
+                tile_mma<DI, NT>(sd, ss, ti * 16 + g, c, qf, acc);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) colsum[nt][e] += fmaxf(acc[nt][e], 0.0f);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                // rows g and g+8 of the same column, then the head weights
+                float x0 = (colsum[nt][0] + colsum[nt][2]) * wq[nt][0];
+                float x1 = (colsum[nt][1] + colsum[nt][3]) * wq[nt][1];
+                float tsum[TPN];
+                if constexpr (HI == 1) {
+                    tsum[0] = x0;
+                    tsum[TPN - 1] = x1;
+                } else {
+                    float x = x0 + x1;
+                    if constexpr (HI >= 4) x += __shfl_xor_sync(0xffffffffu, x, 1);
+                    if constexpr (HI >= 8) x += __shfl_xor_sync(0xffffffffu, x, 2);
+                    tsum[0] = x;
+                }
+#pragma unroll
+                for (int e = 0; e < TPN; ++e) {
+                    float x = tsum[e];
+#pragma unroll
+                    for (int o = 4; o < 32; o <<= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+                    const int t = token_of<HI>(nt, c, e);
+                    if (g == 0 && token_owner<HI>(c) && t < Tq)
+                        block_scores[((int64_t)b * Tq + t) * p.nbmax + n] = (x * (1.0f / kBlock)) * s_t;
+                }
+            }
+            continue;
+        }
+
         float pool[NT][TPN];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
@@ -240,54 +343,8 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
         const int ntiles = (valid + 15) >> 4;
         for (int ti = 0; ti < ntiles; ++ti) {
             const int r0 = ti * 16 + g, r1 = r0 + 8;
-            uint32_t h0[2 * KS], h1[2 * KS];  // f16x2 pairs of rows r0 / r1 (unscaled E2M1)
-            uint32_t s0[KS], s1[KS];          // per k-step E4M3 scale, broadcast f16x2
-            if constexpr (DI == 128) {
-                const uint4 w0 = lds_v4(sd + r0 * 64 + c * 16);
-                const uint4 w1 = lds_v4(sd + r1 * 64 + c * 16);
-                const uint32_t sc0 = lds_u16(ss + r0 * 8 + c * 2);
-                const uint32_t sc1 = lds_u16(ss + r1 * 8 + c * 2);
-                e2m1x8_to_f16x8(w0.x, h0[0], h0[1], h0[2], h0[3]);
-                e2m1x8_to_f16x8(w0.y, h0[4], h0[5], h0[6], h0[7]);
-                e2m1x8_to_f16x8(w0.z, h0[8], h0[9], h0[10], h0[11]);
-                e2m1x8_to_f16x8(w0.w, h0[12], h0[13], h0[14], h0[15]);
-                e2m1x8_to_f16x8(w1.x, h1[0], h1[1], h1[2], h1[3]);
-                e2m1x8_to_f16x8(w1.y, h1[4], h1[5], h1[6], h1[7]);
-                e2m1x8_to_f16x8(w1.z, h1[8], h1[9], h1[10], h1[11]);
-                e2m1x8_to_f16x8(w1.w, h1[12], h1[13], h1[14], h1[15]);
-                const uint32_t a0 = e4m3_bcast_f16x2(sc0), a1 = e4m3_bcast_f16x2(sc0 >> 8);
-                const uint32_t b0 = e4m3_bcast_f16x2(sc1), b1 = e4m3_bcast_f16x2(sc1 >> 8);
-#pragma unroll
-                for (int i = 0; i < KS; ++i) {
-                    s0[i] = i < 4 ? a0 : a1;
-                    s1[i] = i < 4 ? b0 : b1;
-                }
-            } else {
-                const uint2 w0 = lds_v2(sd + r0 * 32 + c * 8);
-                const uint2 w1 = lds_v2(sd + r1 * 32 + c * 8);
-                const uint32_t sc0 = lds_u8(ss + r0 * 4 + c);
-                const uint32_t sc1 = lds_u8(ss + r1 * 4 + c);
-                e2m1x8_to_f16x8(w0.x, h0[0], h0[1], h0[2], h0[3]);
-                e2m1x8_to_f16x8(w0.y, h0[4], h0[5], h0[6], h0[7]);
-                e2m1x8_to_f16x8(w1.x, h1[0], h1[1], h1[2], h1[3]);
-                e2m1x8_to_f16x8(w1.y, h1[4], h1[5], h1[6], h1[7]);
-                const uint32_t a0 = e4m3_bcast_f16x2(sc0), b0 = e4m3_bcast_f16x2(sc1);
-#pragma unroll
-                for (int i = 0; i < KS; ++i) {
-                    s0[i] = a0;
-                    s1[i] = b0;
-                }
-            }
             float acc[NT][4];
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
-#pragma unroll
-            for (int i = 0; i < KS; ++i) {
-                const uint32_t ra0 = hmul2(h0[2 * i], s0[i]), ra2 = hmul2(h0[2 * i + 1], s0[i]);
-                const uint32_t ra1 = hmul2(h1[2 * i], s1[i]), ra3 = hmul2(h1[2 * i + 1], s1[i]);
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt) mma16816(acc[nt], ra0, ra1, ra2, ra3, qf[nt][i][0], qf[nt][i][1]);
-            }
+            tile_mma<DI, NT>(sd, ss, r0, c, qf, acc);
             // epilogue: ReLU * w, sum over heads, mask, pool
             const int64_t j0 = kbase + r0, j1 = kbase + r1;
 #pragma unroll

@@ -11,7 +11,8 @@
 // (order-preserving bits of the fp32 score, then the inverted block index),
 // so "best" is a plain maximum and ties go to the lower index; 15 rounds of
 // "largest key below the previous winner" with two 32-bit warp reductions
-// (redux.sync) each.  Deterministic and independent of the warp layout.
+// (redux.sync) each.  The first 512 candidates of a row live in registers.
+// Deterministic and independent of the warp layout.
 #include "internal.h"
 
 namespace msa {
@@ -41,14 +42,29 @@ __global__ void __launch_bounds__(32 * kSelWarps)
     const float* s = block_scores + row * p.nbmax;
     const int want = (int)min64(kTopK - 1, nvis - 1);
 
+    // The first 512 candidates stay in registers (16 per lane, loads issued together);
+    // longer rows stream the rest from L1/L2 in chunks of 512 every round.
+    constexpr int kPer = 16;
+    uint64_t k0[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) {
+        const int64_t n = j * 32 + lane;
+        k0[j] = (n < nvis && n != r) ? rank_key(__ldg(s + n), n) : 0ull;
+    }
     uint64_t prev = ~0ull;
     int mine = -1;  // lane i < want holds the i-th best
     for (int k = 0; k < want; ++k) {
         uint64_t best = 0;
-        for (int64_t n = lane; n < nvis; n += 32) {
-            if (n == r) continue;
-            const uint64_t key = rank_key(__ldg(s + n), n);
-            if (key < prev && key > best) best = key;
+#pragma unroll
+        for (int j = 0; j < kPer; ++j)
+            if (k0[j] < prev && k0[j] > best) best = k0[j];
+        for (int64_t base = 32 * kPer; base < nvis; base += 32 * kPer) {
+#pragma unroll
+            for (int j = 0; j < kPer; ++j) {
+                const int64_t n = base + j * 32 + lane;
+                const uint64_t key = (n < nvis && n != r) ? rank_key(__ldg(s + n), n) : 0ull;
+                if (key < prev && key > best) best = key;
+            }
         }
         const uint32_t hi = __reduce_max_sync(0xffffffffu, (uint32_t)(best >> 32));
         const uint32_t lo = __reduce_max_sync(0xffffffffu, (uint32_t)(best >> 32) == hi ? (uint32_t)best : 0u);

@@ -134,7 +134,7 @@ class MsaProblem:
         B, Tq, Hq, D = self.q.shape
         HI, DI = self.q_idx.shape[2], self.q_idx.shape[3]
         Hkv = self.k.data.shape[1]
-        lmax = self.k.data.shape[2]
+        lmax = self.ik.data.shape[2]  # every cache of a problem has the same capacity
         return _Params(B, Tq, Hq, Hkv, D, HI, DI, lmax, self.seq_lens.data_ptr(), self.k._c(), self.v._c(),
                        self.ik._c(), self.q.data_ptr(), self.q_idx.data_ptr(),
                        None if self.w_idx is None else self.w_idx.data_ptr(), self.softmax_scale, self.pool_mode,
@@ -142,7 +142,7 @@ class MsaProblem:
 
     @property
     def nbmax(self) -> int:
-        return self.k.data.shape[2] // MSA_BLOCK_TOKENS
+        return self.ik.data.shape[2] // MSA_BLOCK_TOKENS
 
 
 # --------------------------------------------------------------------------- codec
