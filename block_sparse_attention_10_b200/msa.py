@@ -27,7 +27,8 @@ MSA_STATUS_TIMEOUT = 4
 
 # names exported by the C ABI (include/msa.h)
 EXPORTS = ("msa_status_string", "msa_version", "msa_nvfp4_encode", "msa_nvfp4_decode", "msa_nvfp4_amax",
-           "msa_workspace_size", "msa_index", "msa_select", "msa_attend", "msa_decode")
+           "msa_workspace_size", "msa_index", "msa_select", "msa_attend", "msa_decode", "msa_decode_static")
+MSA_STATIC_SCRATCH_BYTES = 4 << 20
 
 
 class MsaError(RuntimeError):
@@ -73,6 +74,7 @@ def lib() -> ctypes.CDLL:
         L.msa_select.argtypes = [P, vp, vp, vp]
         L.msa_attend.argtypes = [P, vp, vp, vp, vp]
         L.msa_decode.argtypes = [P, vp, ctypes.c_size_t, vp, vp, vp, vp]
+        L.msa_decode_static.argtypes = [P, vp, vp, vp, vp]
         for name in (n for n in EXPORTS if n not in ("msa_status_string", "msa_version", "msa_workspace_size")):
             getattr(L, name).restype = i32
         _lib = L
@@ -200,6 +202,18 @@ def msa_decode(p: MsaProblem, ws: torch.Tensor, out: torch.Tensor, lse: Optional
     prm = p.params()
     _check(lib().msa_decode(ctypes.byref(prm), _ptr(ws), ws.numel() * ws.element_size(), _ptr(out), _ptr(lse),
                             _ptr(sel_out), _stream(stream)), "msa_decode")
+
+
+def msa_decode_static(p: MsaProblem, out: torch.Tensor, lse: Optional[torch.Tensor] = None,
+                      sel_out: Optional[torch.Tensor] = None, stream=None):
+    """msa_decode with the library's own static device scratch (no allocation anywhere).
+
+    For callers that cannot allocate device memory; calls that overlap on the GPU race
+    (they share one scratch array), and the first call on a device should precede any
+    stream capture."""
+    prm = p.params()
+    _check(lib().msa_decode_static(ctypes.byref(prm), _ptr(out), _ptr(lse), _ptr(sel_out), _stream(stream)),
+           "msa_decode_static")
 
 
 def alloc_workspace(p: MsaProblem) -> torch.Tensor:

@@ -176,6 +176,35 @@ int msa_attend(const msa_params_t* p, const int32_t* sel, float* out, float* lse
 int msa_decode(const msa_params_t* p, void* ws, size_t ws_bytes, float* out, float* lse,
                int32_t* sel_out, cudaStream_t stream);
 
+/* ---------------------------------------------------------------------------
+ * Decode without caller scratch.  No counterpart in the paper: this is a
+ * convenience of this library for callers that cannot allocate device memory.
+ * ------------------------------------------------------------------------- */
+
+/* Size of the library-owned device scratch array used by msa_decode_static. */
+#define MSA_STATIC_SCRATCH_BYTES (4u << 20) /* 4 MiB */
+
+/* msa_decode with its scratch (block scores + selection) in a fixed device
+ * array of MSA_STATIC_SCRATCH_BYTES owned by the library, for callers that
+ * cannot call cudaMalloc: a plugin handed only its inputs and outputs by a host
+ * framework that owns all device memory, or a hot loop that must not risk the
+ * device-wide synchronisation an allocation can cause.  Allocates and frees
+ * nothing, on the device or the host.
+ *   p, out, lse, sel_out, stream   as for msa_decode
+ * Returns the msa_decode argument errors, or MSA_EWORKSPACE when
+ * msa_workspace_size(p) exceeds MSA_STATIC_SCRATCH_BYTES (e.g. B * Tq *
+ * lmax / 128 * 4 bytes of block scores beyond about 4 MiB), or MSA_ECUDA if
+ * the array's device address cannot be obtained.
+ * Notes:
+ *   - every GPU that loads libmsa.so holds the array until the process exits;
+ *   - the first call on each device looks up the array's address (once, with
+ *     that device current); make that first call before any stream capture;
+ *   - all calls share the one array, which keeps the last call's contents:
+ *     calls that overlap on the GPU (other streams, other host threads) race
+ *     and must be serialised by the caller. */
+int msa_decode_static(const msa_params_t* p, float* out, float* lse, int32_t* sel_out,
+                      cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
