@@ -63,6 +63,26 @@ def _algorithmic_bytes(w, seq_lens):
     return idx, att
 
 
+def rank_workload(w, rank: int):
+    """The shard a rank owns: its own sequences, i.e. the workload with a rank-specific seed."""
+    return synth.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank})
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """Max of a per-rank time over all ranks (identity without a process group)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_throughput(tokens_per_rank: int, world: int, seconds: float) -> float:
+    """Whole-job query tokens per second: every rank's tokens over the slowest rank's time."""
+    return tokens_per_rank * world / seconds
+
+
 def _measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -145,11 +165,10 @@ class ClockSampler:
                 "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
-def build_problem(w, batch_ids, seed_offset, device):
+def build_problem(w, batch_ids, device):
     """GPU-resident NVFP4 caches (encoded by the library) + queries for `batch_ids`."""
     from block_sparse_attention_10_b200 import msa
-    ww = synth.Workload(**{**w.__dict__, "seed": w.seed + seed_offset})
-    inp = synth.make_inputs(ww, batch_ids=batch_ids, device=device)
+    inp = synth.make_inputs(w, batch_ids=batch_ids, device=device)
     k = msa.encode_cache(inp.k, inp.s_k)
     v = msa.encode_cache(inp.v, inp.s_v)
     ik = msa.encode_cache(inp.ik, inp.s_ik)
@@ -283,7 +302,7 @@ def run_ours(args):
     w = WORKLOAD
 
     # each rank owns its own 32 sequences (weak scaling): seed offset by rank
-    p0 = build_problem(w, list(range(w.B)), seed_offset=1000 * rank, device=dev)
+    p0 = build_problem(rank_workload(w, rank), list(range(w.B)), device=dev)
     reps = [p0] + [clone_problem(p0) for _ in range(args.replicas - 1)]
     ws_t = msa.alloc_workspace(p0)
     out, lse, sel = msa.outputs(p0)
@@ -324,11 +343,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     if ws_n > 1:
         torch.distributed.barrier()
-    ms = e0.elapsed_time(e1) / args.steps
-    if ws_n > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = t.item()
+    ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
     status = int(p0.status.item())
     assert status == 0, f"device status word {status}"
 
@@ -370,18 +385,14 @@ def run_ours(args):
     e2e_s = (time.perf_counter() - t0) / n_e2e
     h2d = hq.numel() * hq.element_size() + hqi.numel() * hqi.element_size()
     d2h = hout.numel() * hout.element_size()
-    if ws_n > 1:
-        t = torch.tensor([e2e_s], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_s = t.item()
+    e2e_s = max_over_ranks(e2e_s, dev)
 
     cpu = None
     if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(w)
 
     if rank == 0:
-        tokens = w.B * w.Tq * ws_n
-        value = tokens / (ms * 1e-3)
+        value = aggregate_throughput(w.B * w.Tq, ws_n, ms * 1e-3)
         step_bytes = idx_bytes + att_bytes
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws_n, "steps": args.steps,
@@ -402,7 +413,7 @@ def run_ours(args):
                          "algorithmic_bytes_per_launch": idx_bytes, "launch_ms": idx_ms,
                          "traffic": _profile_traffic("index_decode.cu", w.name)},
             "cpu_baseline": cpu,
-            "e2e": {"value": w.B * w.Tq * ws_n / e2e_s, "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "e2e": {"value": aggregate_throughput(w.B * w.Tq, ws_n, e2e_s), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": 3 * args.steps,
             "clocks": clk.summary(),

@@ -8,25 +8,26 @@
 //
 // Design (B200): one thread-block cluster of 4 CTAs x 4 warps per
 // (sequence, query token, KV head): each of the 16 warps takes one selected
-// block (split-K over the <= 16 blocks), so the whole gather of <= 2,048 keys
-// is in flight at once.  Per 16 keys a warp computes
-//   S   = Q K^T    mma m16n8k16: A = the G query heads of this KV head
-//                  (zero-padded to 16 rows), B = dequantised K (exact f16);
-//   P   = online softmax of S in the exp2 domain (fp32);
-//   O^T += V^T P^T mma m16n8k16: A = dequantised V (exact f16), B = P as
-//                  fp16 taken straight from S's accumulator layout, so the
-//                  output tile [128 dims x 8 heads] wastes no rows.
+// block (split-K over the <= 16 blocks).  Each warp brings its whole block (K
+// and V nibbles + scales of up to 128 keys, 18 KB) into its own shared-memory
+// stage with four untiled bulk copies (cp.async.bulk, no multicast) on one
+// mbarrier, so every selected byte is requested at kernel start.  Then:
+//   S^T = K Q^T    mma m16n8k16, A = dequantised K (exact f16, 16 keys),
+//                  B = the G query heads of this KV head (8 columns) — the
+//                  same tile routine as the indexer, no padded rows;
+//   softmax        once per block (max over all its keys, exp2 domain), no
+//                  per-tile rescaling;
+//   O^T += V^T P^T mma m16n8k16, A = dequantised V, B = P^T obtained from the
+//                  S^T accumulators by one movmatrix (8x8 transpose) per 8 keys;
+//                  output tile [128 dims x 8 heads], no padded rows.
 // The partial (m, l, O) of the 4 warps are merged in shared memory, then the 4
 // CTAs of the cluster merge through distributed shared memory (each CTA
 // finalises 32 of the 128 dims).  No global scratch, no second launch, a
-// fixed merge order (bitwise deterministic).  Each warp brings its whole
-// block (K and V nibbles + scales of up to 128 keys, 18 KB) into its own
-// shared-memory stage with four untiled bulk copies (cp.async.bulk, no
-// multicast) on one mbarrier, so every selected byte is requested at kernel
-// start; the math then reads shared memory only.
+// fixed merge order (bitwise deterministic).
 #include <cooperative_groups.h>
 
 #include "internal.h"
+#include "nvfp4_mma.cuh"
 
 namespace msa {
 namespace {
@@ -99,31 +100,32 @@ __global__ void __cluster_dims__(kAttCluster, 1, 1) __launch_bounds__(kAttThread
         }
     }
 
-    // Q rows (query heads kvh*G + g), dims [32c, 32c+32) as 16 f16x2 pairs
-    uint32_t qa[8][2];
+    // query fragments: column g = query head kvh*G + g, dims permuted as the K rows
+    uint32_t qf[1][8][2];
     if (g < G) {
         const __nv_bfloat16* qrow = p.q + ((bt * p.Hq) + (int64_t)kvh * G + g) * kD + c * 32;
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
             const uint4 w4 = *reinterpret_cast<const uint4*>(qrow + 8 * v);
-            qa[2 * v][0] = bf16x2_to_f16x2(w4.x);
-            qa[2 * v][1] = bf16x2_to_f16x2(w4.y);
-            qa[2 * v + 1][0] = bf16x2_to_f16x2(w4.z);
-            qa[2 * v + 1][1] = bf16x2_to_f16x2(w4.w);
+            qf[0][2 * v][0] = bf16x2_to_f16x2(w4.x);
+            qf[0][2 * v][1] = bf16x2_to_f16x2(w4.y);
+            qf[0][2 * v + 1][0] = bf16x2_to_f16x2(w4.z);
+            qf[0][2 * v + 1][1] = bf16x2_to_f16x2(w4.w);
         }
     } else {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) qa[i][0] = qa[i][1] = 0u;
+        for (int i = 0; i < 8; ++i) qf[0][i][0] = qf[0][i][1] = 0u;
     }
 
     const float sc_log2 = p.softmax_scale * p.k.s_t * kLog2e;
-    float m_run = -INFINITY, l_run = 0.0f;
+    // per thread: query heads 2c and 2c+1
+    float m2[2] = {-INFINITY, -INFINITY}, l2[2] = {0.0f, 0.0f};
     float o[8][4];
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.0f;
 
     if (blk >= 0 && !mbar_wait(&bars[warp], 0)) {
-        if (lane == 0) set_status(p.status, MSA_STATUS_TIMEOUT);
+        if (lane == 0) set_status(p.status, MSA_STATUS_TIMEOUT | MSA_STATUS_AT_ATTEND);
         mbar_wait(&bars[warp], 0);  // one more bounded wait for the copies before the stage is reused
         blk = -1;
     }
@@ -133,87 +135,87 @@ __global__ void __cluster_dims__(kAttCluster, 1, 1) __launch_bounds__(kAttThread
         const uint8_t* vd = stage + kKData + kKScale;
         const uint8_t* vsc = stage + 2 * kKData + kKScale;
         const int ntiles = (nk + 15) >> 4;
-        for (int kt = 0; kt < ntiles; ++kt) {
-            // ---- S = Q K^T over 16 keys (two n-tiles of 8 keys)
-            float sacc[2][4];
+        // ---- S^T = K Q^T for every key of the block: st[kt] = rows (keys) g, g+8 x cols 2c, 2c+1
+        float st[8][4];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int key = kt * 16 + 8 * h + g;
-                const uint4 kw = lds_v4(kd + key * 64 + c * 16);
-                const uint32_t ks = e4m3x2_to_f16x2(lds_u16(ksc + key * 8 + c * 2));
-                sacc[h][0] = sacc[h][1] = sacc[h][2] = sacc[h][3] = 0.0f;
-                uint32_t kh[16];
-                e2m1x8_to_f16x8(kw.x, kh[0], kh[1], kh[2], kh[3]);
-                e2m1x8_to_f16x8(kw.y, kh[4], kh[5], kh[6], kh[7]);
-                e2m1x8_to_f16x8(kw.z, kh[8], kh[9], kh[10], kh[11]);
-                e2m1x8_to_f16x8(kw.w, kh[12], kh[13], kh[14], kh[15]);
-                const uint32_t slo = prmt(ks, ks, 0x1010u), shi = prmt(ks, ks, 0x3232u);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const uint32_t sc = i < 4 ? slo : shi;
-                    mma16816(sacc[h], qa[i][0], 0u, qa[i][1], 0u, hmul2(kh[2 * i], sc), hmul2(kh[2 * i + 1], sc));
-                }
+        for (int kt = 0; kt < 8; ++kt) {
+            if (kt < ntiles) {
+                float acc[1][4];
+                nvfp4_tile_mma<128, 1>(kd, ksc, kt * 16 + g, c, qf, acc);
+                const bool v0 = kt * 16 + g < nk, v1 = kt * 16 + g + 8 < nk;
+                st[kt][0] = v0 ? acc[0][0] * sc_log2 : -INFINITY;
+                st[kt][1] = v0 ? acc[0][1] * sc_log2 : -INFINITY;
+                st[kt][2] = v1 ? acc[0][2] * sc_log2 : -INFINITY;
+                st[kt][3] = v1 ? acc[0][3] * sc_log2 : -INFINITY;
+            } else {
+                st[kt][0] = st[kt][1] = st[kt][2] = st[kt][3] = -INFINITY;
             }
-            // ---- online softmax for query row g (exp2 domain)
-            float x[4];
+        }
+        // ---- softmax statistics over the block (query heads 2c, 2c+1)
 #pragma unroll
-            for (int h = 0; h < 2; ++h)
+        for (int e = 0; e < 2; ++e) {
+            float mx = -INFINITY;
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    const int key = kt * 16 + 8 * h + 2 * c + e;
-                    x[2 * h + e] = key < nk ? sacc[h][e] * sc_log2 : -INFINITY;
-                }
-            float mx = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-            const float m_new = fmaxf(m_run, mx);
-            const float corr = exp2f(m_run - m_new);
-            float pr[4];
+            for (int kt = 0; kt < 8; ++kt) mx = fmaxf(mx, fmaxf(st[kt][e], st[kt][2 + e]));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+            m2[e] = mx;
+            float l = 0.0f;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) pr[e] = exp2f(x[e] - m_new);
-            l_run = l_run * corr + (pr[0] + pr[1]) + (pr[2] + pr[3]);
-            m_run = m_new;
-            const uint32_t pb0 = pack_f16x2(pr[0], pr[1]), pb1 = pack_f16x2(pr[2], pr[3]);
-            // rescale O^T columns: this thread holds query rows 2c and 2c+1
-            const float c0 = __shfl_sync(0xffffffffu, corr, 8 * c), c1 = __shfl_sync(0xffffffffu, corr, 8 * c + 4);
-            // ---- O^T += V^T P^T; V of keys 2c, 2c+1, 2c+8, 2c+9 (masked keys read as 0)
-            uint32_t vh[4][8];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int key = kt * 16 + 2 * c + (i & 1) + 8 * (i >> 1);
-                uint2 vw = make_uint2(0u, 0u);
-                uint32_t vs = 0u;
-                if (key < nk) {
-                    vw = lds_v2(vd + key * 64 + g * 8);
-                    vs = lds_u8(vsc + key * 8 + g);
-                }
-                e2m1x8_to_f16x8(vw.x, vh[i][0], vh[i][1], vh[i][2], vh[i][3]);
-                e2m1x8_to_f16x8(vw.y, vh[i][4], vh[i][5], vh[i][6], vh[i][7]);
-                const uint32_t sc = e4m3_bcast_f16x2(vs);
-#pragma unroll
-                for (int m = 0; m < 8; ++m) vh[i][m] = hmul2(vh[i][m], sc);
+            for (int kt = 0; kt < 8; ++kt) {
+                st[kt][e] = exp2f(st[kt][e] - mx);
+                st[kt][2 + e] = exp2f(st[kt][2 + e] - mx);
+                l += st[kt][e] + st[kt][2 + e];
             }
+            l2[e] = l;
+        }
+        // ---- O^T += V^T P^T, 16 keys at a time
 #pragma unroll
-            for (int mt = 0; mt < 8; ++mt) {
-                o[mt][0] *= c0;
-                o[mt][1] *= c1;
-                o[mt][2] *= c0;
-                o[mt][3] *= c1;
-                const uint32_t a0 = prmt(vh[0][mt], vh[1][mt], 0x5410u);
-                const uint32_t a1 = prmt(vh[0][mt], vh[1][mt], 0x7632u);
-                const uint32_t a2 = prmt(vh[2][mt], vh[3][mt], 0x5410u);
-                const uint32_t a3 = prmt(vh[2][mt], vh[3][mt], 0x7632u);
-                mma16816(o[mt], a0, a1, a2, a3, pb0, pb1);
+        for (int kt = 0; kt < 8; ++kt) {
+            if (kt < ntiles) {
+                // P^T fragment (keys x heads) -> B operand (k = keys 2c.., n = head g)
+                const uint32_t pb0 = movmatrix_trans(pack_f16x2(st[kt][0], st[kt][1]));
+                const uint32_t pb1 = movmatrix_trans(pack_f16x2(st[kt][2], st[kt][3]));
+                uint32_t vh[4][8];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int key = kt * 16 + 2 * c + (i & 1) + 8 * (i >> 1);
+                    uint2 vw = make_uint2(0u, 0u);
+                    uint32_t vs = 0u;
+                    if (key < nk) {  // masked keys read as 0 (their P is 0; V may hold anything)
+                        vw = lds_v2(vd + key * 64 + g * 8);
+                        vs = lds_u8(vsc + key * 8 + g);
+                    }
+                    e2m1x8_to_f16x8(vw.x, vh[i][0], vh[i][1], vh[i][2], vh[i][3]);
+                    e2m1x8_to_f16x8(vw.y, vh[i][4], vh[i][5], vh[i][6], vh[i][7]);
+                    const uint32_t sc = e4m3_bcast_f16x2(vs);
+#pragma unroll
+                    for (int m = 0; m < 8; ++m) vh[i][m] = hmul2(vh[i][m], sc);
+                }
+#pragma unroll
+                for (int mt = 0; mt < 8; ++mt) {
+                    const uint32_t a0 = prmt(vh[0][mt], vh[1][mt], 0x5410u);
+                    const uint32_t a1 = prmt(vh[0][mt], vh[1][mt], 0x7632u);
+                    const uint32_t a2 = prmt(vh[2][mt], vh[3][mt], 0x5410u);
+                    const uint32_t a3 = prmt(vh[2][mt], vh[3][mt], 0x7632u);
+                    mma16816(o[mt], a0, a1, a2, a3, pb0, pb1);
+                }
             }
         }
     }
 
     // ---- merge the 4 warps of this CTA (each warp's partial O goes into its own stage)
-    l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
-    l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
-    if (c == 0) {
-        sM[warp][g] = m_run;
-        sL[warp][g] = l_run;
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+        float l = l2[e];
+        l += __shfl_xor_sync(0xffffffffu, l, 4);
+        l += __shfl_xor_sync(0xffffffffu, l, 8);
+        l += __shfl_xor_sync(0xffffffffu, l, 16);
+        if (g == 0) {
+            sM[warp][2 * c + e] = m2[e];
+            sL[warp][2 * c + e] = l;
+        }
     }
     __syncwarp();
     float* sOw = reinterpret_cast<float*>(stage);  // [8][kD]

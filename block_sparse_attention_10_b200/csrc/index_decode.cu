@@ -29,6 +29,7 @@
 //     shuffles, causal / length masking, block pooling, one store per
 //     (token, block).
 #include "internal.h"
+#include "nvfp4_mma.cuh"
 
 namespace msa {
 namespace {
@@ -66,61 +67,6 @@ __device__ __forceinline__ bool token_owner(int c) {
     if constexpr (HI <= 2) return true;
     else if constexpr (HI == 4) return (c & 1) == 0;
     else return c == 0;
-}
-
-// One 16-key tile: rows r0 and r0 + 8 of the stage, dequantised (E2M1 * E4M3, exact in
-// f16) into A fragments, times the resident query fragments; acc = [NT n-tiles][c0..c3].
-template <int DI, int NT>
-__device__ __forceinline__ void tile_mma(const uint8_t* sd, const uint8_t* ss, int r0, int c,
-                                         const uint32_t (&qf)[NT][DI / 16][2], float (&acc)[NT][4]) {
-    constexpr int KS = DI / 16;
-    const int r1 = r0 + 8;
-    uint32_t h0[2 * KS], h1[2 * KS];
-    uint32_t s0[KS], s1[KS];
-    if constexpr (DI == 128) {
-        const uint4 w0 = lds_v4(sd + r0 * 64 + c * 16);
-        const uint4 w1 = lds_v4(sd + r1 * 64 + c * 16);
-        const uint32_t sc0 = e4m3x2_to_f16x2(lds_u16(ss + r0 * 8 + c * 2));
-        const uint32_t sc1 = e4m3x2_to_f16x2(lds_u16(ss + r1 * 8 + c * 2));
-        e2m1x8_to_f16x8(w0.x, h0[0], h0[1], h0[2], h0[3]);
-        e2m1x8_to_f16x8(w0.y, h0[4], h0[5], h0[6], h0[7]);
-        e2m1x8_to_f16x8(w0.z, h0[8], h0[9], h0[10], h0[11]);
-        e2m1x8_to_f16x8(w0.w, h0[12], h0[13], h0[14], h0[15]);
-        e2m1x8_to_f16x8(w1.x, h1[0], h1[1], h1[2], h1[3]);
-        e2m1x8_to_f16x8(w1.y, h1[4], h1[5], h1[6], h1[7]);
-        e2m1x8_to_f16x8(w1.z, h1[8], h1[9], h1[10], h1[11]);
-        e2m1x8_to_f16x8(w1.w, h1[12], h1[13], h1[14], h1[15]);
-        const uint32_t a0 = prmt(sc0, sc0, 0x1010u), a1 = prmt(sc0, sc0, 0x3232u);
-        const uint32_t b0 = prmt(sc1, sc1, 0x1010u), b1 = prmt(sc1, sc1, 0x3232u);
-#pragma unroll
-        for (int i = 0; i < KS; ++i) {
-            s0[i] = i < 4 ? a0 : a1;
-            s1[i] = i < 4 ? b0 : b1;
-        }
-    } else {
-        const uint2 w0 = lds_v2(sd + r0 * 32 + c * 8);
-        const uint2 w1 = lds_v2(sd + r1 * 32 + c * 8);
-        const uint32_t a0 = e4m3_bcast_f16x2(lds_u8(ss + r0 * 4 + c));
-        const uint32_t b0 = e4m3_bcast_f16x2(lds_u8(ss + r1 * 4 + c));
-        e2m1x8_to_f16x8(w0.x, h0[0], h0[1], h0[2], h0[3]);
-        e2m1x8_to_f16x8(w0.y, h0[4], h0[5], h0[6], h0[7]);
-        e2m1x8_to_f16x8(w1.x, h1[0], h1[1], h1[2], h1[3]);
-        e2m1x8_to_f16x8(w1.y, h1[4], h1[5], h1[6], h1[7]);
-#pragma unroll
-        for (int i = 0; i < KS; ++i) {
-            s0[i] = a0;
-            s1[i] = b0;
-        }
-    }
-#pragma unroll
-    for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
-#pragma unroll
-    for (int i = 0; i < KS; ++i) {
-        const uint32_t ra0 = hmul2(h0[2 * i], s0[i]), ra2 = hmul2(h0[2 * i + 1], s0[i]);
-        const uint32_t ra1 = hmul2(h1[2 * i], s1[i]), ra3 = hmul2(h1[2 * i + 1], s1[i]);
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) mma16816(acc[nt], ra0, ra1, ra2, ra3, qf[nt][i][0], qf[nt][i][1]);
-    }
 }
 
 template <int DI, int HI, int NT>
@@ -188,7 +134,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
                 const int s = k % S;
                 const uint32_t round = (uint32_t)(k / S);
                 if (round > 0 && !mbar_wait(&empty[s], (round - 1) & 1u)) {
-                    set_status(p.status, MSA_STATUS_TIMEOUT);
+                    set_status(p.status, MSA_STATUS_TIMEOUT | MSA_STATUS_AT_INDEX_PRODUCER);
                     ok = false;
                     break;
                 }
@@ -208,7 +154,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
             const int issued = k;
             for (int j = max(0, issued - S); j < issued; ++j) {
                 if (!mbar_wait(&full[j % S], (uint32_t)(j / S) & 1u)) {
-                    set_status(p.status, MSA_STATUS_TIMEOUT);
+                    set_status(p.status, MSA_STATUS_TIMEOUT | MSA_STATUS_AT_INDEX_DRAIN);
                     break;
                 }
             }
@@ -240,8 +186,15 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
 
     for (int k = cw; k < nu; k += kIdxConsumers) {
         const int s = k % S;
-        if (!mbar_wait(&full[s], (uint32_t)(k / S) & 1u)) {
-            set_status(p.status, MSA_STATUS_TIMEOUT);
+        const uint32_t round = (uint32_t)(k / S);
+        // Units go to consumers round-robin, so this warp may reach stage s while the
+        // stage's previous copy (unit k - S, another warp's) is still landing, and a parity
+        // wait on full[s] cannot tell "phase round - 1 still open" from "phase round
+        // complete".  The stage's empty barrier settles it: its phase round - 1 completes
+        // only after that earlier unit was consumed (so full[s] is past phase round - 1),
+        // and it cannot move past phase round before this warp releases the stage.
+        if ((round > 0 && !mbar_wait(&empty[s], (round - 1) & 1u)) || !mbar_wait(&full[s], round & 1u)) {
+            set_status(p.status, MSA_STATUS_TIMEOUT | MSA_STATUS_AT_INDEX_CONSUMER);
             break;
         }
         const int64_t u = u_begin + k;
@@ -298,7 +251,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
 #pragma unroll 2
             for (int ti = 0; ti < kBlock / 16; ++ti) {
                 float acc[NT][4];
-                tile_mma<DI, NT>(sd, ss, ti * 16 + g, c, qf, acc);
+                nvfp4_tile_mma<DI, NT>(sd, ss, ti * 16 + g, c, qf, acc);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -344,7 +297,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
         for (int ti = 0; ti < ntiles; ++ti) {
             const int r0 = ti * 16 + g, r1 = r0 + 8;
             float acc[NT][4];
-            tile_mma<DI, NT>(sd, ss, r0, c, qf, acc);
+            nvfp4_tile_mma<DI, NT>(sd, ss, r0, c, qf, acc);
             // epilogue: ReLU * w, sum over heads, mask, pool
             const int64_t j0 = kbase + r0, j1 = kbase + r1;
 #pragma unroll

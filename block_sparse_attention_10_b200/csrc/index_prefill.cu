@@ -1,0 +1,387 @@
+// index_prefill.cu — MSA indexer + block pooling for a chunk of many query tokens
+// (chunked prefill), on the fifth-generation tensor cores.
+//
+// Method ("vLLM Adds Day-0 Support for MiniMax-M3.1-Flash", ainewsbites.com,
+// "A model built for efficient inference"): every query scores every visible
+// key with the lightweight indexer, and the scores are pooled per 128-token
+// block.  With Tq query tokens and HI heads this is a dense contraction
+// [Tq*HI rows x DI] x [DI x L keys] per sequence with a causal mask at the end
+// of the context — the pages' prefill optimisation is a fused prefill path.
+// Reading: s = sum_h w_h ReLU(q_h . k); mean over the block's visible keys.
+// Because the mean is linear, the block score of token t is
+//     S[t, n] = (1/cnt) * sum_h w_h * sum_{j in n, j <= pos_t} ReLU(q_{t,h} . k_j),
+// so each accumulator row (one (token, head)) only needs its own ReLU-sum over
+// the block's columns; the head sum happens once per (token, block).
+//
+// Design (B200, one persistent CTA per SM, 10 warps):
+//   * work unit = (sequence, 256 keys = 2 MSA blocks, up to 64 query tiles);
+//   * warps 0-7 dequantise the unit's 256 NVFP4 keys into a bf16 shared tile
+//     in the canonical K-major 128-byte-swizzle layout (e2m1*e4m3 is exact in
+//     bf16; the fp32 tensor scale is applied to the pooled score), then run
+//     the epilogue;
+//   * warp 9 (one lane) streams 128-row query tiles [128 x DI] bf16 with TMA
+//     (128-byte swizzle, no multicast) into a 4-stage ring;
+//   * warp 8 (one lane) issues tcgen05.mma 128 x 256 x 16 (bf16 -> fp32 in
+//     tensor memory), double-buffered over 2 x 256 TMEM columns, and commits
+//     to mbarriers;
+//   * epilogue: each warp reads its 32 TMEM lanes x 128 columns (one block)
+//     with tcgen05.ld, sums ReLU over the visible columns, applies head
+//     weights, sums heads with shuffles and writes one pooled score.
+// Query tiles whose tokens see none of the unit's keys are skipped entirely.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "internal.h"
+#include "tcgen05.cuh"
+
+namespace msa {
+namespace {
+
+constexpr int kPfEpiWarps = 8;
+constexpr int kPfMmaWarp = 8;
+constexpr int kPfTmaWarp = 9;
+constexpr int kPfThreads = 32 * 10;
+constexpr int kPfQStages = 4;
+constexpr int kPfRows = 128;    // M: query rows (token, head) per tile
+constexpr int kPfKeys = 256;    // N: keys per unit (2 MSA blocks)
+constexpr int kPfQChunk = 64;   // query tiles per unit
+constexpr int kPfTmemCols = 512;
+
+template <int DI>
+struct PfGeom {
+    static constexpr int kKB = DI / 64;                   // 128-byte K-blocks per row
+    static constexpr int kQStage = kPfRows * DI * 2;      // bytes per query stage
+    static constexpr int kQBlock = kPfRows * 128;         // one K-block of a query stage
+    static constexpr int kKTile = kPfKeys * DI * 2;       // bf16 key tile
+    static constexpr int kKBlock = kPfKeys * 128;         // one K-block of the key tile
+    static constexpr size_t kSmem = 1024 + kKTile + kPfQStages * kQStage + 256;
+};
+
+struct PfShape {
+    int nqt;      // query tiles per sequence
+    int nqc;      // query chunks per sequence
+    int nkt;      // key tiles (2 blocks) per sequence capacity
+    int64_t units;
+};
+
+__device__ __forceinline__ PfShape pf_shape(const Problem& p, int HI) {
+    PfShape s;
+    s.nqt = (p.Tq * HI + kPfRows - 1) / kPfRows;
+    s.nqc = (s.nqt + kPfQChunk - 1) / kPfQChunk;
+    s.nkt = (int)((p.nbmax + 1) / 2);
+    s.units = (int64_t)p.B * s.nkt * s.nqc;
+    return s;
+}
+
+// Does any token of query tile qt see any of the keys [k0, k0 + 256)?
+template <int HI>
+__device__ __forceinline__ bool pf_tile_live(int qt, int64_t k0, int64_t L, int Tq) {
+    const int tb = min(Tq, (qt + 1) * (kPfRows / HI));  // one past the tile's last token
+    return k0 < L && k0 <= L - Tq + tb - 1;
+}
+
+template <int DI, int HI>
+__global__ void __launch_bounds__(kPfThreads, 1)
+    index_prefill_kernel(const Problem p, float* __restrict__ block_scores, const __grid_constant__ CUtensorMap tmap) {
+    using G = PfGeom<DI>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* kbuf = smem;
+    uint8_t* qbuf = smem + G::kKTile;
+    uint64_t* q_full = reinterpret_cast<uint64_t*>(qbuf + kPfQStages * G::kQStage);
+    uint64_t* q_empty = q_full + kPfQStages;
+    uint64_t* t_full = q_empty + kPfQStages;
+    uint64_t* t_empty = t_full + 2;
+    uint64_t* k_ready = t_empty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(k_ready + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_wait();
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kPfQStages; ++s) {
+            mbar_init(&q_full[s], 1);
+            mbar_init(&q_empty[s], 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&t_full[s], 1);
+            mbar_init(&t_empty[s], kPfEpiWarps);
+        }
+        mbar_init(k_ready, kPfEpiWarps);
+        fence_mbar_init();
+    }
+    if (warp == kPfMmaWarp) {
+        tmem_alloc(tmem_slot, kPfTmemCols);
+        tmem_relinquish();
+    }
+    tcgen05_fence_before();
+    __syncthreads();
+    tcgen05_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    pdl_launch_dependents();
+
+    const PfShape sh = pf_shape(p, HI);
+    const int Tq = p.Tq;
+    const float s_t = p.ik.s_t;
+
+    if (warp == kPfTmaWarp) {
+        // ------------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t qi = 0;
+            bool ok = true;
+            for (int64_t u = blockIdx.x; u < sh.units && ok; u += gridDim.x) {
+                const int b = (int)(u / ((int64_t)sh.nkt * sh.nqc));
+                const int64_t rem = u % ((int64_t)sh.nkt * sh.nqc);
+                const int64_t k0 = (rem / sh.nqc) * kPfKeys;
+                const int qc = (int)(rem % sh.nqc);
+                const int64_t L = clamp_len(p.seq_lens[b], Tq, p.lmax, nullptr);
+                for (int qt = qc * kPfQChunk; qt < min(sh.nqt, (qc + 1) * kPfQChunk); ++qt) {
+                    if (!pf_tile_live<HI>(qt, k0, L, Tq)) continue;
+                    const int s = (int)(qi % kPfQStages);
+                    if (qi >= (uint32_t)kPfQStages && !mbar_wait(&q_empty[s], ((qi / kPfQStages) - 1) & 1u)) {
+                        set_status(p.status, MSA_STATUS_TIMEOUT | MSA_STATUS_AT_INDEX_PRODUCER);
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_expect_tx(&q_full[s], (uint32_t)G::kQStage);
+#pragma unroll
+                    for (int kb = 0; kb < G::kKB; ++kb)
+                        tma_load_3d(qbuf + s * G::kQStage + kb * G::kQBlock, &tmap, kb * 64, qt * kPfRows, b,
+                                    &q_full[s]);
+                    ++qi;
+                }
+            }
+            // never leave with copies in flight into this CTA's shared memory
+            for (uint32_t j = qi > (uint32_t)kPfQStages ? qi - kPfQStages : 0u; j < qi; ++j)
+                if (!mbar_wait(&q_full[j % kPfQStages], (j / kPfQStages) & 1u)) {
+                    set_status(p.status, MSA_STATUS_TIMEOUT | MSA_STATUS_AT_INDEX_DRAIN);
+                    break;
+                }
+        }
+    } else if (warp == kPfMmaWarp) {
+        // ------------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = umma_idesc_bf16_f32(kPfRows, kPfKeys);
+            uint32_t qi = 0, ui = 0;
+            bool ok = true;
+            for (int64_t u = blockIdx.x; u < sh.units && ok; u += gridDim.x) {
+                const int b = (int)(u / ((int64_t)sh.nkt * sh.nqc));
+                const int64_t rem = u % ((int64_t)sh.nkt * sh.nqc);
+                const int64_t k0 = (rem / sh.nqc) * kPfKeys;
+                const int qc = (int)(rem % sh.nqc);
+                const int64_t L = clamp_len(p.seq_lens[b], Tq, p.lmax, nullptr);
+                const int qt_end = min(sh.nqt, (qc + 1) * kPfQChunk);
+                bool any = false;
+                for (int qt = qc * kPfQChunk; qt < qt_end; ++qt) any |= pf_tile_live<HI>(qt, k0, L, Tq);
+                if (!any) continue;
+                if (!mbar_wait(k_ready, ui & 1u)) {
+                    set_status(p.status, MSA_STATUS_TIMEOUT | MSA_STATUS_AT_INDEX_CONSUMER);
+                    break;
+                }
+                tcgen05_fence_after();
+                for (int qt = qc * kPfQChunk; qt < qt_end; ++qt) {
+                    if (!pf_tile_live<HI>(qt, k0, L, Tq)) continue;
+                    const int s = (int)(qi % kPfQStages);
+                    const int buf = (int)(qi & 1u);
+                    if (!mbar_wait(&q_full[s], (qi / kPfQStages) & 1u) ||
+                        (qi >= 2 && !mbar_wait(&t_empty[buf], ((qi >> 1) - 1) & 1u))) {
+                        set_status(p.status, MSA_STATUS_TIMEOUT | MSA_STATUS_AT_INDEX_CONSUMER);
+                        ok = false;
+                        break;
+                    }
+                    tcgen05_fence_after();
+                    const uint32_t qs = smem_u32(qbuf + s * G::kQStage), ks = smem_u32(kbuf);
+#pragma unroll
+                    for (int k = 0; k < DI / 16; ++k) {
+                        const int kb = k >> 2, kk = k & 3;
+                        umma_bf16_ss(tmem_base + (uint32_t)(buf * kPfKeys),
+                                     umma_desc_k_sw128(qs + kb * G::kQBlock + kk * 32),
+                                     umma_desc_k_sw128(ks + kb * G::kKBlock + kk * 32), idesc, k > 0 ? 1u : 0u);
+                    }
+                    umma_commit(&q_empty[s]);
+                    umma_commit(&t_full[buf]);
+                    ++qi;
+                }
+                ++ui;
+            }
+        }
+    } else {
+        // ------------------------------------------------------------------ epilogue warps
+        const int et = threadIdx.x;  // 0..255
+        // blocks past each sequence's length score -inf
+        {
+            const int64_t total = (int64_t)p.B * Tq * p.nbmax;
+            for (int64_t i = (int64_t)blockIdx.x * 256 + et; i < total; i += (int64_t)gridDim.x * 256) {
+                const int64_t n = i % p.nbmax;
+                const int b = (int)(i / (p.nbmax * Tq));
+                const int64_t L = clamp_len(p.seq_lens[b], Tq, p.lmax, blockIdx.x == 0 && i < 256 ? p.status : nullptr);
+                if (n >= (L + kBlock - 1) / kBlock) block_scores[i] = -INFINITY;
+            }
+        }
+        const int quad = warp & 3, hb = warp >> 2;
+        uint32_t qi = 0;
+        bool ok = true;
+        for (int64_t u = blockIdx.x; u < sh.units && ok; u += gridDim.x) {
+            const int b = (int)(u / ((int64_t)sh.nkt * sh.nqc));
+            const int64_t rem = u % ((int64_t)sh.nkt * sh.nqc);
+            const int64_t k0 = (rem / sh.nqc) * kPfKeys;
+            const int qc = (int)(rem % sh.nqc);
+            const int64_t L = clamp_len(p.seq_lens[b], Tq, p.lmax, nullptr);
+            const int64_t nb_b = (L + kBlock - 1) / kBlock;
+            const int64_t n = k0 / kBlock + hb;  // this warp's block
+            const int qt_end = min(sh.nqt, (qc + 1) * kPfQChunk);
+            bool any = false;
+            for (int qt = qc * kPfQChunk; qt < qt_end; ++qt) any |= pf_tile_live<HI>(qt, k0, L, Tq);
+            if (any) {
+                // dequantise the unit's 256 keys into the bf16 K-major SW128 tile (keys >= L read as 0)
+                constexpr int kChunksPerRow = DI / 8;
+                for (int ci = et; ci < kPfKeys * kChunksPerRow; ci += 256) {
+                    const int j = ci / kChunksPerRow, cr = ci % kChunksPerRow;
+                    const int64_t key = k0 + j;
+                    uint32_t w = 0u, sc = 0u;
+                    if (key < L) {
+                        const int64_t vec = (int64_t)b * p.lmax + key;
+                        w = *reinterpret_cast<const uint32_t*>(p.ik.data + vec * (DI / 2) + cr * 4);
+                        sc = p.ik.scale[vec * (DI / 16) + (cr >> 1)];
+                    }
+                    uint32_t h[4];
+                    e2m1x8_to_f16x8(w, h[0], h[1], h[2], h[3]);
+                    const uint32_t s2 = e4m3_bcast_f16x2(sc);
+                    uint4 o;
+                    uint32_t* op = &o.x;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint32_t m = hmul2(h[i], s2);  // e2m1 * e4m3, exact in f16 and in bf16
+                        const __half2 vm = *reinterpret_cast<const __half2*>(&m);
+                        const __nv_bfloat162 bb = __floats2bfloat162_rn(__low2float(vm), __high2float(vm));
+                        op[i] = *reinterpret_cast<const uint32_t*>(&bb);
+                    }
+                    const int kb = cr >> 3, cc = cr & 7;
+                    *reinterpret_cast<uint4*>(kbuf + kb * G::kKBlock + j * 128 + ((cc ^ (j & 7)) << 4)) = o;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(k_ready);
+            }
+            for (int qt = qc * kPfQChunk; qt < qt_end; ++qt) {
+                const int row = quad * 32 + lane;
+                const int R = qt * kPfRows + row;
+                const int t = R / HI, h = R % HI;
+                const bool live = pf_tile_live<HI>(qt, k0, L, Tq);
+                float sum = 0.0f;
+                int64_t cnt = 0;
+                if (t < Tq && n < nb_b) cnt = min64(kBlock, max64(0, L - Tq + t + 1 - n * kBlock));
+                if (live) {
+                    const int buf = (int)(qi & 1u);
+                    if (!mbar_wait(&t_full[buf], (qi >> 1) & 1u)) {
+                        set_status(p.status, MSA_STATUS_TIMEOUT | MSA_STATUS_AT_INDEX_CONSUMER);
+                        ok = false;
+                        break;
+                    }
+                    tcgen05_fence_after();
+                    const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * kPfKeys + hb * kBlock);
+#pragma unroll
+                    for (int c4 = 0; c4 < kBlock / 32; ++c4) {
+                        float v[32];
+                        tmem_ld32(taddr + c4 * 32, v);
+                        tmem_wait_ld();
+                        if (cnt >= (c4 + 1) * 32) {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) sum += fmaxf(v[i], 0.0f);
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i)
+                                if (c4 * 32 + i < cnt) sum += fmaxf(v[i], 0.0f);
+                        }
+                    }
+                    tcgen05_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&t_empty[buf]);
+                    ++qi;
+                }
+                float x = t < Tq ? sum * (p.w_idx ? p.w_idx[((int64_t)b * Tq + t) * HI + h] : 1.0f) : 0.0f;
+#pragma unroll
+                for (int o = 1; o < HI; o <<= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+                if (h == 0 && t < Tq && n < nb_b)
+                    block_scores[((int64_t)b * Tq + t) * p.nbmax + n] = cnt > 0 ? (x / (float)cnt) * s_t : -INFINITY;
+            }
+        }
+    }
+
+    tcgen05_fence_before();
+    __syncthreads();
+    if (warp == kPfMmaWarp) {
+        tcgen05_fence_after();
+        tmem_dealloc(tmem_base, kPfTmemCols);
+    }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (fn == nullptr) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+template <int DI, int HI>
+int launch_pf(const Problem& p, float* bs, bool pdl, cudaStream_t st) {
+    using G = PfGeom<DI>;
+    auto enc = tensor_map_encoder();
+    if (enc == nullptr) return MSA_ECUDA;
+    // query rows of one sequence: [B][Tq*HI][DI] bf16, 128 x 64 boxes, 128-byte swizzle
+    CUtensorMap tmap;
+    const cuuint64_t dims[3] = {(cuuint64_t)DI, (cuuint64_t)p.Tq * HI, (cuuint64_t)p.B};
+    const cuuint64_t strides[2] = {(cuuint64_t)DI * 2, (cuuint64_t)p.Tq * HI * DI * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)kPfRows, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<__nv_bfloat16*>(p.q_idx), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return MSA_ECUDA;
+    auto kern = index_prefill_kernel<DI, HI>;
+    static int configured_dev = -1;
+    const DeviceInfo& di = device_info();
+    if (configured_dev != di.device) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)G::kSmem) != cudaSuccess)
+            return MSA_ECUDA;
+        configured_dev = di.device;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)di.num_sms);
+    cfg.blockDim = dim3(kPfThreads);
+    cfg.dynamicSmemBytes = G::kSmem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, kern, p, bs, tmap) != cudaSuccess) return MSA_ECUDA;
+    return MSA_OK;
+}
+
+template <int DI>
+int launch_pf_hi(const Problem& p, float* bs, bool pdl, cudaStream_t st) {
+    switch (p.HI) {
+        case 1: return launch_pf<DI, 1>(p, bs, pdl, st);
+        case 2: return launch_pf<DI, 2>(p, bs, pdl, st);
+        case 4: return launch_pf<DI, 4>(p, bs, pdl, st);
+        case 8: return launch_pf<DI, 8>(p, bs, pdl, st);
+        default: return MSA_EUNSUPPORTED;
+    }
+}
+
+}  // namespace
+
+int launch_index_prefill(const Problem& p, float* block_scores, bool pdl, cudaStream_t st) {
+    if (p.pool_mode != 0) return MSA_EUNSUPPORTED;
+    if (p.DI == 128) return launch_pf_hi<128>(p, block_scores, pdl, st);
+    if (p.DI == 64) return launch_pf_hi<64>(p, block_scores, pdl, st);
+    return MSA_EUNSUPPORTED;
+}
+
+}  // namespace msa

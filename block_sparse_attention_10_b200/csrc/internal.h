@@ -49,6 +49,10 @@ int launch_nvfp4_amax(const float* x, int64_t n, float* amax_out, cudaStream_t s
 
 // Indexer + pooling over every visible key (decode: Tq * HI <= 32).
 int launch_index_decode(const Problem& p, float* block_scores, float* token_scores, bool pdl, cudaStream_t st);
+// Indexer + pooling for many query tokens (chunked prefill, tcgen05; mean pooling).
+int launch_index_prefill(const Problem& p, float* block_scores, bool pdl, cudaStream_t st);
+// Picks the decode or the prefill indexer for the problem's Tq * HI.
+int launch_index(const Problem& p, float* block_scores, float* token_scores, bool pdl, cudaStream_t st);
 // Top-16 selection, recent block forced.
 int launch_select(const Problem& p, const float* block_scores, int32_t* sel, int32_t* sel_copy, bool pdl,
                   cudaStream_t st);

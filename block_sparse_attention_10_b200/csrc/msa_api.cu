@@ -1,6 +1,7 @@
 // msa_api.cu — the C ABI of libmsa.so (see include/msa.h): host-side argument
 // checks, then the kernel launches.  No allocation, no host synchronisation.
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -56,7 +57,7 @@ int check_params(const msa_params_t* p, bool need_index, bool need_attend) {
         if (!aligned16(p->q_idx)) return MSA_EALIGN;
         if (p->DI != 64 && p->DI != 128) return MSA_EUNSUPPORTED;
         if (!is_pow2_le8(p->HI)) return MSA_EUNSUPPORTED;
-        if ((int64_t)p->Tq * p->HI > 32) return MSA_EUNSUPPORTED;
+        if ((int64_t)p->Tq * p->HI > 32 && p->pool_mode != 0) return MSA_EUNSUPPORTED;  // prefill: mean only
         if (p->B > 4096) return MSA_EUNSUPPORTED;
     }
     if (need_attend) {
@@ -95,6 +96,26 @@ Problem to_problem(const msa_params_t* p) {
     q.status = p->status;
     return q;
 }
+
+// Programmatic dependent launch between the decode kernels (on unless MSA_PDL=0).
+bool pdl_enabled() {
+    static const bool on = [] {
+        const char* e = std::getenv("MSA_PDL");
+        return !(e != nullptr && e[0] == '0');
+    }();
+    return on;
+}
+
+}  // namespace
+
+// Decode indexer (mma.sync, Tq * HI <= 32) or prefill indexer (tcgen05, larger Tq * HI).
+int launch_index(const Problem& p, float* block_scores, float* token_scores, bool pdl, cudaStream_t st) {
+    if ((int64_t)p.Tq * p.HI <= 32) return launch_index_decode(p, block_scores, token_scores, pdl, st);
+    if (token_scores != nullptr) return MSA_EUNSUPPORTED;
+    return launch_index_prefill(p, block_scores, pdl, st);
+}
+
+namespace {
 
 constexpr size_t kAlign = 256;
 size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
@@ -158,7 +179,7 @@ size_t msa_workspace_size(const msa_params_t* p) {
 int msa_index(const msa_params_t* p, float* block_scores, float* token_scores, cudaStream_t stream) {
     if (int r = check_params(p, true, false)) return r;
     if (!block_scores) return MSA_EINVAL;
-    return launch_index_decode(to_problem(p), block_scores, token_scores, false, stream);
+    return launch_index(to_problem(p), block_scores, token_scores, false, stream);
 }
 
 int msa_select(const msa_params_t* p, const float* block_scores, int32_t* sel, cudaStream_t stream) {
@@ -184,9 +205,10 @@ int msa_decode(const msa_params_t* p, void* ws, size_t ws_bytes, float* out, flo
     float* bs = static_cast<float*>(ws);
     int32_t* sel = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + ws_block_scores_bytes(p));
     const Problem q = to_problem(p);
-    if (int r = launch_index_decode(q, bs, nullptr, true, stream)) return r;
-    if (int r = launch_select(q, bs, sel, sel_out, true, stream)) return r;
-    return launch_attend(q, sel, out, lse, true, stream);
+    const bool pdl = pdl_enabled();
+    if (int r = launch_index(q, bs, nullptr, pdl, stream)) return r;
+    if (int r = launch_select(q, bs, sel, sel_out, pdl, stream)) return r;
+    return launch_attend(q, sel, out, lse, pdl, stream);
 }
 
 }  // extern "C"

@@ -71,6 +71,11 @@ typedef enum msa_status {
 #define MSA_STATUS_SEQLEN 1u   /* some seq_lens[b] < Tq or > lmax: clamped */
 #define MSA_STATUS_SELECT 2u   /* a selected block id >= the visible block count: skipped */
 #define MSA_STATUS_TIMEOUT 4u  /* a bounded wait inside a kernel gave up (results invalid) */
+/* With MSA_STATUS_TIMEOUT, which wait gave up: */
+#define MSA_STATUS_AT_INDEX_PRODUCER 0x100u /* indexer: producer waiting for a free stage */
+#define MSA_STATUS_AT_INDEX_DRAIN 0x200u    /* indexer: producer draining its last copies */
+#define MSA_STATUS_AT_INDEX_CONSUMER 0x400u /* indexer: consumer waiting for a stage's bytes */
+#define MSA_STATUS_AT_ATTEND 0x800u         /* attention: warp waiting for its block's bytes */
 
 /* One NVFP4 cache tensor (K, V or index-K); the layout is given above. */
 typedef struct msa_nvfp4_cache {
@@ -84,8 +89,10 @@ typedef struct msa_nvfp4_cache {
  *   B, Tq     sequences and query tokens per sequence (Tq >= 1)
  *   Hq, Hkv   attention query / KV heads; Hq / Hkv in {1, 2, 4, 8}
  *   D         attention head dim; 128
- *   HI, DI    indexer heads / dim; HI in {1, 2, 4, 8}, DI in {64, 128},
- *             Tq * HI <= 32 (decode indexer)
+ *   HI, DI    indexer heads / dim; HI in {1, 2, 4, 8}, DI in {64, 128};
+ *             Tq * HI <= 32 runs the decode indexer, larger Tq * HI (chunked
+ *             prefill) the tensor-core indexer, which supports mean pooling
+ *             only and no token_scores output
  *   lmax      cache capacity in tokens, a multiple of 128
  *   seq_lens  device int32 [B], Tq <= L_b <= lmax
  *   k, v      caches with Hkv heads of dim D; ik: 1 head of dim DI

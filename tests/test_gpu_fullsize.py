@@ -91,3 +91,21 @@ def test_full_size_decode_sampled(w, samples):
             assert (s >= 0).sum() == 16 and pos // 128 in s
     recalled = [_check_sequence(w, p, meta, b, sel_h, out_h) for b in samples]
     assert all(recalled), "planted needle blocks not all selected"
+
+
+def test_repeated_decode_is_deterministic_and_never_times_out():
+    """300 back-to-back decode steps on the 32 x 64K workload: every in-kernel wait
+    completes (status word stays 0) and every step gives the same bits."""
+    w = configs.DECODE_B32_64K
+    p, meta = _gpu_problem(w)
+    ws = msa.alloc_workspace(p)
+    out, lse, sel = msa.outputs(p)
+    msa.msa_decode(p, ws, out, lse, sel)
+    ref = out.clone()
+    acc = torch.zeros_like(out, dtype=torch.int32)
+    for _ in range(300):
+        msa.msa_decode(p, ws, out, lse, sel)
+        acc |= (out.view(torch.int32) ^ ref.view(torch.int32))
+    torch.cuda.synchronize()
+    assert int(p.status.item()) == 0
+    assert int(acc.abs().max().item()) == 0
