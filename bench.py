@@ -83,19 +83,21 @@ def aggregate_throughput(tokens_per_rank: int, world: int, seconds: float) -> fl
     return tokens_per_rank * world / seconds
 
 
-def _measured_peaks():
+def _measured_peak(key, fallback):
+    """A peak from MEASURED_PEAKS.json (measured on this machine), else the recipe's fallback."""
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        return float(d["hbm_gbs"]), "measured"
-    return 6650.0, "fallback"
+        if key in d:
+            return float(d[key]), "measured"
+    return fallback, "fallback"
 
 
-def _profile_traffic(kernel_file, workload_name):
+def _profile_traffic(kernel_file, kernel, workload_name):
     """DRAM bytes per launch from the committed ncu summary, if the kernel source is unchanged."""
     src = os.path.join(ROOT, "block_sparse_attention_10_b200", "csrc", kernel_file)
-    prof = os.path.join(ROOT, "profiles", f"index_decode_{workload_name}.md")
+    prof = os.path.join(ROOT, "profiles", f"{kernel}_{workload_name}.md")
     if not (os.path.exists(src) and os.path.exists(prof)):
         return None
     digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
@@ -223,26 +225,51 @@ def time_oracle(samples):
     return time.perf_counter() - t0
 
 
-def cpu_baseline(w, n_seq=16):
-    import oracle
-    oracle.build()
-    # 16 sequences at a time is about 10-15 s of CPU work: all 8 indexer heads over
-    # 64K keys per sequence plus attention of 32 heads over 2,048 keys
-    samples = oracle_sample(w, n_seq)
-    # the oracle parallelises over (sequence, token[, head]): run all sampled sequences in one call
+def _concat(samples):
     import oracle as O
     qs = np.concatenate([s[0] for s in samples])
     qis = np.concatenate([s[1] for s in samples])
     cat = lambda i: O.Nvfp4(np.concatenate([s[i].data for s in samples]),  # noqa: E731
                             np.concatenate([s[i].scale for s in samples]), samples[0][i].tensor_scale)
-    k, v, ik = cat(2), cat(3), cat(4)
-    lens = [s[5][0] for s in samples]
-    t0 = time.perf_counter()
-    O.decode(qs, qis, k, v, ik, lens)
-    dt = time.perf_counter() - t0
-    return {"value": n_seq * w.Tq / dt, "unit": UNIT, "cores": O.num_threads(), "kind": "oracle",
-            "sample": f"{n_seq} of the 32 sequences (full 64K context, 1 query token each), "
-                      f"oracle decode (index, pool, select, attend) in one call, {dt:.2f} s wall"}
+    return qs, qis, cat(2), cat(3), cat(4), [s[5][0] for s in samples]
+
+
+def _prefill_token_samples(w, n_tok):
+    """n_tok query tokens of sequence 0 spread over the chunk, each as a one-token step at its
+    own position (causal truncation): the oracle's inputs for a bounded prefill sample."""
+    import oracle as O
+    (q, qi, k, v, ik, lens), = oracle_sample(w, 1)
+    L = lens[0]
+    toks = [int(x) for x in np.linspace(0, w.Tq - 1, n_tok)]
+    pos = [L - w.Tq + t for t in toks]
+    rep = lambda c: O.Nvfp4(np.repeat(c.data, n_tok, 0), np.repeat(c.scale, n_tok, 0), c.tensor_scale)  # noqa
+    return (np.ascontiguousarray(q[0, toks][:, None]), np.ascontiguousarray(qi[0, toks][:, None]), rep(k), rep(v),
+            rep(ik), [p_ + 1 for p_ in pos])
+
+
+def cpu_baseline(w):
+    """The oracle as it stands on the host cores, on a bounded sample of the workload."""
+    import oracle as O
+    O.build()
+    if w.Tq * w.HI <= 32:
+        n_seq = min(w.B, 16)
+        q, qi, k, v, ik, lens = _concat(oracle_sample(w, n_seq))
+        t0 = time.perf_counter()
+        O.decode(q, qi, k, v, ik, lens)
+        dt = time.perf_counter() - t0
+        units = n_seq * w.Tq
+        sample = (f"{n_seq} of the {w.B} sequences (whole context, all {w.Tq} query token(s) each), oracle "
+                  f"decode (index, pool, select, attend) in one call, {dt:.2f} s wall")
+    else:
+        n_tok = 16
+        q, qi, k, v, ik, lens = _prefill_token_samples(w, n_tok)
+        t0 = time.perf_counter()
+        O.decode(q, qi, k, v, ik, lens)
+        dt = time.perf_counter() - t0
+        units = n_tok
+        sample = (f"{n_tok} query tokens of sequence 0 spread over the {w.Tq}-token chunk, each scored as a "
+                  f"one-token step at its own position, oracle decode in one call, {dt:.2f} s wall")
+    return {"value": units / dt, "unit": UNIT, "cores": O.num_threads(), "kind": "oracle", "sample": sample}
 
 
 def run_reference(args):
@@ -251,34 +278,45 @@ def run_reference(args):
         return
     import oracle
     oracle.build()
-    w = WORKLOAD
-    # per-step sample: one query token of one sequence; if K+W full tokens would not fit in
-    # about 150 s, each step takes the same fraction of one token's work (context prefix of
-    # that fraction for the indexer, that fraction of the query heads for attention)
-    probe = oracle_sample(w, 1)
+    w = configs.BY_NAME[args.workload]
+    prefill = w.Tq * w.HI > 32
+    # per-step sample: one sequence (all its query tokens) for decode workloads, one query token
+    # for the prefill chunk; if K+W such samples would not fit in about 150 s, every step takes the
+    # same fraction of that work (indexer over that fraction of the context, that fraction of the
+    # query heads for attention) and the value counts that fraction of the sample's tokens
+    probe = [_prefill_token_samples(w, 1)] if prefill else oracle_sample(w, 1)
+    tok = 1 if prefill else w.Tq
     t1 = time_oracle(probe)
     total = args.steps + args.warmup
     frac = min(1.0, 150.0 / max(1e-9, total * t1))
     heads = None
+    samples = probe
     if frac < 1.0:
-        heads = max(w.Hq // w.Hkv, int(round(w.Hq * frac)) // (w.Hq // w.Hkv) * (w.Hq // w.Hkv))
-        samples = oracle_sample(w, 1, key_frac=frac, heads=heads)
-    else:
-        samples = probe
+        g = w.Hq // w.Hkv
+        heads = max(g, int(round(w.Hq * frac)) // g * g)
+        q, qi, k, v, ik, lens = probe[0]
+        Ls = [max(128, int(L * frac)) for L in lens] if not prefill else lens
+        if prefill:  # shorten the token's own prefix
+            Ls = [max(1, int(L * frac)) for L in lens]
+        kvh = max(1, heads // g)
+        sub = lambda c, hh: oracle.Nvfp4(c.data[:, :hh], c.scale[:, :hh], c.tensor_scale)  # noqa: E731
+        samples = [(np.ascontiguousarray(q[:, :, :heads]), qi, sub(k, kvh), sub(v, kvh), ik, Ls)]
     for _ in range(args.warmup):
         time_oracle(samples)
     t0 = time.perf_counter()
     for _ in range(args.steps):
         time_oracle(samples)
     dt = time.perf_counter() - t0
-    value = args.steps * frac / dt
-    sample = ("one query token of sequence 0 per step (full 64K context, 32 heads)" if frac >= 1.0 else
-              f"per step {frac:.4f} of one query token's work: indexer over the first {frac:.4f} of the "
-              f"64K context, attention for {heads} of the 32 query heads; value counts {frac:.4f} token/step")
+    value = args.steps * frac * tok / dt
+    what = "one query token of sequence 0" if prefill else f"sequence 0 ({w.Tq} query token(s), whole context)"
+    sample = (f"per step: {what}, oracle decode" if frac >= 1.0 else
+              f"per step {frac:.4f} of {what}: indexer over that fraction of the context, attention for "
+              f"{heads} of the {w.Hq} query heads; the value counts {frac:.4f} of its tokens per step")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "global_batch": w.B, "seq_len": w.seq_len, "query_tokens": w.Tq},
+            "config": {"workload": w.name, "global_batch": w.B, "seq_len": w.seq_len or list(w.seq_len_range),
+                       "query_tokens": w.Tq},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -286,6 +324,32 @@ def run_reference(args):
 
 
 # ----------------------------------------------------------------------------- our arm
+
+def step_work(w, seq_lens, sel):
+    """Algorithmic bytes and flops of one msa_decode step, from the step's own selection.
+
+    index: every visible index key once (DI/2 + DI/16 bytes), 2*HI*DI flop per (token, visible key);
+    attention: K and V (2 x (D/2 + D/16) bytes per KV head) of the union over a sequence's
+    tokens of their selected visible keys; 4*D*Hq flop per (token, selected visible key)."""
+    kvb = 2 * (w.D // 2 + w.D // 16)
+    idx_bytes = idx_flops = att_bytes = att_flops = 0
+    for b, L in enumerate(seq_lens):
+        idx_bytes += L * (w.DI // 2 + w.DI // 16)
+        union = set()
+        for t in range(w.Tq):
+            pos = L - w.Tq + t
+            idx_flops += 2 * w.HI * w.DI * (pos + 1)
+            keys = 0
+            for n in sel[b, t]:
+                if n < 0:
+                    continue
+                lo, hi = int(n) * 128, min(int(n) * 128 + 128, pos + 1)
+                keys += max(0, hi - lo)
+                union.add(int(n))
+            att_flops += 4 * w.D * w.Hq * keys
+        att_bytes += sum(min(128, L - n * 128) for n in union) * kvb * w.Hkv
+    return idx_bytes, idx_flops, att_bytes, att_flops
+
 
 def run_ours(args):
     from block_sparse_attention_10_b200 import msa
@@ -299,14 +363,25 @@ def run_ours(args):
     else:
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
-    w = WORKLOAD
+    w = configs.BY_NAME[args.workload]
+    prefill = w.Tq * w.HI > 32
 
-    # each rank owns its own 32 sequences (weak scaling): seed offset by rank
+    # each rank owns its own sequences (weak scaling): rank-specific seed
     p0 = build_problem(rank_workload(w, rank), list(range(w.B)), device=dev)
-    reps = [p0] + [clone_problem(p0) for _ in range(args.replicas - 1)]
     ws_t = msa.alloc_workspace(p0)
     out, lse, sel = msa.outputs(p0)
     stream = torch.cuda.Stream()
+    msa.msa_decode(p0, ws_t, out, lse, sel)
+    torch.cuda.synchronize()
+    lens = [int(x) for x in p0.seq_lens.tolist()]
+    idx_bytes, idx_flops, att_bytes, att_flops = step_work(w, lens, sel.cpu().numpy())
+    step_bytes = idx_bytes + att_bytes
+    # rotate enough cache replicas that every step reads data no earlier step left in L2
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    cache_bytes = sum(x.numel() for c in (p0.k, p0.v, p0.ik) for x in (c.data, c.scale))
+    n_rep = args.replicas or int(min(2048, max(2, math.ceil(4 * l2 / step_bytes)),
+                                     max(2, (40 << 30) // max(1, cache_bytes))))
+    reps = [p0] + [clone_problem(p0) for _ in range(n_rep - 1)]
     torch.cuda.synchronize()
 
     def step(i, s):
@@ -316,18 +391,17 @@ def run_ours(args):
         for i in range(max(3, args.warmup)):
             step(i, stream)
     torch.cuda.synchronize()
-    # capture G steps in one graph (launch overhead off the host); replays cover K steps
-    G = math.gcd(args.steps, 50) if args.steps % 50 else 50
-    G = max(1, min(G, args.steps))
-    if args.steps % G:
-        G = 1
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        for i in range(G):
-            step(i, stream)
+    # CUDA graphs of G steps cycling through every replica; a tail graph covers K mod G
+    G = min(args.steps, max(50, n_rep))
+    graphs = []
+    for n_steps in [G] + ([args.steps % G] if args.steps % G else []):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(n_steps):
+                step(i, stream)
+        graphs.append(g)
     torch.cuda.synchronize()
-    for _ in range(2):
-        graph.replay()
+    graphs[0].replay()
     torch.cuda.synchronize()
     if ws_n > 1:
         torch.distributed.barrier()
@@ -337,7 +411,9 @@ def run_ours(args):
         with torch.cuda.stream(stream):
             e0.record(stream)
             for _ in range(args.steps // G):
-                graph.replay()
+                graphs[0].replay()
+            if len(graphs) > 1:
+                graphs[1].replay()
             e1.record(stream)
         e1.synchronize()
     torch.cuda.synchronize()
@@ -345,9 +421,9 @@ def run_ours(args):
         torch.distributed.barrier()
     ms = max_over_ranks(e0.elapsed_time(e1) / args.steps, dev)
     status = int(p0.status.item())
-    assert status == 0, f"device status word {status}"
+    assert status == 0, f"device status word {status:#x}"
 
-    # dominant kernel (indexer): per-launch CUDA events on its stream
+    # dominant kernel (the indexer): per-launch CUDA events on its stream
     nb_i = min(args.steps, 200)
     bs = torch.empty(w.B, w.Tq, p0.nbmax, dtype=torch.float32, device=dev)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nb_i)]
@@ -360,10 +436,20 @@ def run_ours(args):
             b.record(stream)
     torch.cuda.synchronize()
     idx_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
-    lens = [int(x) for x in p0.seq_lens.tolist()]
-    idx_bytes, att_bytes = _algorithmic_bytes(w, lens)
-    peak, peak_kind = _measured_peaks()
-    achieved = idx_bytes / (idx_ms * 1e-3) / 1e9
+    if prefill:
+        peak, peak_kind = _measured_peak("bf16_tflops", 1590.0)
+        achieved = idx_flops / (idx_ms * 1e-3) / 1e12
+        roof = {"kernel": "index_prefill", "bound": "tensor", "achieved": achieved, "peak": peak,
+                "peak_kind": peak_kind, "unit": "TFLOP/s", "frac": achieved / peak,
+                "algorithmic_flops_per_launch": idx_flops, "launch_ms": idx_ms,
+                "traffic": _profile_traffic("index_prefill.cu", "index_prefill", w.name)}
+    else:
+        peak, peak_kind = _measured_peak("hbm_gbs", 6650.0)
+        achieved = idx_bytes / (idx_ms * 1e-3) / 1e9
+        roof = {"kernel": "index_decode", "bound": "hbm", "achieved": achieved, "peak": peak,
+                "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                "frac_of_8tbs": achieved / CONTRACT_HBM_GBS, "algorithmic_bytes_per_launch": idx_bytes,
+                "launch_ms": idx_ms, "traffic": _profile_traffic("index_decode.cu", "index_decode", w.name)}
 
     # end to end through the public API: pinned host queries -> device, decode, output -> host
     n_e2e = min(args.steps, 200)
@@ -382,10 +468,9 @@ def run_ours(args):
             msa.msa_decode(r, ws_t, out, lse, None, stream=stream)
             hout.copy_(out, non_blocking=True)
             stream.synchronize()
-    e2e_s = (time.perf_counter() - t0) / n_e2e
+    e2e_s = max_over_ranks((time.perf_counter() - t0) / n_e2e, dev)
     h2d = hq.numel() * hq.element_size() + hqi.numel() * hqi.element_size()
     d2h = hout.numel() * hout.element_size()
-    e2e_s = max_over_ranks(e2e_s, dev)
 
     cpu = None
     if rank == 0 and ws_n == 1 and not args.no_cpu_baseline:
@@ -393,25 +478,23 @@ def run_ours(args):
 
     if rank == 0:
         value = aggregate_throughput(w.B * w.Tq, ws_n, ms * 1e-3)
-        step_bytes = idx_bytes + att_bytes
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws_n, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "nvfp4 caches, f16 tensor-core math, f32 accumulate/output",
+            "vs_baseline": None, "dtype": "nvfp4 caches, f16/bf16 tensor-core math, f32 accumulate/output",
             "data": "synthetic",
-            "config": {"workload": w.name, "global_batch": w.B * ws_n, "seq_len": w.seq_len, "query_tokens": w.Tq,
-                       "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "HI": w.HI, "DI": w.DI, "top_blocks": 16,
-                       "block_tokens": 128, "parallelism": f"replicas x{ws_n} (own sequences per GPU)",
-                       "l2": f"inputs larger than L2: {step_bytes / 1e6:.0f} MB read per step, "
-                             f"{args.replicas} rotating cache replicas of "
-                             f"{(p0.k.data.numel() + p0.k.scale.numel()) * 2 / 1e9 + (p0.ik.data.numel() + p0.ik.scale.numel()) / 1e9:.2f} GB"},
+            "config": {"workload": w.name, "global_batch": w.B * ws_n, "seq_len": w.seq_len or list(w.seq_len_range),
+                       "query_tokens": w.Tq, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "HI": w.HI, "DI": w.DI,
+                       "top_blocks": 16, "block_tokens": 128,
+                       "parallelism": f"replicas x{ws_n} (own sequences per GPU)",
+                       "l2": f"inputs larger than L2: {step_bytes / 1e6:.1f} MB read per step, {n_rep} rotating "
+                             f"cache replicas ({n_rep * step_bytes / 1e6:.0f} MB touched per cycle, L2 "
+                             f"{l2 / 1e6:.0f} MB)"},
+            "step_algorithmic_bytes": step_bytes, "step_algorithmic_flops": idx_flops + att_flops,
             "step_gbs": step_bytes / (ms * 1e-3) / 1e9,
             "step_frac_of_8tbs": step_bytes / (ms * 1e-3) / 1e9 / CONTRACT_HBM_GBS,
-            "roofline": {"kernel": "index_decode", "bound": "hbm", "achieved": achieved, "peak": peak,
-                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
-                         "frac_of_8tbs": achieved / CONTRACT_HBM_GBS,
-                         "algorithmic_bytes_per_launch": idx_bytes, "launch_ms": idx_ms,
-                         "traffic": _profile_traffic("index_decode.cu", w.name)},
+            "step_tflops": (idx_flops + att_flops) / (ms * 1e-3) / 1e12,
+            "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": {"value": aggregate_throughput(w.B * w.Tq, ws_n, e2e_s), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
@@ -419,7 +502,7 @@ def run_ours(args):
             "clocks": clk.summary(),
         }
         print(json.dumps(line), flush=True)
-    del graph
+    del graphs
     if ws_n > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
@@ -431,7 +514,8 @@ def main():
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--replicas", type=int, default=2)
+    ap.add_argument("--replicas", type=int, default=0, help="cache replicas (0: enough to defeat L2)")
+    ap.add_argument("--workload", default=WORKLOAD.name, choices=sorted(configs.BY_NAME))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.impl == "reference":

@@ -46,33 +46,37 @@ class _Nvfp4(ctypes.Structure):
 _lib = None
 
 
+def configure(L):
+    """Declare the C signatures on a loaded oracle library."""
+    L.orc_e2m1_value.restype = ctypes.c_double
+    L.orc_e2m1_value.argtypes = [ctypes.c_uint8]
+    L.orc_e4m3_value.restype = ctypes.c_double
+    L.orc_e4m3_value.argtypes = [ctypes.c_uint8]
+    L.orc_e4m3_encode.restype = ctypes.c_uint8
+    L.orc_e4m3_encode.argtypes = [ctypes.c_float]
+    L.orc_e2m1_encode.restype = ctypes.c_uint8
+    L.orc_e2m1_encode.argtypes = [ctypes.c_float]
+    L.orc_tensor_scale.restype = ctypes.c_float
+    L.orc_tensor_scale.argtypes = [ctypes.c_void_p, ctypes.c_int64]
+    L.orc_nvfp4_encode.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float,
+                                   ctypes.c_void_p, ctypes.c_void_p]
+    L.orc_nvfp4_decode.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
+                                   ctypes.c_float, ctypes.c_void_p]
+    L.orc_index.argtypes = [ctypes.c_int] * 4 + [ctypes.c_void_p] * 3 + [ctypes.POINTER(_Nvfp4), ctypes.c_int,
+                                                                          ctypes.c_void_p, ctypes.c_void_p]
+    L.orc_select.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
+                             ctypes.c_void_p]
+    L.orc_attend.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(_Nvfp4),
+                                                  ctypes.POINTER(_Nvfp4), ctypes.c_void_p, ctypes.c_double,
+                                                  ctypes.c_void_p, ctypes.c_void_p]
+    L.orc_num_threads.restype = ctypes.c_int
+    return L
+
+
 def lib():
     global _lib
     if _lib is None:
-        _lib = ctypes.CDLL(build())
-        L = _lib
-        L.orc_e2m1_value.restype = ctypes.c_double
-        L.orc_e2m1_value.argtypes = [ctypes.c_uint8]
-        L.orc_e4m3_value.restype = ctypes.c_double
-        L.orc_e4m3_value.argtypes = [ctypes.c_uint8]
-        L.orc_e4m3_encode.restype = ctypes.c_uint8
-        L.orc_e4m3_encode.argtypes = [ctypes.c_float]
-        L.orc_e2m1_encode.restype = ctypes.c_uint8
-        L.orc_e2m1_encode.argtypes = [ctypes.c_float]
-        L.orc_tensor_scale.restype = ctypes.c_float
-        L.orc_tensor_scale.argtypes = [ctypes.c_void_p, ctypes.c_int64]
-        L.orc_nvfp4_encode.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float,
-                                       ctypes.c_void_p, ctypes.c_void_p]
-        L.orc_nvfp4_decode.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int,
-                                       ctypes.c_float, ctypes.c_void_p]
-        L.orc_index.argtypes = [ctypes.c_int] * 4 + [ctypes.c_void_p] * 3 + [ctypes.POINTER(_Nvfp4), ctypes.c_int,
-                                                                              ctypes.c_void_p, ctypes.c_void_p]
-        L.orc_select.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_void_p, ctypes.c_void_p,
-                                 ctypes.c_void_p]
-        L.orc_attend.argtypes = [ctypes.c_int] * 5 + [ctypes.c_void_p, ctypes.c_void_p, ctypes.POINTER(_Nvfp4),
-                                                      ctypes.POINTER(_Nvfp4), ctypes.c_void_p, ctypes.c_double,
-                                                      ctypes.c_void_p, ctypes.c_void_p]
-        L.orc_num_threads.restype = ctypes.c_int
+        _lib = configure(ctypes.CDLL(build()))
     return _lib
 
 

@@ -57,7 +57,7 @@ def test_workspace_size_host_only(L):
 
 @pytest.mark.parametrize("field,value,code", [
     ("lmax", 4000, 1), ("B", 0, 1), ("Tq", 0, 1), ("seq_lens", None, 1), ("pool_mode", 2, 1),
-    ("D", 64, 2), ("DI", 96, 2), ("HI", 3, 2), ("Hq", 24, 2), ("Tq", 9, 2),
+    ("D", 64, 2), ("DI", 96, 2), ("HI", 3, 2), ("Hq", 24, 2), ("B", 5000, 2),
     ("q", 0x8001, 3), ("q_idx", 0x9008, 3),
 ])
 def test_decode_rejects_bad_params(L, field, value, code):
@@ -65,6 +65,15 @@ def test_decode_rejects_bad_params(L, field, value, code):
     ws = ctypes.c_void_p(0x10000)
     r = L.msa_decode(ctypes.byref(p), ws, 1 << 20, ctypes.c_void_p(0x20000), None, None, None)
     assert r == code, (field, r)
+
+
+def test_prefill_path_is_mean_pooling_only(L):
+    # Tq * HI > 32 selects the tensor-core prefill indexer, which pools by mean only
+    p = _params(Tq=9, pool_mode=1)
+    r = L.msa_decode(ctypes.byref(p), ctypes.c_void_p(0x10000), 1 << 20, ctypes.c_void_p(0x20000), None, None, None)
+    assert r == 2
+    p = _params(Tq=9)
+    assert L.msa_workspace_size(ctypes.byref(p)) > 0
 
 
 def test_bad_cache_and_workspace(L):
