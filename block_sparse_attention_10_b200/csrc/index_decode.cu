@@ -8,50 +8,51 @@
 //
 // Design (B200): the kernel is HBM-bound — it must stream every index key
 // (DI/2 + DI/16 bytes per token) exactly once for all Tq query tokens.
-//   * Persistent grid, 2 CTAs per SM.  Each CTA owns a contiguous range of
-//     (sequence, block) units; one producer lane streams each unit's NVFP4
-//     nibbles and scales (one 128-token block: 9 KB at DI = 128) into a ring
-//     of shared-memory stages with untiled bulk copies (cp.async.bulk, no
-//     multicast), signalled through mbarriers; 8 consumer warps take units
-//     round-robin.
-//   * Consumers dequantise in registers with the sm_100a converters
-//     (E2M1x2 -> f16x2, E4M3 -> f16; e2m1*e4m3 is exact in f16) and run the
-//     [16 keys x DI] x [DI x 8 queries] products on tensor cores
-//     (mma.sync m16n8k16, f32 accumulate).  The per-tensor fp32 scale is
-//     applied once, after pooling (ReLU and both pools commute with a
-//     positive scale).
+//   * 2 CTAs of 8 warps per SM; each warp owns a contiguous range of
+//     (sequence, block) units and streams them itself: its lane 0 issues
+//     untiled bulk copies (cp.async.bulk, no multicast) of 64-key half-blocks
+//     (4.5 KB at DI = 128) into the warp's private ring of shared-memory
+//     stages, two half-blocks ahead of the one being computed, each stage with
+//     its own mbarrier.  A warp only ever waits on its own stages, in order, so
+//     ~150 KB per SM are in flight while every warp computes.
+//   * Dequantisation in registers with the sm_100a converters (E2M1x2 ->
+//     f16x2, E4M3 -> f16; e2m1*e4m3 is exact in f16) feeding tensor-core
+//     mma.sync m16n8k16 ([16 keys x DI] x [DI x 8 queries], f32 accumulate).
+//     The per-tensor fp32 scale is applied once, after pooling (ReLU and both
+//     pools commute with a positive scale).
 //   * Each thread reads the 16 (DI = 128) or 8 (DI = 64) contiguous bytes of
 //     a key that its A-fragment needs: the head dim is permuted identically
-//     on the key and query side (a dot product does not depend on the order
-//     of its terms), which makes every shared-memory read a 128/64-bit
-//     conflict-free load.
+//     on the key and query side, so every shared-memory read is one 128/64-bit
+//     load.
 //   * Epilogue in registers: ReLU, head weights, sum over heads with warp
 //     shuffles, causal / length masking, block pooling, one store per
-//     (token, block).
+//     (token, block).  Full, fully visible blocks under mean pooling take a
+//     fast path that sums ReLU'd accumulators and reduces heads/rows once.
 #include "internal.h"
 #include "nvfp4_mma.cuh"
 
 namespace msa {
 namespace {
 
-constexpr int kIdxConsumers = 8;
-constexpr int kIdxThreads = 32 * (kIdxConsumers + 1);
+constexpr int kIdxWarps = 8;
+constexpr int kIdxThreads = 32 * kIdxWarps;
 constexpr int kMaxB = 4096;
+constexpr int kHalf = 64;  // keys per shared-memory stage
 
 template <int DI>
 struct IdxGeom {
     static constexpr int kRowBytes = DI / 2;
     static constexpr int kSclBytes = DI / 16;
-    static constexpr int kDataBytes = kBlock * kRowBytes;
-    static constexpr int kStageBytes = kBlock * (kRowBytes + kSclBytes);
-    static constexpr int kStages = DI == 128 ? 10 : 20;
+    static constexpr int kDataBytes = kHalf * kRowBytes;
+    static constexpr int kStageBytes = kHalf * (kRowBytes + kSclBytes);
+    static constexpr int kStages = DI == 128 ? 3 : 6;  // per warp: 13.5 KB either way
     static constexpr int kKSteps = DI / 16;
     static constexpr int kPairs = DI / 8;  // f16x2 pairs of q per thread
 };
 
 template <int DI>
 constexpr size_t idx_smem_bytes(int B) {
-    return (size_t)IdxGeom<DI>::kStages * IdxGeom<DI>::kStageBytes + 2 * IdxGeom<DI>::kStages * sizeof(uint64_t) +
+    return (size_t)kIdxWarps * IdxGeom<DI>::kStages * (IdxGeom<DI>::kStageBytes + sizeof(uint64_t)) +
            (size_t)(2 * B + 2) * sizeof(int);
 }
 
@@ -73,22 +74,23 @@ template <int DI, int HI, int NT>
 __global__ void __launch_bounds__(kIdxThreads, 2)
     index_decode_kernel(const Problem p, float* __restrict__ block_scores, float* __restrict__ token_scores) {
     using G = IdxGeom<DI>;
-    constexpr int S = G::kStages;
+    constexpr int R = G::kStages;
     constexpr int KS = G::kKSteps;
     constexpr int TPN = HI == 1 ? 2 : 1;  // tokens per thread per n-tile
 
     extern __shared__ __align__(128) uint8_t smem[];
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * G::kStageBytes);
-    uint64_t* empty = full + S;
-    int* prefix = reinterpret_cast<int*>(empty + S);  // [B + 1] units before sequence b
-    int* lens = prefix + (p.B + 1);                   // [B] clamped lengths
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kIdxWarps * R * G::kStageBytes);
+    int* prefix = reinterpret_cast<int*>(bars + kIdxWarps * R);  // [B + 1] units before sequence b
+    int* lens = prefix + (p.B + 1);                               // [B] clamped lengths
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 2, c = lane & 3;
     const int B = p.B, Tq = p.Tq;
     const int NQ = Tq * HI;
+    uint8_t* my_stages = smem + warp * R * G::kStageBytes;
+    uint64_t* my_bars = bars + warp * R;
 
     pdl_wait();
-
     if (warp == 0) {
         int carry = 0;
         if (lane == 0) prefix[0] = 0;
@@ -109,95 +111,69 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
             if (b < B) prefix[b + 1] = carry + x;
             carry += __shfl_sync(0xffffffffu, x, 31);
         }
-        if (lane == 0) {
-            for (int s = 0; s < S; ++s) {
-                mbar_init(&full[s], 1);
-                mbar_init(&empty[s], 1);
-            }
-            fence_mbar_init();
-        }
+    }
+    if (lane == 0) {
+        for (int s = 0; s < R; ++s) mbar_init(&my_bars[s], 1);
+        fence_mbar_init();
     }
     __syncthreads();
     pdl_launch_dependents();
 
-    const int64_t U = prefix[B];
-    const int64_t u_begin = U * blockIdx.x / gridDim.x;
-    const int nu = (int)(U * (blockIdx.x + 1) / gridDim.x - u_begin);
-
-    if (warp == 0) {
-        // ------------------------------------------------------------------ producer
-        if (lane == 0) {
-            int b = 0;
-            int k = 0;
-            bool ok = true;
-            for (; k < nu; ++k) {
-                const int s = k % S;
-                const uint32_t round = (uint32_t)(k / S);
-                if (round > 0 && !mbar_wait(&empty[s], (round - 1) & 1u)) {
-                    set_status(p.status, MSA_STATUS_TIMEOUT | MSA_STATUS_AT_INDEX_PRODUCER);
-                    ok = false;
-                    break;
-                }
-                const int64_t u = u_begin + k;
-                while (prefix[b + 1] <= u) ++b;
-                const int64_t n = u - prefix[b];
-                const int valid = (int)min64(kBlock, lens[b] - n * kBlock);
-                const int rows = (valid + 15) & ~15;
-                const uint32_t db = (uint32_t)(rows * G::kRowBytes), sb = (uint32_t)(rows * G::kSclBytes);
-                const int64_t row0 = (int64_t)b * p.lmax + n * kBlock;
-                uint8_t* st = smem + (size_t)s * G::kStageBytes;
-                mbar_arrive_expect_tx(&full[s], db + sb);
-                bulk_g2s(st, p.ik.data + row0 * G::kRowBytes, db, &full[s]);
-                bulk_g2s(st + G::kDataBytes, p.ik.scale + row0 * G::kSclBytes, sb, &full[s]);
-            }
-            // drain: never leave with copies in flight into this CTA's shared memory
-            const int issued = k;
-            for (int j = max(0, issued - S); j < issued; ++j) {
-                if (!mbar_wait(&full[j % S], (uint32_t)(j / S) & 1u)) {
-                    set_status(p.status, MSA_STATUS_TIMEOUT | MSA_STATUS_AT_INDEX_DRAIN);
-                    break;
-                }
-            }
-            (void)ok;
-        }
-        return;
-    }
-
-    // ---------------------------------------------------------------------- consumers
-    const int cw = warp - 1;
-    const int g = lane >> 2, c = lane & 3;
     const float s_t = p.ik.s_t;
-
     // blocks past a sequence's length score -inf (no unit covers them)
     {
         const int64_t total = (int64_t)B * Tq * p.nbmax;
-        const int64_t stride = (int64_t)gridDim.x * kIdxConsumers * 32;
-        for (int64_t i = (int64_t)blockIdx.x * kIdxConsumers * 32 + cw * 32 + lane; i < total; i += stride) {
+        const int64_t stride = (int64_t)gridDim.x * kIdxThreads;
+        for (int64_t i = (int64_t)blockIdx.x * kIdxThreads + threadIdx.x; i < total; i += stride) {
             const int64_t n = i % p.nbmax;
             const int b = (int)(i / (p.nbmax * Tq));
             if (n >= prefix[b + 1] - prefix[b]) block_scores[i] = -INFINITY;
         }
     }
 
+    // this warp's contiguous range of units
+    const int64_t U = prefix[B];
+    const int64_t Wt = (int64_t)gridDim.x * kIdxWarps;
+    const int64_t gw = (int64_t)blockIdx.x * kIdxWarps + warp;
+    const int64_t u_begin = U * gw / Wt, u_end = U * (gw + 1) / Wt;
+
+    // issue side: walks the same (unit, half) sequence as the compute side, R halves ahead
+    int64_t iu = u_begin;
+    int ih = 0, ib = 0;
+    uint32_t slot_issued = 0;
+    auto issue_upto = [&](uint32_t limit) {
+        while (slot_issued < limit && iu < u_end) {
+            while (prefix[ib + 1] <= iu) ++ib;
+            const int64_t n = iu - prefix[ib];
+            const int valid = (int)min64(kBlock, lens[ib] - n * kBlock) - ih * kHalf;
+            if (valid > 0) {
+                if (lane == 0) {
+                    const int rows = (min(valid, kHalf) + 15) & ~15;
+                    const int s = (int)(slot_issued % R);
+                    const int64_t row0 = (int64_t)ib * p.lmax + n * kBlock + ih * kHalf;
+                    uint8_t* st = my_stages + s * G::kStageBytes;
+                    const uint32_t db = (uint32_t)(rows * G::kRowBytes), sb = (uint32_t)(rows * G::kSclBytes);
+                    mbar_arrive_expect_tx(&my_bars[s], db + sb);
+                    bulk_g2s(st, p.ik.data + row0 * G::kRowBytes, db, &my_bars[s]);
+                    bulk_g2s(st + G::kDataBytes, p.ik.scale + row0 * G::kSclBytes, sb, &my_bars[s]);
+                }
+                ++slot_issued;
+            }
+            if (++ih == 2) {
+                ih = 0;
+                ++iu;
+            }
+        }
+    };
+
     uint32_t qf[NT][KS][2];
     float wq[NT][2];
     int cur_b = -1;
     int b = 0;
+    uint32_t slot = 0;
+    bool failed = false;
 
-    for (int k = cw; k < nu; k += kIdxConsumers) {
-        const int s = k % S;
-        const uint32_t round = (uint32_t)(k / S);
-        // Units go to consumers round-robin, so this warp may reach stage s while the
-        // stage's previous copy (unit k - S, another warp's) is still landing, and a parity
-        // wait on full[s] cannot tell "phase round - 1 still open" from "phase round
-        // complete".  The stage's empty barrier settles it: its phase round - 1 completes
-        // only after that earlier unit was consumed (so full[s] is past phase round - 1),
-        // and it cannot move past phase round before this warp releases the stage.
-        if ((round > 0 && !mbar_wait(&empty[s], (round - 1) & 1u)) || !mbar_wait(&full[s], round & 1u)) {
-            set_status(p.status, MSA_STATUS_TIMEOUT | MSA_STATUS_AT_INDEX_CONSUMER);
-            break;
-        }
-        const int64_t u = u_begin + k;
+    for (int64_t u = u_begin; u < u_end && !failed; ++u) {
         while (prefix[b + 1] <= u) ++b;
         const int64_t n = u - prefix[b];
         const int L = lens[b];
@@ -237,28 +213,46 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
             }
         }
 
-        const uint8_t* sd = smem + (size_t)s * G::kStageBytes;
-        const uint8_t* ss = sd + G::kDataBytes;
         // fast path: a full block that every query token sees entirely, mean pooling, no
         // per-token output.  The pooled mean is linear, so ReLU'd products are summed per
         // accumulator element over all tiles and reduced over heads and rows once per block.
         const bool fast = valid == kBlock && kbase + (kBlock - 1) <= (int64_t)L - Tq && p.pool_mode == 0 &&
                           token_scores == nullptr;
+        // acquire the next half-block of this warp's stream (in order), or flag a timeout
+        auto acquire = [&](int& s_out) -> bool {
+            issue_upto(slot + R);
+            const int s = (int)(slot % R);
+            if (!mbar_wait(&my_bars[s], (slot / R) & 1u)) {
+                if (lane == 0) set_status(p.status, MSA_STATUS_TIMEOUT | MSA_STATUS_AT_INDEX_CONSUMER);
+                failed = true;
+                return false;
+            }
+            ++slot;
+            s_out = s;
+            return true;
+        };
+
         if (fast) {
             float colsum[NT][4];
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) colsum[nt][0] = colsum[nt][1] = colsum[nt][2] = colsum[nt][3] = 0.0f;
-#pragma unroll 2
-            for (int ti = 0; ti < kBlock / 16; ++ti) {
-                float acc[NT][4];
-                nvfp4_tile_mma<DI, NT>(sd, ss, ti * 16 + g, c, qf, acc);
+            for (int half = 0; half < 2; ++half) {
+                int s;
+                if (!acquire(s)) break;
+                const uint8_t* sd = my_stages + s * G::kStageBytes;
+                const uint8_t* ss = sd + G::kDataBytes;
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
+                for (int ti = 0; ti < kHalf / 16; ++ti) {
+                    float acc[NT][4];
+                    nvfp4_tile_mma<DI, NT>(sd, ss, ti * 16 + g, c, qf, acc);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) colsum[nt][e] += fmaxf(acc[nt][e], 0.0f);
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) colsum[nt][e] += fmaxf(acc[nt][e], 0.0f);
+                }
+                __syncwarp();  // every lane is done reading stage s before it is refilled
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
+            if (failed) break;
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 // rows g and g+8 of the same column, then the head weights
@@ -292,57 +286,65 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int e = 0; e < TPN; ++e) pool[nt][e] = p.pool_mode == 1 ? -INFINITY : 0.0f;
-
-        const int ntiles = (valid + 15) >> 4;
-        for (int ti = 0; ti < ntiles; ++ti) {
-            const int r0 = ti * 16 + g, r1 = r0 + 8;
-            float acc[NT][4];
-            nvfp4_tile_mma<DI, NT>(sd, ss, r0, c, qf, acc);
-            // epilogue: ReLU * w, sum over heads, mask, pool
-            const int64_t j0 = kbase + r0, j1 = kbase + r1;
+        for (int half = 0; half < 2; ++half) {
+            const int hvalid = min(valid - half * kHalf, kHalf);
+            if (hvalid <= 0) break;
+            int s;
+            if (!acquire(s)) break;
+            const uint8_t* sd = my_stages + s * G::kStageBytes;
+            const uint8_t* ss = sd + G::kDataBytes;
+            const int64_t hbase = kbase + half * kHalf;
+            const int ntiles = (hvalid + 15) >> 4;
+            for (int ti = 0; ti < ntiles; ++ti) {
+                const int r0 = ti * 16 + g, r1 = r0 + 8;
+                float acc[NT][4];
+                nvfp4_tile_mma<DI, NT>(sd, ss, r0, c, qf, acc);
+                // epilogue: ReLU * w, sum over heads, mask, pool
+                const int64_t j0 = hbase + r0, j1 = hbase + r1;
 #pragma unroll
-            for (int nt = 0; nt < NT; ++nt) {
-                float v[2][2];  // [row][col]
+                for (int nt = 0; nt < NT; ++nt) {
+                    float v[2][2];  // [row][col]
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    v[0][e] = fmaxf(acc[nt][e], 0.0f) * wq[nt][e];
-                    v[1][e] = fmaxf(acc[nt][2 + e], 0.0f) * wq[nt][e];
-                }
-                float tsum[2][TPN];
-#pragma unroll
-                for (int rr = 0; rr < 2; ++rr) {
-                    if constexpr (HI == 1) {
-                        tsum[rr][0] = v[rr][0];
-                        tsum[rr][TPN - 1] = v[rr][1];
-                    } else {
-                        float x = v[rr][0] + v[rr][1];
-                        if constexpr (HI >= 4) x += __shfl_xor_sync(0xffffffffu, x, 1);
-                        if constexpr (HI >= 8) x += __shfl_xor_sync(0xffffffffu, x, 2);
-                        tsum[rr][0] = x;
+                    for (int e = 0; e < 2; ++e) {
+                        v[0][e] = fmaxf(acc[nt][e], 0.0f) * wq[nt][e];
+                        v[1][e] = fmaxf(acc[nt][2 + e], 0.0f) * wq[nt][e];
                     }
-                }
+                    float tsum[2][TPN];
 #pragma unroll
-                for (int e = 0; e < TPN; ++e) {
-                    const int t = token_of<HI>(nt, c, e);
-                    const int64_t pos = (int64_t)L - Tq + t;
-                    const bool vis0 = t < Tq && j0 <= pos, vis1 = t < Tq && j1 <= pos;
-                    const float x0 = vis0 ? tsum[0][e] : 0.0f, x1 = vis1 ? tsum[1][e] : 0.0f;
-                    if (p.pool_mode == 1) {
-                        if (vis0) pool[nt][e] = fmaxf(pool[nt][e], x0);
-                        if (vis1) pool[nt][e] = fmaxf(pool[nt][e], x1);
-                    } else {
-                        pool[nt][e] += x0 + x1;
+                    for (int rr = 0; rr < 2; ++rr) {
+                        if constexpr (HI == 1) {
+                            tsum[rr][0] = v[rr][0];
+                            tsum[rr][TPN - 1] = v[rr][1];
+                        } else {
+                            float x = v[rr][0] + v[rr][1];
+                            if constexpr (HI >= 4) x += __shfl_xor_sync(0xffffffffu, x, 1);
+                            if constexpr (HI >= 8) x += __shfl_xor_sync(0xffffffffu, x, 2);
+                            tsum[rr][0] = x;
+                        }
                     }
-                    if (token_scores != nullptr && token_owner<HI>(c)) {
-                        float* ts = token_scores + ((int64_t)b * Tq + t) * p.lmax;
-                        if (vis0) ts[j0] = x0 * s_t;
-                        if (vis1) ts[j1] = x1 * s_t;
+#pragma unroll
+                    for (int e = 0; e < TPN; ++e) {
+                        const int t = token_of<HI>(nt, c, e);
+                        const int64_t pos = (int64_t)L - Tq + t;
+                        const bool vis0 = t < Tq && j0 <= pos, vis1 = t < Tq && j1 <= pos;
+                        const float x0 = vis0 ? tsum[0][e] : 0.0f, x1 = vis1 ? tsum[1][e] : 0.0f;
+                        if (p.pool_mode == 1) {
+                            if (vis0) pool[nt][e] = fmaxf(pool[nt][e], x0);
+                            if (vis1) pool[nt][e] = fmaxf(pool[nt][e], x1);
+                        } else {
+                            pool[nt][e] += x0 + x1;
+                        }
+                        if (token_scores != nullptr && token_owner<HI>(c)) {
+                            float* ts = token_scores + ((int64_t)b * Tq + t) * p.lmax;
+                            if (vis0) ts[j0] = x0 * s_t;
+                            if (vis1) ts[j1] = x1 * s_t;
+                        }
                     }
                 }
             }
+            __syncwarp();  // every lane is done reading stage s before it is refilled
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);
+        if (failed) break;
 
         // pool across the 8 row groups and store one score per (token, block)
 #pragma unroll
@@ -366,6 +368,12 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
             }
         }
     }
+    // never leave with copies in flight into this warp's stages
+    for (uint32_t j = slot; j < slot_issued; ++j)
+        if (!mbar_wait(&my_bars[j % R], (j / R) & 1u)) {
+            if (lane == 0) set_status(p.status, MSA_STATUS_TIMEOUT | MSA_STATUS_AT_INDEX_DRAIN);
+            break;
+        }
 }
 
 template <int DI, int HI, int NT>

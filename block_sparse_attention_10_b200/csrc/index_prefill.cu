@@ -279,6 +279,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     }
                     tcgen05_fence_after();
                     const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * kPfKeys + hb * kBlock);
+                    // ReLU-sum over the visible columns: 4 independent packed accumulators
+                    float2 acc2[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
                     for (int c4 = 0; c4 < kBlock / 32; ++c4) {
                         float v[32];
@@ -286,13 +288,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                         tmem_wait_ld();
                         if (cnt >= (c4 + 1) * 32) {
 #pragma unroll
-                            for (int i = 0; i < 32; ++i) sum += fmaxf(v[i], 0.0f);
+                            for (int i = 0; i < 16; ++i)
+                                acc2[i & 3] = add_f32x2(acc2[i & 3], make_float2(fmaxf(v[2 * i], 0.0f), fmaxf(v[2 * i + 1], 0.0f)));
                         } else {
 #pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                if (c4 * 32 + i < cnt) sum += fmaxf(v[i], 0.0f);
+                            for (int i = 0; i < 16; ++i) {
+                                const int col = c4 * 32 + 2 * i;
+                                acc2[i & 3] = add_f32x2(acc2[i & 3], make_float2(col < cnt ? fmaxf(v[2 * i], 0.0f) : 0.0f,
+                                                                                col + 1 < cnt ? fmaxf(v[2 * i + 1], 0.0f) : 0.0f));
+                            }
                         }
                     }
+                    sum = ((acc2[0].x + acc2[0].y) + (acc2[1].x + acc2[1].y)) + ((acc2[2].x + acc2[2].y) + (acc2[3].x + acc2[3].y));
                     tcgen05_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&t_empty[buf]);

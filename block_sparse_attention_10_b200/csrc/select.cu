@@ -7,18 +7,19 @@
 // min(15, r) other blocks under the total order (score desc, index asc); the
 // list is written ascending and padded with -1.
 //
-// One warp per (sequence, query token).  Each candidate becomes a 64-bit key
-// (order-preserving bits of the fp32 score, then the inverted block index),
-// so "best" is a plain maximum and ties go to the lower index; 15 rounds of
-// "largest key below the previous winner" with two 32-bit warp reductions
-// (redux.sync) each.  The first 512 candidates of a row live in registers.
-// Deterministic and independent of the warp layout.
+// One CTA of 256 threads per (sequence, query token).  Each candidate becomes a
+// 64-bit key (order-preserving bits of the fp32 score, then the inverted block
+// index), so "best" is a plain maximum and ties go to the lower index; 15 rounds
+// of "largest key below the previous winner".  Rows of up to 4,096 blocks live
+// in registers.  Deterministic and independent of the thread layout.
 #include "internal.h"
 
 namespace msa {
 namespace {
 
-constexpr int kSelWarps = 4;
+constexpr int kSelThreads = 256;
+constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kPer = 16;  // candidates per thread held in registers (rows of <= 4,096 blocks)
 
 __device__ __forceinline__ uint64_t rank_key(float s, int64_t n) {
     uint32_t u = __float_as_uint(s);
@@ -26,14 +27,25 @@ __device__ __forceinline__ uint64_t rank_key(float s, int64_t n) {
     return ((uint64_t)u << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)n);
 }
 
-__global__ void __launch_bounds__(32 * kSelWarps)
+__device__ __forceinline__ uint64_t warp_max64(uint64_t v) {
+    const uint32_t hi = __reduce_max_sync(0xffffffffu, (uint32_t)(v >> 32));
+    const uint32_t lo = __reduce_max_sync(0xffffffffu, (uint32_t)(v >> 32) == hi ? (uint32_t)v : 0u);
+    return ((uint64_t)hi << 32) | lo;
+}
+
+// One CTA per (sequence, query token).  Thread i holds candidates i, i + 256, ... of the
+// row in registers; each of the 15 rounds takes the largest key below the previous winner
+// with a warp reduction (redux.sync) and one exchange of 8 warp maxima through shared
+// memory (double-buffered, one __syncthreads per round).
+__global__ void __launch_bounds__(kSelThreads)
     select_kernel(const Problem p, const float* __restrict__ block_scores, int32_t* __restrict__ sel,
                   int32_t* __restrict__ sel_copy) {
+    __shared__ uint64_t wmax[2][kSelWarps];
+    __shared__ int chosen[kTopK];
     pdl_wait();
     pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t row = (int64_t)blockIdx.x * kSelWarps + warp;
-    if (row >= (int64_t)p.B * p.Tq) return;
+    const int64_t row = blockIdx.x;
     const int b = (int)(row / p.Tq), t = (int)(row % p.Tq);
     const int64_t L = clamp_len(p.seq_lens[b], p.Tq, p.lmax, nullptr);
     const int64_t pos = L - p.Tq + t;
@@ -42,12 +54,78 @@ __global__ void __launch_bounds__(32 * kSelWarps)
     const float* s = block_scores + row * p.nbmax;
     const int want = (int)min64(kTopK - 1, nvis - 1);
 
-    // The first 512 candidates stay in registers (16 per lane, loads issued together);
-    // longer rows stream the rest from L1/L2 in chunks of 512 every round.
-    constexpr int kPer = 16;
     uint64_t k0[kPer];
 #pragma unroll
     for (int j = 0; j < kPer; ++j) {
+        const int64_t n = (int64_t)j * kSelThreads + threadIdx.x;
+        k0[j] = (n < nvis && n != r) ? rank_key(__ldg(s + n), n) : 0ull;
+    }
+    uint64_t prev = ~0ull;
+    for (int k = 0; k < want; ++k) {
+        uint64_t best = 0;
+#pragma unroll
+        for (int j = 0; j < kPer; ++j)
+            if (k0[j] < prev && k0[j] > best) best = k0[j];
+        for (int64_t base = (int64_t)kPer * kSelThreads; base < nvis; base += (int64_t)kPer * kSelThreads) {
+#pragma unroll 4
+            for (int j = 0; j < kPer; ++j) {
+                const int64_t n = base + (int64_t)j * kSelThreads + threadIdx.x;
+                const uint64_t key = (n < nvis && n != r) ? rank_key(__ldg(s + n), n) : 0ull;
+                if (key < prev && key > best) best = key;
+            }
+        }
+        best = warp_max64(best);
+        if (lane == 0) wmax[k & 1][warp] = best;
+        __syncthreads();
+        uint64_t m = 0;
+#pragma unroll
+        for (int w = 0; w < kSelWarps; ++w) m = wmax[k & 1][w] > m ? wmax[k & 1][w] : m;
+        prev = m;
+        if (threadIdx.x == 0) chosen[k] = (int)(0xFFFFFFFFu - (uint32_t)m);
+    }
+    if (threadIdx.x == 0) chosen[want] = (int)r;
+    __syncthreads();
+    // ascending order: rank = number of smaller ids
+    const int nsel = want + 1;
+    if (threadIdx.x < kTopK) {
+        int32_t* out = sel + row * kTopK;
+        int32_t* o2 = sel_copy ? sel_copy + row * kTopK : nullptr;
+        if (threadIdx.x < nsel) {
+            const int mine = chosen[threadIdx.x];
+            int rank = 0;
+            for (int i = 0; i < nsel; ++i) rank += chosen[i] < mine ? 1 : 0;
+            out[rank] = mine;
+            if (o2) o2[rank] = mine;
+        } else {
+            out[threadIdx.x] = -1;
+            if (o2) o2[threadIdx.x] = -1;
+        }
+    }
+}
+
+// Short rows (<= 1,024 blocks): one warp per (sequence, query token), 32
+// candidates per lane in registers, 15 rounds of two redux.sync each.
+constexpr int kWarpRows = 4;
+constexpr int kWarpPer = 32;
+
+__global__ void __launch_bounds__(32 * kWarpRows)
+    select_warp_kernel(const Problem p, const float* __restrict__ block_scores, int32_t* __restrict__ sel,
+                       int32_t* __restrict__ sel_copy) {
+    pdl_wait();
+    pdl_launch_dependents();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t row = (int64_t)blockIdx.x * kWarpRows + warp;
+    if (row >= (int64_t)p.B * p.Tq) return;
+    const int b = (int)(row / p.Tq), t = (int)(row % p.Tq);
+    const int64_t L = clamp_len(p.seq_lens[b], p.Tq, p.lmax, nullptr);
+    const int64_t pos = L - p.Tq + t;
+    const int64_t r = pos / kBlock;
+    const int64_t nvis = r + 1;
+    const float* s = block_scores + row * p.nbmax;
+    const int want = (int)min64(kTopK - 1, nvis - 1);
+    uint64_t k0[kWarpPer];
+#pragma unroll
+    for (int j = 0; j < kWarpPer; ++j) {
         const int64_t n = j * 32 + lane;
         k0[j] = (n < nvis && n != r) ? rank_key(__ldg(s + n), n) : 0ull;
     }
@@ -56,36 +134,23 @@ __global__ void __launch_bounds__(32 * kSelWarps)
     for (int k = 0; k < want; ++k) {
         uint64_t best = 0;
 #pragma unroll
-        for (int j = 0; j < kPer; ++j)
+        for (int j = 0; j < kWarpPer; ++j)
             if (k0[j] < prev && k0[j] > best) best = k0[j];
-        for (int64_t base = 32 * kPer; base < nvis; base += 32 * kPer) {
-#pragma unroll
-            for (int j = 0; j < kPer; ++j) {
-                const int64_t n = base + j * 32 + lane;
-                const uint64_t key = (n < nvis && n != r) ? rank_key(__ldg(s + n), n) : 0ull;
-                if (key < prev && key > best) best = key;
-            }
-        }
-        const uint32_t hi = __reduce_max_sync(0xffffffffu, (uint32_t)(best >> 32));
-        const uint32_t lo = __reduce_max_sync(0xffffffffu, (uint32_t)(best >> 32) == hi ? (uint32_t)best : 0u);
-        prev = ((uint64_t)hi << 32) | lo;
-        if (lane == k) mine = (int)(0xFFFFFFFFu - lo);
+        prev = warp_max64(best);
+        if (lane == k) mine = (int)(0xFFFFFFFFu - (uint32_t)prev);
     }
     if (lane == want) mine = (int)r;
     const int nsel = want + 1;
-    // ascending order: rank = number of smaller ids
     int rank = 0;
-    for (int i = 0; i < nsel; ++i) {
-        const int other = __shfl_sync(0xffffffffu, mine, i);
-        rank += (other < mine) ? 1 : 0;
-    }
+    for (int i = 0; i < nsel; ++i) rank += (__shfl_sync(0xffffffffu, mine, i) < mine) ? 1 : 0;
     int32_t* out = sel + row * kTopK;
-    if (lane < nsel) out[rank] = mine;
-    else if (lane < kTopK) out[lane] = -1;
-    if (sel_copy != nullptr) {
-        int32_t* o2 = sel_copy + row * kTopK;
-        if (lane < nsel) o2[rank] = mine;
-        else if (lane < kTopK) o2[lane] = -1;
+    int32_t* o2 = sel_copy ? sel_copy + row * kTopK : nullptr;
+    if (lane < nsel) {
+        out[rank] = mine;
+        if (o2) o2[rank] = mine;
+    } else if (lane < kTopK) {
+        out[lane] = -1;
+        if (o2) o2[lane] = -1;
     }
 }
 
@@ -94,16 +159,20 @@ __global__ void __launch_bounds__(32 * kSelWarps)
 int launch_select(const Problem& p, const float* block_scores, int32_t* sel, int32_t* sel_copy, bool pdl,
                   cudaStream_t st) {
     const int64_t rows = (int64_t)p.B * p.Tq;
+    if (rows > 0x7FFFFFFFll) return MSA_EUNSUPPORTED;
+    const bool short_rows = p.nbmax <= 32 * kWarpPer;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)((rows + kSelWarps - 1) / kSelWarps));
-    cfg.blockDim = dim3(32 * kSelWarps);
+    cfg.gridDim = dim3(short_rows ? (unsigned)((rows + kWarpRows - 1) / kWarpRows) : (unsigned)rows);
+    cfg.blockDim = dim3(short_rows ? 32 * kWarpRows : kSelThreads);
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, select_kernel, p, block_scores, sel, sel_copy) != cudaSuccess) return MSA_ECUDA;
+    const cudaError_t e = short_rows ? cudaLaunchKernelEx(&cfg, select_warp_kernel, p, block_scores, sel, sel_copy)
+                                     : cudaLaunchKernelEx(&cfg, select_kernel, p, block_scores, sel, sel_copy);
+    if (e != cudaSuccess) return MSA_ECUDA;
     return MSA_OK;
 }
 
