@@ -423,19 +423,31 @@ def run_ours(args):
     status = int(p0.status.item())
     assert status == 0, f"device status word {status:#x}"
 
-    # dominant kernel (the indexer): per-launch CUDA events on its stream
-    nb_i = min(args.steps, 200)
+    # dominant kernel (the indexer) alone: a CUDA graph of back-to-back launches on its stream,
+    # CUDA events around the replays (no host launch gaps inside the timed region)
+    nb_i = max(1, min(args.steps, 50))
     bs = torch.empty(w.B, w.Tq, p0.nbmax, dtype=torch.float32, device=dev)
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nb_i)]
     with torch.cuda.stream(stream):
-        for i in range(5):
+        for i in range(3):
             msa.msa_index(reps[i % len(reps)], bs, None, stream=stream)
-        for i, (a, b) in enumerate(evs):
-            a.record(stream)
-            msa.msa_index(reps[i % len(reps)], bs, None, stream=stream)
-            b.record(stream)
     torch.cuda.synchronize()
-    idx_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    gi = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gi, stream=stream):
+        for i in range(nb_i):
+            msa.msa_index(reps[i % len(reps)], bs, None, stream=stream)
+    torch.cuda.synchronize()
+    gi.replay()
+    torch.cuda.synchronize()
+    ia, ib_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_rep_i = max(1, min(20, args.steps // nb_i))
+    with torch.cuda.stream(stream):
+        ia.record(stream)
+        for _ in range(n_rep_i):
+            gi.replay()
+        ib_.record(stream)
+    torch.cuda.synchronize()
+    idx_ms = ia.elapsed_time(ib_) / (n_rep_i * nb_i)
+    del gi
     if prefill:
         peak, peak_kind = _measured_peak("bf16_tflops", 1590.0)
         achieved = idx_flops / (idx_ms * 1e-3) / 1e12

@@ -8,15 +8,16 @@
 //
 // Design (B200): one thread-block cluster of 4 CTAs x 4 warps per
 // (sequence, query token, KV head): each of the 16 warps takes one selected
-// block (split-K over the <= 16 blocks).  Each warp brings its whole block (K
-// and V nibbles + scales of up to 128 keys, 18 KB) into its own shared-memory
-// stage with four untiled bulk copies (cp.async.bulk, no multicast) on one
-// mbarrier, so every selected byte is requested at kernel start.  Then:
+// block (split-K over the <= 16 blocks).  Each warp streams its block as four
+// 32-key quarters (K and V nibbles + scales, 4.5 KB each) through a private
+// 2-stage shared-memory ring with untiled bulk copies (cp.async.bulk, no
+// multicast), so the next quarter lands while the current one is computed;
+// 37 KB of shared memory and <= 128 registers per CTA let 4 CTAs (16 warps)
+// share an SM and the whole 32 x 64K decode grid run in one wave.  Per quarter:
 //   S^T = K Q^T    mma m16n8k16, A = dequantised K (exact f16, 16 keys),
 //                  B = the G query heads of this KV head (8 columns) — the
 //                  same tile routine as the indexer, no padded rows;
-//   softmax        once per block (max over all its keys, exp2 domain), no
-//                  per-tile rescaling;
+//   softmax        online over quarters (exp2 domain, fp32);
 //   O^T += V^T P^T mma m16n8k16, A = dequantised V, B = P^T obtained from the
 //                  S^T accumulators by one movmatrix (8x8 transpose) per 8 keys;
 //                  output tile [128 dims x 8 heads], no padded rows.
@@ -28,6 +29,7 @@
 
 #include "internal.h"
 #include "nvfp4_mma.cuh"
+#include "select_row.cuh"
 
 namespace msa {
 namespace {
@@ -38,29 +40,38 @@ constexpr int kAttWarps = 4;
 constexpr int kAttCluster = 4;
 constexpr int kAttThreads = 32 * kAttWarps;
 constexpr int kD = 128;
+constexpr int64_t kFusedSelectMaxBlocks = 1024;  // rows one warp selects from registers
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-// Per-warp shared-memory stage: one 128-key block of one KV head.
-constexpr int kKData = kBlock * 64, kKScale = kBlock * 8;
-constexpr int kStage = 2 * (kKData + kKScale);  // 18 KB
-constexpr size_t kAttSmem = (size_t)kAttWarps * kStage + kAttWarps * sizeof(uint64_t) + 2 * 8 * sizeof(float);
+// Per-warp ring of 2 shared-memory stages, each one 32-key quarter of the warp's
+// block (K and V nibbles + scales of one KV head, 4.5 KB).
+constexpr int kQuarter = 32;
+constexpr int kKData = kQuarter * 64, kKScale = kQuarter * 8;
+constexpr int kStage = 2 * (kKData + kKScale);  // 4.5 KB
+constexpr int kWarpSmem = 2 * kStage;           // 9 KB: also holds the warp's partial O (4 KB) at the end
+constexpr size_t kAttSmem = (size_t)kAttWarps * kWarpSmem + 2 * kAttWarps * sizeof(uint64_t) + 2 * 8 * sizeof(float);
 
-template <int G>
-__global__ void __cluster_dims__(kAttCluster, 1, 1) __launch_bounds__(kAttThreads, 3)
-    attend_kernel(const Problem p, const int32_t* __restrict__ sel, float* __restrict__ out,
-                  float* __restrict__ lse) {
+// FUSED: the CTA first selects its row's blocks from the pooled scores (warp 0,
+// rows of <= 1,024 blocks) instead of reading a selection written by select.cu.
+template <int G, bool FUSED>
+__global__ void __cluster_dims__(kAttCluster, 1, 1) __launch_bounds__(kAttThreads, 4)
+    attend_kernel(const Problem p, const int32_t* __restrict__ sel, const float* __restrict__ block_scores,
+                  int32_t* __restrict__ sel_out, float* __restrict__ out, float* __restrict__ lse) {
     extern __shared__ __align__(128) uint8_t smem[];
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kAttWarps * kStage);
-    float* cM = reinterpret_cast<float*>(bars + kAttWarps);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kAttWarps * kWarpSmem);  // [warp][2]
+    float* cM = reinterpret_cast<float*>(bars + 2 * kAttWarps);
     float* cL = cM + 8;
     __shared__ float sM[kAttWarps][8], sL[kAttWarps][8];
+    __shared__ int sh_sel[kTopK];
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, c = lane & 3;
-    uint8_t* stage = smem + warp * kStage;
+    uint8_t* wsm = smem + warp * kWarpSmem;
+    uint64_t* wb = bars + 2 * warp;
     if (lane == 0) {
-        mbar_init(&bars[warp], 1);
+        mbar_init(&wb[0], 1);
+        mbar_init(&wb[1], 1);
         fence_mbar_init();
     }
     __syncwarp();
@@ -79,27 +90,6 @@ __global__ void __cluster_dims__(kAttCluster, 1, 1) __launch_bounds__(kAttThread
     const int64_t nvis = pos / kBlock + 1;
     const int gw = crank * kAttWarps + warp;
 
-    // this warp's block: issue its bulk copies first, then read Q while they fly
-    int blk = gw < kTopK ? sel[bt * kTopK + gw] : -1;
-    if (blk >= nvis) {
-        if (lane == 0) set_status(p.status, MSA_STATUS_SELECT);
-        blk = -1;
-    }
-    int nk = 0;
-    if (blk >= 0) {
-        const int64_t kbase = (int64_t)blk * kBlock;
-        nk = (int)min64(kBlock, pos + 1 - kbase);
-        if (lane == 0) {
-            const int rows = (nk + 15) & ~15;
-            const int64_t vec0 = ((int64_t)b * p.Hkv + kvh) * p.lmax + kbase;
-            mbar_arrive_expect_tx(&bars[warp], (uint32_t)(2 * rows * (64 + 8)));
-            bulk_g2s(stage, p.k.data + vec0 * 64, (uint32_t)(rows * 64), &bars[warp]);
-            bulk_g2s(stage + kKData, p.k.scale + vec0 * 8, (uint32_t)(rows * 8), &bars[warp]);
-            bulk_g2s(stage + kKData + kKScale, p.v.data + vec0 * 64, (uint32_t)(rows * 64), &bars[warp]);
-            bulk_g2s(stage + 2 * kKData + kKScale, p.v.scale + vec0 * 8, (uint32_t)(rows * 8), &bars[warp]);
-        }
-    }
-
     // query fragments: column g = query head kvh*G + g, dims permuted as the K rows
     uint32_t qf[1][8][2];
     if (g < G) {
@@ -117,6 +107,50 @@ __global__ void __cluster_dims__(kAttCluster, 1, 1) __launch_bounds__(kAttThread
         for (int i = 0; i < 8; ++i) qf[0][i][0] = qf[0][i][1] = 0u;
     }
 
+    int blk;
+    if constexpr (FUSED) {
+        if (warp == 0) {
+            const float* srow = block_scores + bt * p.nbmax;
+            const int64_t r = nvis - 1;
+            const int id = nvis <= 512 ? select_row_warp<16>(srow, nvis, r, lane) : select_row_warp<32>(srow, nvis, r, lane);
+            if (lane < kTopK) {
+                sh_sel[lane] = id;
+                if (sel_out != nullptr && crank == 0 && kvh == 0) sel_out[bt * kTopK + lane] = id;
+            }
+        }
+        __syncthreads();
+        blk = gw < kTopK ? sh_sel[gw] : -1;
+    } else {
+        blk = gw < kTopK ? sel[bt * kTopK + gw] : -1;
+    }
+    if (blk >= nvis) {
+        if (lane == 0) set_status(p.status, MSA_STATUS_SELECT);
+        blk = -1;
+    }
+    int nk = 0, nq = 0;
+    int64_t vec0 = 0;
+    if (blk >= 0) {
+        const int64_t kbase = (int64_t)blk * kBlock;
+        nk = (int)min64(kBlock, pos + 1 - kbase);
+        nq = (nk + kQuarter - 1) / kQuarter;
+        vec0 = ((int64_t)b * p.Hkv + kvh) * p.lmax + kbase;
+    }
+    // quarter j of the block -> stage j & 1 (rows rounded up to 16; the cache holds whole blocks)
+    auto issue = [&](int j) {
+        const int rows = (min(kQuarter, nk - j * kQuarter) + 15) & ~15;
+        uint8_t* st = wsm + (j & 1) * kStage;
+        const int64_t v = vec0 + j * kQuarter;
+        mbar_arrive_expect_tx(&wb[j & 1], (uint32_t)(2 * rows * (64 + 8)));
+        bulk_g2s(st, p.k.data + v * 64, (uint32_t)(rows * 64), &wb[j & 1]);
+        bulk_g2s(st + kKData, p.k.scale + v * 8, (uint32_t)(rows * 8), &wb[j & 1]);
+        bulk_g2s(st + kKData + kKScale, p.v.data + v * 64, (uint32_t)(rows * 64), &wb[j & 1]);
+        bulk_g2s(st + 2 * kKData + kKScale, p.v.scale + v * 8, (uint32_t)(rows * 8), &wb[j & 1]);
+    };
+    if (lane == 0) {
+        if (nq > 0) issue(0);
+        if (nq > 1) issue(1);
+    }
+
     const float sc_log2 = p.softmax_scale * p.k.s_t * kLog2e;
     // per thread: query heads 2c and 2c+1
     float m2[2] = {-INFINITY, -INFINITY}, l2[2] = {0.0f, 0.0f};
@@ -124,66 +158,80 @@ __global__ void __cluster_dims__(kAttCluster, 1, 1) __launch_bounds__(kAttThread
 #pragma unroll
     for (int mt = 0; mt < 8; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.0f;
 
-    if (blk >= 0 && !mbar_wait(&bars[warp], 0)) {
-        if (lane == 0) set_status(p.status, MSA_STATUS_TIMEOUT | MSA_STATUS_AT_ATTEND);
-        mbar_wait(&bars[warp], 0);  // one more bounded wait for the copies before the stage is reused
-        blk = -1;
-    }
-    if (blk >= 0) {
-        const uint8_t* kd = stage;
-        const uint8_t* ksc = stage + kKData;
-        const uint8_t* vd = stage + kKData + kKScale;
-        const uint8_t* vsc = stage + 2 * kKData + kKScale;
-        const int ntiles = (nk + 15) >> 4;
-        // ---- S^T = K Q^T for every key of the block: st[kt] = rows (keys) g, g+8 x cols 2c, 2c+1
-        float st[8][4];
+    for (int j = 0; j < nq; ++j) {
+        if (!mbar_wait(&wb[j & 1], (j >> 1) & 1u)) {
+            if (lane == 0) set_status(p.status, MSA_STATUS_TIMEOUT | MSA_STATUS_AT_ATTEND);
+            // one more bounded wait for the copies still in flight before the stages are reused
+            for (int jj = j; jj < min(nq, j + 2); ++jj) mbar_wait(&wb[jj & 1], (jj >> 1) & 1u);
+            nq = j;
+            break;
+        }
+        const uint8_t* st = wsm + (j & 1) * kStage;
+        const uint8_t* kd = st;
+        const uint8_t* ksc = st + kKData;
+        const uint8_t* vd = st + kKData + kKScale;
+        const uint8_t* vsc = st + 2 * kKData + kKScale;
+        const int qvalid = min(kQuarter, nk - j * kQuarter);
+        const int ntiles = (qvalid + 15) >> 4;
+        // ---- S^T = K Q^T for the quarter's keys: st4[kt] = rows (keys) g, g+8 x cols 2c, 2c+1
+        float s4[2][4];
 #pragma unroll
-        for (int kt = 0; kt < 8; ++kt) {
+        for (int kt = 0; kt < 2; ++kt) {
             if (kt < ntiles) {
                 float acc[1][4];
                 nvfp4_tile_mma<128, 1>(kd, ksc, kt * 16 + g, c, qf, acc);
-                const bool v0 = kt * 16 + g < nk, v1 = kt * 16 + g + 8 < nk;
-                st[kt][0] = v0 ? acc[0][0] * sc_log2 : -INFINITY;
-                st[kt][1] = v0 ? acc[0][1] * sc_log2 : -INFINITY;
-                st[kt][2] = v1 ? acc[0][2] * sc_log2 : -INFINITY;
-                st[kt][3] = v1 ? acc[0][3] * sc_log2 : -INFINITY;
+                const bool v0 = kt * 16 + g < qvalid, v1 = kt * 16 + g + 8 < qvalid;
+                s4[kt][0] = v0 ? acc[0][0] * sc_log2 : -INFINITY;
+                s4[kt][1] = v0 ? acc[0][1] * sc_log2 : -INFINITY;
+                s4[kt][2] = v1 ? acc[0][2] * sc_log2 : -INFINITY;
+                s4[kt][3] = v1 ? acc[0][3] * sc_log2 : -INFINITY;
             } else {
-                st[kt][0] = st[kt][1] = st[kt][2] = st[kt][3] = -INFINITY;
+                s4[kt][0] = s4[kt][1] = s4[kt][2] = s4[kt][3] = -INFINITY;
             }
         }
-        // ---- softmax statistics over the block (query heads 2c, 2c+1)
+        // ---- online softmax over the quarter (query heads 2c, 2c+1), exp2 domain
+        float corr[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
-            float mx = -INFINITY;
-#pragma unroll
-            for (int kt = 0; kt < 8; ++kt) mx = fmaxf(mx, fmaxf(st[kt][e], st[kt][2 + e]));
+            float mx = fmaxf(fmaxf(s4[0][e], s4[0][2 + e]), fmaxf(s4[1][e], s4[1][2 + e]));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-            m2[e] = mx;
+            const float m_new = fmaxf(m2[e], mx);
+            corr[e] = exp2f(m2[e] - m_new);
+            m2[e] = m_new;
             float l = 0.0f;
 #pragma unroll
-            for (int kt = 0; kt < 8; ++kt) {
-                st[kt][e] = exp2f(st[kt][e] - mx);
-                st[kt][2 + e] = exp2f(st[kt][2 + e] - mx);
-                l += st[kt][e] + st[kt][2 + e];
+            for (int kt = 0; kt < 2; ++kt) {
+                s4[kt][e] = exp2f(s4[kt][e] - m_new);
+                s4[kt][2 + e] = exp2f(s4[kt][2 + e] - m_new);
+                l += s4[kt][e] + s4[kt][2 + e];
             }
-            l2[e] = l;
+            l2[e] = l2[e] * corr[e] + l;
+        }
+        if (j > 0) {
+#pragma unroll
+            for (int mt = 0; mt < 8; ++mt) {
+                o[mt][0] *= corr[0];
+                o[mt][1] *= corr[1];
+                o[mt][2] *= corr[0];
+                o[mt][3] *= corr[1];
+            }
         }
         // ---- O^T += V^T P^T, 16 keys at a time
 #pragma unroll
-        for (int kt = 0; kt < 8; ++kt) {
+        for (int kt = 0; kt < 2; ++kt) {
             if (kt < ntiles) {
                 // P^T fragment (keys x heads) -> B operand (k = keys 2c.., n = head g)
-                const uint32_t pb0 = movmatrix_trans(pack_f16x2(st[kt][0], st[kt][1]));
-                const uint32_t pb1 = movmatrix_trans(pack_f16x2(st[kt][2], st[kt][3]));
+                const uint32_t pb0 = movmatrix_trans(pack_f16x2(s4[kt][0], s4[kt][1]));
+                const uint32_t pb1 = movmatrix_trans(pack_f16x2(s4[kt][2], s4[kt][3]));
                 uint32_t vh[4][8];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int key = kt * 16 + 2 * c + (i & 1) + 8 * (i >> 1);
                     uint2 vw = make_uint2(0u, 0u);
                     uint32_t vs = 0u;
-                    if (key < nk) {  // masked keys read as 0 (their P is 0; V may hold anything)
+                    if (key < qvalid) {  // masked keys read as 0 (their P is 0; V may hold anything)
                         vw = lds_v2(vd + key * 64 + g * 8);
                         vs = lds_u8(vsc + key * 8 + g);
                     }
@@ -203,7 +251,10 @@ __global__ void __cluster_dims__(kAttCluster, 1, 1) __launch_bounds__(kAttThread
                 }
             }
         }
+        __syncwarp();  // every lane is done with stage j & 1
+        if (lane == 0 && j + 2 < nq) issue(j + 2);
     }
+    uint8_t* stage = wsm;
 
     // ---- merge the 4 warps of this CTA (each warp's partial O goes into its own stage)
 #pragma unroll
@@ -245,7 +296,7 @@ __global__ void __cluster_dims__(kAttCluster, 1, 1) __launch_bounds__(kAttThread
         for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
 #pragma unroll
         for (int w = 0; w < kAttWarps; ++w) {
-            const float* src = reinterpret_cast<const float*>(smem + w * kStage) + q * kD + d0;
+            const float* src = reinterpret_cast<const float*>(smem + w * kWarpSmem) + q * kD + d0;
 #pragma unroll
             for (int j = 0; j < 8; ++j) acc[j] += f[w] * src[j];
         }
@@ -296,14 +347,15 @@ __global__ void __cluster_dims__(kAttCluster, 1, 1) __launch_bounds__(kAttThread
     cluster.sync();  // keep this CTA's shared memory alive until every peer has read it
 }
 
-template <int G>
-int launch_g(const Problem& p, const int32_t* sel, float* out, float* lse, bool pdl, cudaStream_t st) {
+template <int G, bool FUSED>
+int launch_g(const Problem& p, const int32_t* sel, const float* bs, int32_t* sel_out, float* out, float* lse,
+             bool pdl, cudaStream_t st) {
     const int64_t units = (int64_t)p.B * p.Tq * p.Hkv;
     static int configured_dev = -1;
     const DeviceInfo& di = device_info();
     if (configured_dev != di.device) {
-        if (cudaFuncSetAttribute(attend_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttSmem) !=
-            cudaSuccess)
+        if (cudaFuncSetAttribute(attend_kernel<G, FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)kAttSmem) != cudaSuccess)
             return MSA_ECUDA;
         configured_dev = di.device;
     }
@@ -317,23 +369,36 @@ int launch_g(const Problem& p, const int32_t* sel, float* out, float* lse, bool 
     attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, attend_kernel<G>, p, sel, out, lse) != cudaSuccess) return MSA_ECUDA;
+    if (cudaLaunchKernelEx(&cfg, attend_kernel<G, FUSED>, p, sel, bs, sel_out, out, lse) != cudaSuccess)
+        return MSA_ECUDA;
     return MSA_OK;
+}
+
+template <bool FUSED>
+int launch_any(const Problem& p, const int32_t* sel, const float* bs, int32_t* sel_out, float* out, float* lse,
+               bool pdl, cudaStream_t st) {
+    if (p.D != kD) return MSA_EUNSUPPORTED;
+    const int64_t units = (int64_t)p.B * p.Tq * p.Hkv;
+    if (units * kAttCluster > 0x7FFFFFFFll) return MSA_EUNSUPPORTED;
+    switch (p.Hq / p.Hkv) {
+        case 1: return launch_g<1, FUSED>(p, sel, bs, sel_out, out, lse, pdl, st);
+        case 2: return launch_g<2, FUSED>(p, sel, bs, sel_out, out, lse, pdl, st);
+        case 4: return launch_g<4, FUSED>(p, sel, bs, sel_out, out, lse, pdl, st);
+        case 8: return launch_g<8, FUSED>(p, sel, bs, sel_out, out, lse, pdl, st);
+        default: return MSA_EUNSUPPORTED;
+    }
 }
 
 }  // namespace
 
 int launch_attend(const Problem& p, const int32_t* sel, float* out, float* lse, bool pdl, cudaStream_t st) {
-    if (p.D != kD) return MSA_EUNSUPPORTED;
-    const int64_t units = (int64_t)p.B * p.Tq * p.Hkv;
-    if (units * kAttCluster > 0x7FFFFFFFll) return MSA_EUNSUPPORTED;
-    switch (p.Hq / p.Hkv) {
-        case 1: return launch_g<1>(p, sel, out, lse, pdl, st);
-        case 2: return launch_g<2>(p, sel, out, lse, pdl, st);
-        case 4: return launch_g<4>(p, sel, out, lse, pdl, st);
-        case 8: return launch_g<8>(p, sel, out, lse, pdl, st);
-        default: return MSA_EUNSUPPORTED;
-    }
+    return launch_any<false>(p, sel, nullptr, nullptr, out, lse, pdl, st);
+}
+
+int launch_select_attend(const Problem& p, const float* block_scores, int32_t* sel_out, float* out, float* lse,
+                         bool pdl, cudaStream_t st) {
+    if (p.nbmax > kFusedSelectMaxBlocks) return MSA_EUNSUPPORTED;
+    return launch_any<true>(p, nullptr, block_scores, sel_out, out, lse, pdl, st);
 }
 
 }  // namespace msa

@@ -58,5 +58,8 @@ int launch_select(const Problem& p, const float* block_scores, int32_t* sel, int
                   cudaStream_t st);
 // Sparse attention over the selected blocks.
 int launch_attend(const Problem& p, const int32_t* sel, float* out, float* lse, bool pdl, cudaStream_t st);
+// Selection fused into the attention kernel (rows of <= 1,024 blocks; else MSA_EUNSUPPORTED).
+int launch_select_attend(const Problem& p, const float* block_scores, int32_t* sel_out, float* out, float* lse,
+                         bool pdl, cudaStream_t st);
 
 }  // namespace msa

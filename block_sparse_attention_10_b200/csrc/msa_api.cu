@@ -207,6 +207,8 @@ int msa_decode(const msa_params_t* p, void* ws, size_t ws_bytes, float* out, flo
     const Problem q = to_problem(p);
     const bool pdl = pdl_enabled();
     if (int r = launch_index(q, bs, nullptr, pdl, stream)) return r;
+    // short rows: each attention CTA selects its own row's blocks (one launch fewer)
+    if (q.nbmax <= 1024) return launch_select_attend(q, bs, sel_out, out, lse, pdl, stream);
     if (int r = launch_select(q, bs, sel, sel_out, pdl, stream)) return r;
     return launch_attend(q, sel, out, lse, pdl, stream);
 }

@@ -13,6 +13,7 @@
 // of "largest key below the previous winner".  Rows of up to 4,096 blocks live
 // in registers.  Deterministic and independent of the thread layout.
 #include "internal.h"
+#include "select_row.cuh"
 
 namespace msa {
 namespace {
@@ -20,18 +21,6 @@ namespace {
 constexpr int kSelThreads = 256;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kPer = 16;  // candidates per thread held in registers (rows of <= 4,096 blocks)
-
-__device__ __forceinline__ uint64_t rank_key(float s, int64_t n) {
-    uint32_t u = __float_as_uint(s);
-    u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-    return ((uint64_t)u << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)n);
-}
-
-__device__ __forceinline__ uint64_t warp_max64(uint64_t v) {
-    const uint32_t hi = __reduce_max_sync(0xffffffffu, (uint32_t)(v >> 32));
-    const uint32_t lo = __reduce_max_sync(0xffffffffu, (uint32_t)(v >> 32) == hi ? (uint32_t)v : 0u);
-    return ((uint64_t)hi << 32) | lo;
-}
 
 // One CTA per (sequence, query token).  Thread i holds candidates i, i + 256, ... of the
 // row in registers; each of the 15 rounds takes the largest key below the previous winner
@@ -106,8 +95,9 @@ __global__ void __launch_bounds__(kSelThreads)
 // Short rows (<= 1,024 blocks): one warp per (sequence, query token), 32
 // candidates per lane in registers, 15 rounds of two redux.sync each.
 constexpr int kWarpRows = 4;
-constexpr int kWarpPer = 32;
+constexpr int kWarpPer = 32;  // rows of up to 32 * kWarpPer blocks take the warp kernel
 
+template <int PER>
 __global__ void __launch_bounds__(32 * kWarpRows)
     select_warp_kernel(const Problem p, const float* __restrict__ block_scores, int32_t* __restrict__ sel,
                        int32_t* __restrict__ sel_copy) {
@@ -118,39 +108,11 @@ __global__ void __launch_bounds__(32 * kWarpRows)
     if (row >= (int64_t)p.B * p.Tq) return;
     const int b = (int)(row / p.Tq), t = (int)(row % p.Tq);
     const int64_t L = clamp_len(p.seq_lens[b], p.Tq, p.lmax, nullptr);
-    const int64_t pos = L - p.Tq + t;
-    const int64_t r = pos / kBlock;
-    const int64_t nvis = r + 1;
-    const float* s = block_scores + row * p.nbmax;
-    const int want = (int)min64(kTopK - 1, nvis - 1);
-    uint64_t k0[kWarpPer];
-#pragma unroll
-    for (int j = 0; j < kWarpPer; ++j) {
-        const int64_t n = j * 32 + lane;
-        k0[j] = (n < nvis && n != r) ? rank_key(__ldg(s + n), n) : 0ull;
-    }
-    uint64_t prev = ~0ull;
-    int mine = -1;  // lane i < want holds the i-th best
-    for (int k = 0; k < want; ++k) {
-        uint64_t best = 0;
-#pragma unroll
-        for (int j = 0; j < kWarpPer; ++j)
-            if (k0[j] < prev && k0[j] > best) best = k0[j];
-        prev = warp_max64(best);
-        if (lane == k) mine = (int)(0xFFFFFFFFu - (uint32_t)prev);
-    }
-    if (lane == want) mine = (int)r;
-    const int nsel = want + 1;
-    int rank = 0;
-    for (int i = 0; i < nsel; ++i) rank += (__shfl_sync(0xffffffffu, mine, i) < mine) ? 1 : 0;
-    int32_t* out = sel + row * kTopK;
-    int32_t* o2 = sel_copy ? sel_copy + row * kTopK : nullptr;
-    if (lane < nsel) {
-        out[rank] = mine;
-        if (o2) o2[rank] = mine;
-    } else if (lane < kTopK) {
-        out[lane] = -1;
-        if (o2) o2[lane] = -1;
+    const int64_t r = (L - p.Tq + t) / kBlock;
+    const int id = select_row_warp<PER>(block_scores + row * p.nbmax, r + 1, r, lane);
+    if (lane < kTopK) {
+        sel[row * kTopK + lane] = id;
+        if (sel_copy) sel_copy[row * kTopK + lane] = id;
     }
 }
 
@@ -170,8 +132,10 @@ int launch_select(const Problem& p, const float* block_scores, int32_t* sel, int
     attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const cudaError_t e = short_rows ? cudaLaunchKernelEx(&cfg, select_warp_kernel, p, block_scores, sel, sel_copy)
-                                     : cudaLaunchKernelEx(&cfg, select_kernel, p, block_scores, sel, sel_copy);
+    cudaError_t e;
+    if (!short_rows) e = cudaLaunchKernelEx(&cfg, select_kernel, p, block_scores, sel, sel_copy);
+    else if (p.nbmax <= 32 * 16) e = cudaLaunchKernelEx(&cfg, select_warp_kernel<16>, p, block_scores, sel, sel_copy);
+    else e = cudaLaunchKernelEx(&cfg, select_warp_kernel<32>, p, block_scores, sel, sel_copy);
     if (e != cudaSuccess) return MSA_ECUDA;
     return MSA_OK;
 }
