@@ -7,12 +7,13 @@ Workload (one GPU): 32 sequences x 64K-token context, 1 query token each,
 GQA 32 query / 4 KV heads, head dim 128, indexer 8 heads x 128, NVFP4 K/V and
 index keys (synthetic N(0,1) with 8 needle blocks per sequence), bf16 queries,
 top-16 blocks of 128 tokens with the recent block forced.  A step is one
-msa_decode call (indexer -> select -> attention) over the whole batch.
+msa_decode call (indexer -> select -> attention) over the whole batch; the
+single-launch variant (msa_decode_single_launch) is timed beside it.
 
 Timed region: K steps replayed from a CUDA graph on one stream, CUDA events,
-barrier + synchronize on both sides; two replicas of the caches alternate
-(each step reads ~189 MB, more than the 126 MB L2, and the caches themselves
-are 1.36 GB per replica).  Multi-GPU (torchrun): every rank runs its own 32
+barrier + synchronize on both sides; rotating replicas of the caches (each
+step reads ~189 MB, more than the 126 MB L2; the replicas cycle through at
+least 4x the L2 size).  Multi-GPU (torchrun): every rank runs its own 32
 sequences (weak scaling, no data-path collective); the time is the max over
 ranks.  ``--impl reference`` times the CPU oracle on the host cores instead.
 """
@@ -351,6 +352,36 @@ def step_work(w, seq_lens, sel):
     return idx_bytes, idx_flops, att_bytes, att_flops
 
 
+def launches_per_step(p):
+    """Kernels of ours that one msa_decode call launches: the indexer, then the selection
+    fused into the attention kernel (rows of <= 1,024 blocks) or select + attend."""
+    return 2 if p.nbmax <= 1024 else 3
+
+
+def time_graph(fn, n, stream, reps=5):
+    """Mean ms per call of fn(i), i < n, captured in one CUDA graph; best of reps replays."""
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            fn(i)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(n):
+            fn(i)
+    torch.cuda.synchronize()
+    best = float("inf")
+    for _ in range(reps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            a.record(stream)
+            g.replay()
+            b.record(stream)
+        torch.cuda.synchronize()
+        best = min(best, a.elapsed_time(b) / n)
+    del g
+    return best
+
+
 def run_ours(args):
     from block_sparse_attention_10_b200 import msa
     msa.lib()
@@ -423,7 +454,8 @@ def run_ours(args):
     status = int(p0.status.item())
     assert status == 0, f"device status word {status:#x}"
 
-    # dominant kernel (the indexer) alone: a CUDA graph of back-to-back launches on its stream,
+    # the indexer alone (the dominant kernel of the separate launches): a CUDA graph of
+    # back-to-back launches on its stream,
     # CUDA events around the replays (no host launch gaps inside the timed region)
     nb_i = max(1, min(args.steps, 50))
     bs = torch.empty(w.B, w.Tq, p0.nbmax, dtype=torch.float32, device=dev)
@@ -462,6 +494,18 @@ def run_ours(args):
                 "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                 "frac_of_8tbs": achieved / CONTRACT_HBM_GBS, "algorithmic_bytes_per_launch": idx_bytes,
                 "launch_ms": idx_ms, "traffic": _profile_traffic("index_decode.cu", "index_decode", w.name)}
+
+    # the same step as one persistent launch (msa_decode_single_launch), for comparison
+    single = None
+    if msa.msa_workspace_size_single_launch(p0) > 0:
+        ws1 = msa.alloc_workspace_single_launch(p0)
+        single_ms = time_graph(lambda i: msa.msa_decode_single_launch(reps[i % len(reps)], ws1, out, lse, None,
+                                                                     stream=stream),
+                               max(1, min(args.steps, 50)), stream)
+        single = {"entry": "msa_decode_single_launch", "ms_per_step": single_ms,
+                  "value": aggregate_throughput(w.B * w.Tq, 1, single_ms * 1e-3), "unit": UNIT}
+        del ws1
+        assert int(p0.status.item()) == 0, f"device status word {int(p0.status.item()):#x}"
 
     # end to end through the public API: pinned host queries -> device, decode, output -> host
     n_e2e = min(args.steps, 200)
@@ -507,10 +551,11 @@ def run_ours(args):
             "step_frac_of_8tbs": step_bytes / (ms * 1e-3) / 1e9 / CONTRACT_HBM_GBS,
             "step_tflops": (idx_flops + att_flops) / (ms * 1e-3) / 1e12,
             "roofline": roof,
+            "single_launch_alternative": single,
             "cpu_baseline": cpu,
             "e2e": {"value": aggregate_throughput(w.B * w.Tq, ws_n, e2e_s), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": launches_per_step(p0) * args.steps,
             "clocks": clk.summary(),
         }
         print(json.dumps(line), flush=True)

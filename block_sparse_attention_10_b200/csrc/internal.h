@@ -62,4 +62,14 @@ int launch_attend(const Problem& p, const int32_t* sel, float* out, float* lse, 
 int launch_select_attend(const Problem& p, const float* block_scores, int32_t* sel_out, float* out, float* lse,
                          bool pdl, cudaStream_t st);
 
+// The whole decode step in one persistent launch (decode_fused.cu).  Workspace: byte
+// offsets of its regions; the counter region [0, ctr_bytes) is cleared by the launcher.
+struct FusedLayout {
+    size_t ctr_bytes, bscores, sel, part, total;
+};
+FusedLayout fused_layout(const Problem& p);
+bool fused_supported(const Problem& p);
+int launch_decode_fused(const Problem& p, void* ws, float* out, float* lse, int32_t* sel_out, bool pdl,
+                        cudaStream_t st);
+
 }  // namespace msa

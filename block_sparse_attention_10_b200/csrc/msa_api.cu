@@ -140,7 +140,7 @@ const char* msa_status_string(int code) {
         case MSA_EINVAL: return "MSA_EINVAL: invalid argument";
         case MSA_EUNSUPPORTED: return "MSA_EUNSUPPORTED: shape not supported by the kernels";
         case MSA_EALIGN: return "MSA_EALIGN: pointer not 16-byte aligned";
-        case MSA_EWORKSPACE: return "MSA_EWORKSPACE: workspace missing or too small";
+        case MSA_EWORKSPACE: return "MSA_EWORKSPACE: workspace missing, misaligned or too small";
         case MSA_ECUDA: return "MSA_ECUDA: CUDA launch error";
         default: return "MSA: unknown status";
     }
@@ -174,6 +174,12 @@ int msa_nvfp4_amax(const float* x, int64_t n, float* amax_out, cudaStream_t stre
 size_t msa_workspace_size(const msa_params_t* p) {
     if (check_params(p, true, true) != MSA_OK) return 0;
     return ws_block_scores_bytes(p) + ws_sel_bytes(p);
+}
+
+size_t msa_workspace_size_single_launch(const msa_params_t* p) {
+    if (check_params(p, true, true) != MSA_OK) return 0;
+    const Problem q = to_problem(p);
+    return fused_supported(q) ? fused_layout(q).total : 0;
 }
 
 int msa_index(const msa_params_t* p, float* block_scores, float* token_scores, cudaStream_t stream) {
@@ -211,6 +217,18 @@ int msa_decode(const msa_params_t* p, void* ws, size_t ws_bytes, float* out, flo
     if (q.nbmax <= 1024) return launch_select_attend(q, bs, sel_out, out, lse, pdl, stream);
     if (int r = launch_select(q, bs, sel, sel_out, pdl, stream)) return r;
     return launch_attend(q, sel, out, lse, pdl, stream);
+}
+
+int msa_decode_single_launch(const msa_params_t* p, void* ws, size_t ws_bytes, float* out, float* lse,
+                             int32_t* sel_out, cudaStream_t stream) {
+    if (int r = check_params(p, true, true)) return r;
+    if (!out) return MSA_EINVAL;
+    if (!aligned16(out)) return MSA_EALIGN;
+    const Problem q = to_problem(p);
+    if (!fused_supported(q)) return MSA_EUNSUPPORTED;
+    if (!ws || ws_bytes < fused_layout(q).total || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0)
+        return MSA_EWORKSPACE;
+    return launch_decode_fused(q, ws, out, lse, sel_out, pdl_enabled(), stream);
 }
 
 }  // extern "C"

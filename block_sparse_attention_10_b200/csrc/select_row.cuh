@@ -10,7 +10,8 @@
 // inverted block index), so "best" is a plain maximum and ties go to the lower index.
 // Lane i holds candidates i, i + 32, ... in registers; every round takes, per lane, the
 // largest key below the previous winner with a depth-log2(PER) tree, then the warp
-// maximum with two 32-bit redux.sync.  Deterministic.
+// maximum with two 32-bit redux.sync.  Deterministic.  A key of 0 marks an empty slot
+// (scores are never NaN, so every real key is non-zero).
 #pragma once
 
 #include "common.cuh"
@@ -31,30 +32,36 @@ __device__ __forceinline__ uint64_t warp_max64(uint64_t v) {
     return ((uint64_t)hi << 32) | lo;
 }
 
-// Selection of row `s` (nvis <= 32 * PER visible blocks, forced block r = nvis - 1).
+// Selection of row `s` (nvis visible blocks, forced block r = nvis - 1).  Rows longer than
+// 32 * PER blocks are taken in chunks of that size, the best keys so far carried along.
+// kCoherent: the scores were written by other warps of the same launch (read through L2).
 // Returns, in lane i < 16, the i-th selected block id in ascending order (or -1).
-template <int PER>
+template <int PER, bool kCoherent = false>
 __device__ __forceinline__ int select_row_warp(const float* __restrict__ s, int64_t nvis, int64_t r, int lane) {
     const int want = (int)min64(kTopK - 1, nvis - 1);
-    uint64_t k0[PER];
+    uint64_t best = 0ull;  // lane k < want: the k-th best key among the blocks seen so far
+    for (int64_t base = 0; base < nvis; base += 32 * PER) {
+        uint64_t k0[PER];
 #pragma unroll
-    for (int j = 0; j < PER; ++j) {
-        const int64_t n = (int64_t)j * 32 + lane;
-        k0[j] = (n < nvis && n != r) ? rank_key(__ldg(s + n), n) : 0ull;
+        for (int j = 0; j < PER; ++j) {
+            const int64_t n = base + (int64_t)j * 32 + lane;
+            k0[j] = (n < nvis && n != r) ? rank_key(kCoherent ? __ldcg(s + n) : __ldg(s + n), n) : 0ull;
+        }
+        const uint64_t carry = best;
+        uint64_t prev = ~0ull;
+        for (int k = 0; k < want; ++k) {
+            uint64_t cand[PER];
+#pragma unroll
+            for (int j = 0; j < PER; ++j) cand[j] = k0[j] < prev ? k0[j] : 0ull;
+#pragma unroll
+            for (int w = PER / 2; w >= 1; w >>= 1)
+#pragma unroll
+                for (int j = 0; j < w; ++j) cand[j] = max64(cand[j], cand[j + w]);
+            prev = warp_max64(max64(cand[0], carry < prev ? carry : 0ull));
+            if (lane == k) best = prev;
+        }
     }
-    uint64_t prev = ~0ull;
-    int mine = -1;  // lane k < want holds the k-th best
-    for (int k = 0; k < want; ++k) {
-        uint64_t cand[PER];
-#pragma unroll
-        for (int j = 0; j < PER; ++j) cand[j] = k0[j] < prev ? k0[j] : 0ull;
-#pragma unroll
-        for (int w = PER / 2; w >= 1; w >>= 1)
-#pragma unroll
-            for (int j = 0; j < w; ++j) cand[j] = max64(cand[j], cand[j + w]);
-        prev = warp_max64(cand[0]);
-        if (lane == k) mine = (int)(0xFFFFFFFFu - (uint32_t)prev);
-    }
+    int mine = lane < want ? (int)(0xFFFFFFFFu - (uint32_t)best) : -1;  // lane k < want holds the k-th best
     if (lane == want) mine = (int)r;
     const int nsel = want + 1;
     int rank = 0;

@@ -27,7 +27,8 @@ MSA_STATUS_TIMEOUT = 4
 
 # names exported by the C ABI (include/msa.h)
 EXPORTS = ("msa_status_string", "msa_version", "msa_nvfp4_encode", "msa_nvfp4_decode", "msa_nvfp4_amax",
-           "msa_workspace_size", "msa_index", "msa_select", "msa_attend", "msa_decode", "msa_decode_static")
+           "msa_workspace_size", "msa_index", "msa_select", "msa_attend", "msa_decode", "msa_decode_static",
+           "msa_workspace_size_single_launch", "msa_decode_single_launch")
 MSA_STATIC_SCRATCH_BYTES = 4 << 20
 
 
@@ -74,8 +75,13 @@ def lib() -> ctypes.CDLL:
         L.msa_select.argtypes = [P, vp, vp, vp]
         L.msa_attend.argtypes = [P, vp, vp, vp, vp]
         L.msa_decode.argtypes = [P, vp, ctypes.c_size_t, vp, vp, vp, vp]
+        L.msa_workspace_size_single_launch.restype = ctypes.c_size_t
+        L.msa_workspace_size_single_launch.argtypes = [P]
+        L.msa_decode_single_launch.argtypes = [P, vp, ctypes.c_size_t, vp, vp, vp, vp]
         L.msa_decode_static.argtypes = [P, vp, vp, vp, vp]
-        for name in (n for n in EXPORTS if n not in ("msa_status_string", "msa_version", "msa_workspace_size")):
+        for name in (n for n in EXPORTS
+                     if n not in ("msa_status_string", "msa_version", "msa_workspace_size",
+                                  "msa_workspace_size_single_launch")):
             getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -202,6 +208,26 @@ def msa_decode(p: MsaProblem, ws: torch.Tensor, out: torch.Tensor, lse: Optional
     prm = p.params()
     _check(lib().msa_decode(ctypes.byref(prm), _ptr(ws), ws.numel() * ws.element_size(), _ptr(out), _ptr(lse),
                             _ptr(sel_out), _stream(stream)), "msa_decode")
+
+
+def msa_workspace_size_single_launch(p: MsaProblem) -> int:
+    prm = p.params()
+    return int(lib().msa_workspace_size_single_launch(ctypes.byref(prm)))
+
+
+def msa_decode_single_launch(p: MsaProblem, ws: torch.Tensor, out: torch.Tensor, lse: Optional[torch.Tensor] = None,
+                             sel_out: Optional[torch.Tensor] = None, stream=None):
+    """The decode step as one persistent launch (same results as msa_decode; see msa.h)."""
+    prm = p.params()
+    _check(lib().msa_decode_single_launch(ctypes.byref(prm), _ptr(ws), ws.numel() * ws.element_size(), _ptr(out),
+                                          _ptr(lse), _ptr(sel_out), _stream(stream)), "msa_decode_single_launch")
+
+
+def alloc_workspace_single_launch(p: MsaProblem) -> torch.Tensor:
+    n = msa_workspace_size_single_launch(p)
+    if n == 0:
+        raise MsaError(2, "msa_workspace_size_single_launch")
+    return torch.empty(n, dtype=torch.uint8, device=p.q.device)
 
 
 def msa_decode_static(p: MsaProblem, out: torch.Tensor, lse: Optional[torch.Tensor] = None,

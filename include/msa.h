@@ -76,6 +76,9 @@ typedef enum msa_status {
 #define MSA_STATUS_AT_INDEX_DRAIN 0x200u    /* indexer: producer draining its last copies */
 #define MSA_STATUS_AT_INDEX_CONSUMER 0x400u /* indexer: consumer waiting for a stage's bytes */
 #define MSA_STATUS_AT_ATTEND 0x800u         /* attention: warp waiting for its block's bytes */
+#define MSA_STATUS_AT_DECODE_STAGE 0x1000u  /* single-launch decode: warp waiting for a stage's bytes */
+#define MSA_STATUS_AT_DECODE_WAIT 0x2000u   /* single-launch decode: warp waiting for another warp's
+                                               pooled scores or selection */
 
 /* One NVFP4 cache tensor (K, V or index-K); the layout is given above. */
 typedef struct msa_nvfp4_cache {
@@ -175,13 +178,46 @@ int msa_select(const msa_params_t* p, const float* block_scores, int32_t* sel,
 int msa_attend(const msa_params_t* p, const int32_t* sel, float* out, float* lse,
                cudaStream_t stream);
 
-/* The whole MSA decode step: msa_index -> msa_select -> msa_attend.
+/* The whole MSA decode step: msa_index -> msa_select -> msa_attend (two
+ * launches when the rows have <= 1,024 blocks: the selection then runs inside
+ * the attention kernel).
  *   ws, ws_bytes  device scratch of at least msa_workspace_size(p) bytes,
  *                 256-byte aligned; contents on entry are ignored
  *   out, lse      as for msa_attend
  *   sel_out       int32 [B][Tq][16] copy of the selection, or NULL */
 int msa_decode(const msa_params_t* p, void* ws, size_t ws_bytes, float* out, float* lse,
                int32_t* sel_out, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
+ * The decode step as one persistent launch.  Prior art: the single-launch
+ * "mono" decode path of "vLLM turns MiniMax's day-zero promise into
+ * GPU-specific serving code" (upstreambeat.ai, "What changed").  Same results
+ * as msa_decode (same selection; attention within the stated tolerance, the
+ * per-block partials being combined in another order).  Every warp of the grid
+ * works through one list of index, select and attention items, so the
+ * attention of early sequences overlaps the index stream of later ones.  On
+ * B200 at the decode workloads of this library it is slower than msa_decode
+ * (each select and attention item is a chain on one warp, where the separate
+ * kernels spread the same work over 16 warps); it is kept as a measured
+ * alternative, not used by msa_decode.
+ * ------------------------------------------------------------------------- */
+
+/* Scratch for msa_decode_single_launch (0 if the shape is not supported:
+ * it needs Tq * HI <= 16): counters, pooled scores, selection and per-block
+ * attention partials. */
+size_t msa_workspace_size_single_launch(const msa_params_t* p);
+
+/* As msa_decode, in one launch (plus one cudaMemsetAsync that clears the
+ * workspace's counter region on `stream`).
+ *   ws, ws_bytes  at least msa_workspace_size_single_launch(p) bytes,
+ *                 256-byte aligned; contents on entry are ignored; one call
+ *                 at a time may use it
+ * Returns MSA_EUNSUPPORTED for Tq * HI > 16.  A wait inside the kernel for
+ * another warp's result that exceeds 2 s (all CTAs of the grid must be
+ * resident: another kernel holding SMs for that long) sets MSA_STATUS_TIMEOUT
+ * | MSA_STATUS_AT_DECODE_WAIT and ends the launch. */
+int msa_decode_single_launch(const msa_params_t* p, void* ws, size_t ws_bytes, float* out,
+                             float* lse, int32_t* sel_out, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
  * Decode without caller scratch.  No counterpart in the paper: this is a

@@ -34,10 +34,11 @@ def run_steps(p):
                 out=out.cpu().numpy(), lse=lse.cpu().numpy())
 
 
-def run_decode(p):
-    ws = msa.alloc_workspace(p)
+def run_decode(p, single_launch=False, ws=None):
+    if ws is None:
+        ws = msa.alloc_workspace_single_launch(p) if single_launch else msa.alloc_workspace(p)
     out, lse, sel = msa.outputs(p)
-    msa.msa_decode(p, ws, out, lse, sel)
+    (msa.msa_decode_single_launch if single_launch else msa.msa_decode)(p, ws, out, lse, sel)
     torch.cuda.synchronize()
     return dict(sel=sel.cpu().numpy(), out=out.cpu().numpy(), lse=lse.cpu().numpy())
 

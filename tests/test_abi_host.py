@@ -45,14 +45,37 @@ def _params(**kw):
     return msa._Params(**base)
 
 
+def _r256(x):
+    return (x + 255) // 256 * 256
+
+
 def test_workspace_size_host_only(L):
     p = _params()
+    B, Tq, Hkv, nb = 2, 1, 1, 4096 // 128
     n = L.msa_workspace_size(ctypes.byref(p))
-    nb = 4096 // 128
-    assert n == ((2 * 1 * nb * 4 + 255) // 256) * 256 + ((2 * 16 * 4 + 255) // 256) * 256
+    assert n == _r256(B * Tq * nb * 4) + _r256(B * Tq * 16 * 4)
     assert L.msa_workspace_size(None) == 0
     bad = _params(lmax=4000)
     assert L.msa_workspace_size(ctypes.byref(bad)) == 0
+    # the single-launch path: counters, pooled scores, selection, and 8 partials of
+    # (8 x 128 + 16) floats per (query row, KV head)
+    n1 = L.msa_workspace_size_single_launch(ctypes.byref(p))
+    assert n1 == (_r256((4 + B + B * Tq + B * Tq * Hkv) * 4) + _r256(B * Tq * nb * 4) + _r256(B * Tq * 16 * 4) +
+                  _r256(B * Tq * Hkv * 8 * 1040 * 4))
+    assert L.msa_workspace_size_single_launch(ctypes.byref(_params(Tq=8))) == 0  # Tq * HI > 16
+    assert L.msa_workspace_size_single_launch(ctypes.byref(bad)) == 0
+
+
+def test_single_launch_rejects_before_enqueueing(L):
+    out = ctypes.c_void_p(0x20000)
+    r = L.msa_decode_single_launch(ctypes.byref(_params(Tq=8)), ctypes.c_void_p(0x10000), 1 << 30, out, None, None,
+                                   None)
+    assert r == 2  # MSA_EUNSUPPORTED
+    p = _params()
+    assert L.msa_decode_single_launch(ctypes.byref(p), ctypes.c_void_p(0x10000), 1024, out, None, None, None) == 4
+    assert L.msa_decode_single_launch(ctypes.byref(p), None, 1 << 30, out, None, None, None) == 4
+    assert L.msa_decode_single_launch(ctypes.byref(_params(HI=3)), ctypes.c_void_p(0x10000), 1 << 30, out, None,
+                                      None, None) == 2
 
 
 @pytest.mark.parametrize("field,value,code", [
