@@ -89,11 +89,10 @@ __global__ void __cluster_dims__(kAttCluster, 1, 1) __launch_bounds__(kAttThread
         if (warp == 0) {
             const float* srow = block_scores + bt * p.nbmax;
             const int64_t r = nvis - 1;
-            const int id = nvis <= 512 ? select_row_warp<16>(srow, nvis, r, lane) : select_row_warp<32>(srow, nvis, r, lane);
-            if (lane < kTopK) {
-                sh_sel[lane] = id;
-                if (sel_out != nullptr && crank == 0 && kvh == 0) sel_out[bt * kTopK + lane] = id;
-            }
+            if (nvis <= 512) select_row_warp<16>(srow, nvis, r, lane, sh_sel);
+            else select_row_warp<32>(srow, nvis, r, lane, sh_sel);
+            __syncwarp();
+            if (lane < kTopK && sel_out != nullptr && crank == 0 && kvh == 0) sel_out[bt * kTopK + lane] = sh_sel[lane];
         }
         __syncthreads();
         blk = gw < kTopK ? sh_sel[gw] : -1;

@@ -352,8 +352,12 @@ __global__ void __launch_bounds__(kFThreads, 2) decode_fused_kernel(const Proble
             const int64_t row = (int64_t)cur.b * Tq + cur.t;
             const int64_t pos = L - Tq + cur.t;
             const int64_t nvis = pos / kBlock + 1;
-            const int id = select_row_warp<16, true>(fa.bscores + row * p.nbmax, nvis, nvis - 1, lane);
-            if (lane < kTopK) fa.sel[row * kTopK + lane] = id;
+            if (nvis <= 512) {
+                select_row_warp<16, true>(fa.bscores + row * p.nbmax, nvis, nvis - 1, lane, fa.sel + row * kTopK);
+            } else {
+                const int id = select_row_warp_long<16, true>(fa.bscores + row * p.nbmax, nvis, nvis - 1, lane);
+                if (lane < kTopK) fa.sel[row * kTopK + lane] = id;
+            }
             __threadfence();
             __syncwarp();
             if (lane == 0) st_release_u32(sel_ready + row, 1u);

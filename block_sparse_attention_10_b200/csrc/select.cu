@@ -7,11 +7,13 @@
 // min(15, r) other blocks under the total order (score desc, index asc); the
 // list is written ascending and padded with -1.
 //
-// One CTA of 256 threads per (sequence, query token).  Each candidate becomes a
-// 64-bit key (order-preserving bits of the fp32 score, then the inverted block
-// index), so "best" is a plain maximum and ties go to the lower index; 15 rounds
-// of "largest key below the previous winner".  Rows of up to 4,096 blocks live
-// in registers.  Deterministic and independent of the thread layout.
+// Rows of <= 1,024 blocks: one warp per (sequence, query token), the threshold
+// selection of select_row.cuh.  Rows of <= 4,096 blocks: one CTA of 8 warps per
+// row; each warp selects the best 15 of its 512-block chunk (the row's best 15
+// are among those 120), then one warp selects from the 120 candidates, which
+// sit in ascending block order so the index tie-break carries over.  Longer
+// rows: 64-bit keys (score key, inverted index) and 15 rounds of "largest key
+// below the previous winner" over the whole CTA.  All deterministic.
 #include "internal.h"
 #include "select_row.cuh"
 
@@ -22,10 +24,78 @@ constexpr int kSelThreads = 256;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kPer = 16;  // candidates per thread held in registers (rows of <= 4,096 blocks)
 
-// One CTA per (sequence, query token).  Thread i holds candidates i, i + 256, ... of the
-// row in registers; each of the 15 rounds takes the largest key below the previous winner
-// with a warp reduction (redux.sync) and one exchange of 8 warp maxima through shared
-// memory (double-buffered, one __syncthreads per round).
+// Rows of <= 4,096 blocks: one CTA of 8 warps per (sequence, query token), two levels.
+constexpr int kCtaPer = 16;  // 8 warps x 32 lanes x 16 candidates
+constexpr int kCtaMaxBlocks = kSelWarps * 32 * kCtaPer;
+constexpr int kCand = kTopK - 1;  // candidates kept per chunk
+
+__global__ void __launch_bounds__(kSelThreads)
+    select_cta_kernel(const Problem p, const float* __restrict__ block_scores, int32_t* __restrict__ sel,
+                      int32_t* __restrict__ sel_copy) {
+    __shared__ uint32_t ckey[kSelWarps * kCand];
+    __shared__ int32_t cid[kSelWarps * kCand];
+    __shared__ int32_t res[kTopK];
+    pdl_wait();
+    pdl_launch_dependents();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t row = blockIdx.x;
+    const int b = (int)(row / p.Tq), t = (int)(row % p.Tq);
+    const int64_t L = clamp_len(p.seq_lens[b], p.Tq, p.lmax, nullptr);
+    const int64_t r = (L - p.Tq + t) / kBlock;  // forced block
+    const int64_t nvis = r + 1;
+    const float* s = block_scores + row * p.nbmax;
+
+    // level 1: the best 15 of this warp's chunk, in ascending block order
+    const int base = warp * 32 * kCtaPer;
+    uint32_t k[kCtaPer];
+    int cnt = 0;
+#pragma unroll
+    for (int j = 0; j < kCtaPer; ++j) {
+        const int64_t n = base + j * 32 + lane;
+        k[j] = (n < nvis && n != r) ? score_key(__ldg(s + n)) : 0u;
+        cnt += k[j] != 0u ? 1 : 0;
+    }
+    cnt = (int)__reduce_add_sync(0xffffffffu, (unsigned)cnt);
+    const int want_w = min(kCand, cnt);
+    if (want_w > 0) {
+        int n_gt;
+        const uint32_t T = warp_kth_key(k, want_w, n_gt);
+        warp_compact(k, T, want_w - n_gt, lane, [&](int slot, int j) {
+            ckey[warp * kCand + slot] = k[j];
+            cid[warp * kCand + slot] = base + j * 32 + lane;
+        });
+    }
+    if (lane >= want_w && lane < kCand) ckey[warp * kCand + lane] = 0u;
+    __syncthreads();
+
+    // level 2: the row's best 15 among the 120 candidates
+    if (warp != 0) return;
+    const int want = (int)min64(kCand, nvis - 1);
+    if (want > 0) {
+        uint32_t kk[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int c = j * 32 + lane;
+            kk[j] = c < kSelWarps * kCand ? ckey[c] : 0u;
+        }
+        int n_gt;
+        const uint32_t T = warp_kth_key(kk, want, n_gt);
+        warp_compact(kk, T, want - n_gt, lane, [&](int slot, int j) { res[slot] = cid[j * 32 + lane]; });
+    }
+    if (lane == want) res[want] = (int32_t)r;
+    if (lane > want && lane < kTopK) res[lane] = -1;
+    __syncwarp();
+    if (lane < kTopK) {
+        sel[row * kTopK + lane] = res[lane];
+        if (sel_copy) sel_copy[row * kTopK + lane] = res[lane];
+    }
+}
+
+// Rows of more than 4,096 blocks: one CTA per (sequence, query token).  Thread i holds
+// candidates i, i + 256, ... of the row's first 4,096 blocks in registers (the rest are
+// re-read each round); each of the 15 rounds takes the largest key below the previous
+// winner with a warp reduction (redux.sync) and one exchange of 8 warp maxima through
+// shared memory (double-buffered, one __syncthreads per round).
 __global__ void __launch_bounds__(kSelThreads)
     select_kernel(const Problem p, const float* __restrict__ block_scores, int32_t* __restrict__ sel,
                   int32_t* __restrict__ sel_copy) {
@@ -92,8 +162,8 @@ __global__ void __launch_bounds__(kSelThreads)
     }
 }
 
-// Short rows (<= 1,024 blocks): one warp per (sequence, query token), 32
-// candidates per lane in registers, 15 rounds of two redux.sync each.
+// Short rows (<= 1,024 blocks): one warp per (sequence, query token), up to 32
+// candidates per lane in registers.
 constexpr int kWarpRows = 4;
 constexpr int kWarpPer = 32;  // rows of up to 32 * kWarpPer blocks take the warp kernel
 
@@ -109,10 +179,12 @@ __global__ void __launch_bounds__(32 * kWarpRows)
     const int b = (int)(row / p.Tq), t = (int)(row % p.Tq);
     const int64_t L = clamp_len(p.seq_lens[b], p.Tq, p.lmax, nullptr);
     const int64_t r = (L - p.Tq + t) / kBlock;
-    const int id = select_row_warp<PER>(block_scores + row * p.nbmax, r + 1, r, lane);
+    __shared__ int32_t res[kWarpRows][kTopK];
+    select_row_warp<PER>(block_scores + row * p.nbmax, r + 1, r, lane, res[warp]);
+    __syncwarp();
     if (lane < kTopK) {
-        sel[row * kTopK + lane] = id;
-        if (sel_copy) sel_copy[row * kTopK + lane] = id;
+        sel[row * kTopK + lane] = res[warp][lane];
+        if (sel_copy) sel_copy[row * kTopK + lane] = res[warp][lane];
     }
 }
 
@@ -133,7 +205,9 @@ int launch_select(const Problem& p, const float* block_scores, int32_t* sel, int
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cudaError_t e;
-    if (!short_rows) e = cudaLaunchKernelEx(&cfg, select_kernel, p, block_scores, sel, sel_copy);
+    if (!short_rows && p.nbmax <= kCtaMaxBlocks)
+        e = cudaLaunchKernelEx(&cfg, select_cta_kernel, p, block_scores, sel, sel_copy);
+    else if (!short_rows) e = cudaLaunchKernelEx(&cfg, select_kernel, p, block_scores, sel, sel_copy);
     else if (p.nbmax <= 32 * 16) e = cudaLaunchKernelEx(&cfg, select_warp_kernel<16>, p, block_scores, sel, sel_copy);
     else e = cudaLaunchKernelEx(&cfg, select_warp_kernel<32>, p, block_scores, sel, sel_copy);
     if (e != cudaSuccess) return MSA_ECUDA;

@@ -4,14 +4,19 @@
 // block is always kept" ("vLLM Adds Day-0 Support for MiniMax-M3.1-Flash",
 // ainewsbites.com, "A model built for efficient inference").  Reading: the query's own
 // block r plus the best min(15, r) other blocks under the total order (score desc,
-// index asc), written ascending and padded with -1.
+// index asc), written ascending and padded with -1.  r = nvis - 1 is the last visible
+// block, so it always comes last in the ascending list.
 //
-// Each candidate becomes a 64-bit key (order-preserving bits of the fp32 score, then the
-// inverted block index), so "best" is a plain maximum and ties go to the lower index.
-// Lane i holds candidates i, i + 32, ... in registers; every round takes, per lane, the
-// largest key below the previous winner with a depth-log2(PER) tree, then the warp
-// maximum with two 32-bit redux.sync.  Deterministic.  A key of 0 marks an empty slot
-// (scores are never NaN, so every real key is non-zero).
+// Threshold selection (select_row_warp): every candidate becomes a 32-bit key whose
+// unsigned order is the order of the fp32 scores (-0 ranks below +0; 0 marks an empty
+// slot: scores are never NaN).  Lane i holds candidates i, i + 32, ... in registers.
+// Rounds of "largest key below the previous one, and how many candidates hold it"
+// (two redux.sync each) find T, the want-th best key counted with multiplicity; then
+// one ballot pass in ascending block order writes every block with key > T and, of
+// the blocks with key == T, the lowest-indexed ones still needed — the index tie-break.
+// Rows longer than 32 * PER blocks take select_row_warp_long: 64-bit keys (score key,
+// inverted index) and 15 rounds of "largest key below the previous winner" per chunk
+// of 32 * PER blocks, the best keys so far carried along.  Both are deterministic.
 #pragma once
 
 #include "common.cuh"
@@ -32,12 +37,86 @@ __device__ __forceinline__ uint64_t warp_max64(uint64_t v) {
     return ((uint64_t)hi << 32) | lo;
 }
 
-// Selection of row `s` (nvis visible blocks, forced block r = nvis - 1).  Rows longer than
-// 32 * PER blocks are taken in chunks of that size, the best keys so far carried along.
-// kCoherent: the scores were written by other warps of the same launch (read through L2).
-// Returns, in lane i < 16, the i-th selected block id in ascending order (or -1).
+// Unsigned key with the order of the fp32 score.
+__device__ __forceinline__ uint32_t score_key(float s) {
+    const uint32_t u = __float_as_uint(s);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// T = the want-th largest of the warp's non-zero keys counted with multiplicity, and
+// n_gt = how many keys exceed it.  Needs 1 <= want <= the number of non-zero keys.
+template <int PER>
+__device__ __forceinline__ uint32_t warp_kth_key(const uint32_t (&k)[PER], int want, int& n_gt) {
+    uint32_t prev = 0xFFFFFFFFu;  // above every finite score's key
+    int taken = 0;
+    for (;;) {
+        uint32_t m = 0u;
+#pragma unroll
+        for (int j = 0; j < PER; ++j) m = max(m, k[j] < prev ? k[j] : 0u);
+        const uint32_t v = __reduce_max_sync(0xffffffffu, m);
+        int c = 0;
+#pragma unroll
+        for (int j = 0; j < PER; ++j) c += k[j] == v ? 1 : 0;
+        c = (int)__reduce_add_sync(0xffffffffu, (unsigned)c);
+        if (taken + c >= want) {
+            n_gt = taken;
+            return v;
+        }
+        taken += c;
+        prev = v;
+    }
+}
+
+// Calls put(slot, j) for the lane holding candidate j of the selected ones, slots
+// ascending in candidate order (j-th register of lane l is candidate 32 j + l): every key
+// above T, and the first need_eq keys equal to T.
+template <int PER, class Put>
+__device__ __forceinline__ void warp_compact(const uint32_t (&k)[PER], uint32_t T, int need_eq, int lane, Put&& put) {
+    const uint32_t below = (1u << lane) - 1u;
+    int base = 0;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+        const uint32_t gt = __ballot_sync(0xffffffffu, k[j] > T);
+        uint32_t eq = __ballot_sync(0xffffffffu, k[j] == T);
+        uint32_t keep = 0u;
+        while (need_eq > 0 && eq != 0u) {  // warp-uniform
+            const uint32_t low = eq & (0u - eq);
+            keep |= low;
+            eq ^= low;
+            --need_eq;
+        }
+        const uint32_t sel = gt | keep;
+        if ((sel >> lane) & 1u) put(base + __popc(sel & below), j);
+        base += __popc(sel);
+    }
+}
+
+// Selection of row `s` (nvis <= 32 * PER visible blocks, forced block r = nvis - 1),
+// written to out[0..15] (shared or global memory) by the warp.  kCoherent: the scores
+// were written by other warps of the same launch (read through L2).
 template <int PER, bool kCoherent = false>
-__device__ __forceinline__ int select_row_warp(const float* __restrict__ s, int64_t nvis, int64_t r, int lane) {
+__device__ __forceinline__ void select_row_warp(const float* __restrict__ s, int64_t nvis, int64_t r, int lane,
+                                                int32_t* out) {
+    const int want = (int)min64(kTopK - 1, nvis - 1);
+    if (want > 0) {
+        uint32_t k[PER];
+#pragma unroll
+        for (int j = 0; j < PER; ++j) {
+            const int64_t n = (int64_t)j * 32 + lane;
+            k[j] = (n < nvis && n != r) ? score_key(kCoherent ? __ldcg(s + n) : __ldg(s + n)) : 0u;
+        }
+        int n_gt;
+        const uint32_t T = warp_kth_key(k, want, n_gt);
+        warp_compact(k, T, want - n_gt, lane, [&](int slot, int j) { out[slot] = j * 32 + lane; });
+    }
+    if (lane == want) out[want] = (int32_t)r;
+    if (lane > want && lane < kTopK) out[lane] = -1;
+}
+
+// Any row length: chunks of 32 * PER blocks, the best keys so far carried along.  Returns,
+// in lane i < 16, the i-th selected block id in ascending order (or -1).
+template <int PER, bool kCoherent = false>
+__device__ __forceinline__ int select_row_warp_long(const float* __restrict__ s, int64_t nvis, int64_t r, int lane) {
     const int want = (int)min64(kTopK - 1, nvis - 1);
     uint64_t best = 0ull;  // lane k < want: the k-th best key among the blocks seen so far
     for (int64_t base = 0; base < nvis; base += 32 * PER) {

@@ -5,8 +5,8 @@
 Builds the workload's NVFP4 caches on the GPU (library encoder), releases every
 temporary so only the kernel's own operands stay allocated, then launches the
 chosen step ``--launches`` times on one stream (index = msa_index, select =
-msa_select, attend = msa_attend, decode = msa_decode) and checks the device
-status word.  Used to make the ncu summaries under profiles/.
+msa_select, attend = msa_attend, decode = msa_decode, single =
+msa_decode_single_launch) and checks the device status word.  Used to make the ncu summaries under profiles/.
 """
 from __future__ import annotations
 
@@ -38,19 +38,23 @@ def build(w: synth.Workload, with_kv: bool, device="cuda"):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--workload", default=configs.DECODE_B32_64K.name, choices=sorted(configs.BY_NAME))
-    ap.add_argument("--kernel", default="index", choices=["index", "select", "attend", "decode"])
+    ap.add_argument("--kernel", default="index", choices=["index", "select", "attend", "decode", "single"])
     ap.add_argument("--launches", type=int, default=3)
     a = ap.parse_args(argv)
     w = configs.BY_NAME[a.workload]
     torch.cuda.set_device(0)
     msa.lib()
-    p = build(w, with_kv=a.kernel in ("attend", "decode"))
+    p = build(w, with_kv=a.kernel in ("attend", "decode", "single"))
     lmax = p.ik.data.shape[2]
     B, Tq = w.B, w.Tq
     bs = torch.empty(B, Tq, lmax // 128, dtype=torch.float32, device="cuda")
     sel = torch.empty(B, Tq, 16, dtype=torch.int32, device="cuda")
     out, lse, _ = msa.outputs(p)
-    ws = msa.alloc_workspace(p) if a.kernel == "decode" else None
+    ws = None
+    if a.kernel == "decode":
+        ws = msa.alloc_workspace(p)
+    elif a.kernel == "single":
+        ws = msa.alloc_workspace_single_launch(p)
     torch.cuda.empty_cache()
     s = torch.cuda.current_stream()
     if a.kernel in ("select", "attend"):
@@ -63,8 +67,10 @@ def main(argv=None):
             msa.msa_select(p, bs, sel)
         elif a.kernel == "attend":
             msa.msa_attend(p, sel, out, lse)
-        else:
+        elif a.kernel == "decode":
             msa.msa_decode(p, ws, out, lse, None)
+        else:
+            msa.msa_decode_single_launch(p, ws, out, lse, None)
     s.synchronize()
     st = int(p.status.item())
     print(f"profile_case {a.workload} {a.kernel} x{a.launches}: status={st}, "
