@@ -227,11 +227,18 @@ def time_oracle(samples):
 
 
 def _concat(samples):
+    """One batch from per-sequence samples; caches zero-padded to the longest sequence (the
+    oracle reads every sequence only up to its own length)."""
     import oracle as O
     qs = np.concatenate([s[0] for s in samples])
     qis = np.concatenate([s[1] for s in samples])
-    cat = lambda i: O.Nvfp4(np.concatenate([s[i].data for s in samples]),  # noqa: E731
-                            np.concatenate([s[i].scale for s in samples]), samples[0][i].tensor_scale)
+    lmax = max(s[2].data.shape[2] for s in samples)
+
+    def pad(a):
+        return np.pad(a, [(0, 0), (0, 0), (0, lmax - a.shape[2]), (0, 0)])
+
+    cat = lambda i: O.Nvfp4(np.concatenate([pad(s[i].data) for s in samples]),  # noqa: E731
+                            np.concatenate([pad(s[i].scale) for s in samples]), samples[0][i].tensor_scale)
     return qs, qis, cat(2), cat(3), cat(4), [s[5][0] for s in samples]
 
 
