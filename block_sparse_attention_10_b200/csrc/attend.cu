@@ -67,9 +67,6 @@ __global__ void __cluster_dims__(kAttCluster, 1, 1) __launch_bounds__(kAttThread
     }
     __syncwarp();
 
-    pdl_wait();
-    pdl_launch_dependents();
-
     cg::cluster_group cluster = cg::this_cluster();
     const int crank = (int)cluster.block_rank();
     const int64_t unit = blockIdx.x / kAttCluster;  // ((b * Tq) + t) * Hkv + kvh
@@ -81,8 +78,14 @@ __global__ void __cluster_dims__(kAttCluster, 1, 1) __launch_bounds__(kAttThread
     const int64_t nvis = pos / kBlock + 1;
     const int gw = crank * kAttWarps + warp;
 
+    // The queries and lengths are not written by the kernel this one waits for (the
+    // indexer or the selection, which waited for their own predecessors before letting
+    // this grid start), so they load before the wait.
     uint32_t qf[1][8][2];
     att_load_q(p, bt, kvh, G, g, c, qf);
+
+    pdl_wait();
+    pdl_launch_dependents();
 
     int blk;
     if constexpr (FUSED) {

@@ -10,7 +10,9 @@
 //   softmax        online over quarters, exp2 domain, fp32; the running output is only
 //                  rescaled when a quarter raises the running max;
 //   O^T += V^T P^T mma m16n8k16, A = dequantised V, B = P^T taken from the S^T
-//                  accumulators by one movmatrix (8x8 transpose) per 8 keys.
+//                  accumulators by one movmatrix (8x8 transpose) per 8 keys.  The A
+//                  fragment pairs two keys per dim: the two keys' nibbles are interleaved
+//                  bytewise first, so each converted f16x2 already holds that pair.
 // Shared by the attention kernel (attend.cu) and the single-launch decode kernel
 // (decode_fused.cu).  A quarter stage is K nibbles (32 x 64 B), K scales (32 x 8 B),
 // V nibbles, V scales: 4.5 KB, the same size as an indexer stage.
@@ -137,29 +139,48 @@ __device__ __forceinline__ void att_quarter(const uint8_t* st, int qvalid, bool 
             // P^T fragment (keys x heads) -> B operand (k = keys 2c.., n = head g)
             const uint32_t pb0 = movmatrix_trans(pack_f16x2(s4[kt][0], s4[kt][1]));
             const uint32_t pb1 = movmatrix_trans(pack_f16x2(s4[kt][2], s4[kt][3]));
-            uint32_t vh[4][8];
+            // V^T A fragments: for each key pair (2c, 2c+1) and (2c+8, 2c+9), interleave the two
+            // keys' nibbles so that each byte holds one dim of both keys; the converter then
+            // yields (key a, key b) f16x2 pairs of one dim directly
+            // va[pr][m] / vb[pr][m]: f16x2 (key a, key b) of dim 16g + 2m / 16g + 2m + 1
+            uint32_t va[2][8], vb[2][8];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int key = kt * 16 + 2 * c + (i & 1) + 8 * (i >> 1);
-                uint2 vw = make_uint2(0u, 0u);
-                uint32_t vs = 0u;
-                if (qvalid == kAttQuarter || key < qvalid) {  // masked keys read as 0 (P is 0; V may hold anything)
-                    vw = lds_v2(vd + key * 64 + g * 8);
-                    vs = lds_u8(vsc + key * 8 + g);
+            for (int pr = 0; pr < 2; ++pr) {
+                const int ka = kt * 16 + 2 * c + 8 * pr, kb = ka + 1;
+                uint2 wa = make_uint2(0u, 0u), wb = make_uint2(0u, 0u);
+                uint32_t sa = 0u, sb = 0u;
+                if (qvalid == kAttQuarter || ka < qvalid) {
+                    wa = lds_v2(vd + ka * 64 + g * 8);
+                    sa = lds_u8(vsc + ka * 8 + g);
                 }
-                e2m1x8_to_f16x8(vw.x, vh[i][0], vh[i][1], vh[i][2], vh[i][3]);
-                e2m1x8_to_f16x8(vw.y, vh[i][4], vh[i][5], vh[i][6], vh[i][7]);
-                const uint32_t sc = e4m3_bcast_f16x2(vs);
+                if (qvalid == kAttQuarter || kb < qvalid) {
+                    wb = lds_v2(vd + kb * 64 + g * 8);
+                    sb = lds_u8(vsc + kb * 8 + g);
+                }
+                const uint32_t sc = e4m3x2_to_f16x2(sa | (sb << 8));  // (scale a, scale b)
 #pragma unroll
-                for (int m = 0; m < 8; ++m) vh[i][m] = hmul2(vh[i][m], sc);
+                for (int h = 0; h < 2; ++h) {
+                    const uint32_t A = h ? wa.y : wa.x, Bw = h ? wb.y : wb.x;
+                    const uint32_t ev = (A & 0x0F0F0F0Fu) | ((Bw << 4) & 0xF0F0F0F0u);  // dims 8h + 0, 2, 4, 6
+                    const uint32_t od = ((A >> 4) & 0x0F0F0F0Fu) | (Bw & 0xF0F0F0F0u);  // dims 8h + 1, 3, 5, 7
+                    uint32_t e0, e1, e2, e3, o0, o1, o2, o3;
+                    e2m1x8_to_f16x8(ev, e0, e1, e2, e3);
+                    e2m1x8_to_f16x8(od, o0, o1, o2, o3);
+                    // e2m1x8_to_f16x8 pairs nibbles (2k, 2k+1) of its word, i.e. byte k = (key a, key b) of one dim
+                    va[pr][4 * h + 0] = hmul2(e0, sc);  // dim 8h + 0
+                    va[pr][4 * h + 1] = hmul2(e1, sc);  // dim 8h + 2
+                    va[pr][4 * h + 2] = hmul2(e2, sc);  // dim 8h + 4
+                    va[pr][4 * h + 3] = hmul2(e3, sc);  // dim 8h + 6
+                    vb[pr][4 * h + 0] = hmul2(o0, sc);  // dim 8h + 1
+                    vb[pr][4 * h + 1] = hmul2(o1, sc);  // dim 8h + 3
+                    vb[pr][4 * h + 2] = hmul2(o2, sc);  // dim 8h + 5
+                    vb[pr][4 * h + 3] = hmul2(o3, sc);  // dim 8h + 7
+                }
             }
 #pragma unroll
             for (int mt = 0; mt < 8; ++mt) {
-                const uint32_t a0 = prmt(vh[0][mt], vh[1][mt], 0x5410u);
-                const uint32_t a1 = prmt(vh[0][mt], vh[1][mt], 0x7632u);
-                const uint32_t a2 = prmt(vh[2][mt], vh[3][mt], 0x5410u);
-                const uint32_t a3 = prmt(vh[2][mt], vh[3][mt], 0x7632u);
-                mma16816(a.o[mt], a0, a1, a2, a3, pb0, pb1);
+                // rows g / g+8 of m-tile mt are dims 16g + 2mt / 16g + 2mt + 1
+                mma16816(a.o[mt], va[0][mt], vb[0][mt], va[1][mt], vb[1][mt], pb0, pb1);
             }
         }
     }
