@@ -8,8 +8,10 @@
 //
 // Design (B200): one thread-block cluster of 4 CTAs x 4 warps per
 // (sequence, query token, KV head): each of the 16 warps takes one selected
-// block (split-K over the <= 16 blocks).  Each warp streams its block as four
-// 32-key quarters (K and V nibbles + scales, 4.5 KB each) through a private
+// block (split-K over the <= 16 blocks); grids of few such units (at most half
+// the SM count) use clusters of 8 CTAs, two warps per block, to halve each
+// warp's serial chain.  Each warp streams its keys as 32-key quarters
+// (K and V nibbles + scales, 4.5 KB each) through a private
 // 2-stage shared-memory ring with untiled bulk copies (cp.async.bulk, no
 // multicast), so the next quarter lands while the current one is computed;
 // 37 KB of shared memory and <= 128 registers per CTA let 4 CTAs (16 warps)
@@ -17,11 +19,11 @@
 // per-quarter step (S^T = K Q^T, online softmax, O^T += V^T P^T on mma.sync
 // m16n8k16 with K and V dequantised in registers) is att_quarter() of
 // attend_quarter.cuh.
-// The partial (m, l, O) of the 4 warps are merged in shared memory, then the 4
+// The partial (m, l, O) of the 4 warps are merged in shared memory, then the
 // CTAs of the cluster merge through distributed shared memory (each CTA
-// finalises 32 of the 128 dims).  With the selection fused in (rows of <= 1,024
-// blocks), warp 0 of every CTA first selects the row's blocks.  No global scratch, no second launch, a
-// fixed merge order (bitwise deterministic).
+// finalises 128 / CL of the 128 dims).  With the selection fused in (rows of
+// <= 1,024 blocks), warp 0 of every CTA first selects the row's blocks.  No global scratch,
+// no second launch, a fixed merge order (bitwise deterministic).
 #include <cooperative_groups.h>
 
 #include "internal.h"
@@ -34,7 +36,6 @@ namespace {
 namespace cg = cooperative_groups;
 
 constexpr int kAttWarps = 4;
-constexpr int kAttCluster = 4;
 constexpr int kAttThreads = 32 * kAttWarps;
 constexpr int kD = kAttD;
 constexpr int64_t kFusedSelectMaxBlocks = 1024;  // rows one warp selects from registers
@@ -43,10 +44,10 @@ constexpr int64_t kFusedSelectMaxBlocks = 1024;  // rows one warp selects from r
 constexpr int kWarpSmem = 2 * kAttStageBytes;  // 9 KB: also holds the warp's partial O (4 KB) at the end
 constexpr size_t kAttSmem = (size_t)kAttWarps * kWarpSmem + 2 * kAttWarps * sizeof(uint64_t) + 2 * 8 * sizeof(float);
 
-// FUSED: the CTA first selects its row's blocks from the pooled scores (warp 0,
-// rows of <= 1,024 blocks) instead of reading a selection written by select.cu.
-template <int G, bool FUSED>
-__global__ void __cluster_dims__(kAttCluster, 1, 1) __launch_bounds__(kAttThreads, 4)
+// FUSED: the CTA first selects its row's blocks from the pooled scores (warp 0, rows of
+// <= 1,024 blocks) instead of reading a selection written by select.cu.
+template <int G, bool FUSED, int CL>
+__global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(kAttThreads, 4)
     attend_kernel(const Problem p, const int32_t* __restrict__ sel, const float* __restrict__ block_scores,
                   int32_t* __restrict__ sel_out, float* __restrict__ out, float* __restrict__ lse) {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -69,7 +70,9 @@ __global__ void __cluster_dims__(kAttCluster, 1, 1) __launch_bounds__(kAttThread
 
     cg::cluster_group cluster = cg::this_cluster();
     const int crank = (int)cluster.block_rank();
-    const int64_t unit = blockIdx.x / kAttCluster;  // ((b * Tq) + t) * Hkv + kvh
+    constexpr int kWPB = CL / 4;             // warps per selected block (1 or 2)
+    constexpr int kQPW = 4 / kWPB;           // quarters per warp
+    const int64_t unit = blockIdx.x / CL;  // ((b * Tq) + t) * Hkv + kvh
     const int kvh = (int)(unit % p.Hkv);
     const int64_t bt = unit / p.Hkv;
     const int b = (int)(bt / p.Tq), t = (int)(bt % p.Tq);
@@ -89,18 +92,18 @@ __global__ void __cluster_dims__(kAttCluster, 1, 1) __launch_bounds__(kAttThread
 
     int blk;
     if constexpr (FUSED) {
+        const float* srow = block_scores + bt * p.nbmax;
+        const int64_t r = nvis - 1;
         if (warp == 0) {
-            const float* srow = block_scores + bt * p.nbmax;
-            const int64_t r = nvis - 1;
             if (nvis <= 512) select_row_warp<16>(srow, nvis, r, lane, sh_sel);
             else select_row_warp<32>(srow, nvis, r, lane, sh_sel);
-            __syncwarp();
-            if (lane < kTopK && sel_out != nullptr && crank == 0 && kvh == 0) sel_out[bt * kTopK + lane] = sh_sel[lane];
         }
         __syncthreads();
-        blk = gw < kTopK ? sh_sel[gw] : -1;
+        if (warp == 0 && lane < kTopK && sel_out != nullptr && crank == 0 && kvh == 0)
+            sel_out[bt * kTopK + lane] = sh_sel[lane];
+        blk = sh_sel[gw / kWPB];
     } else {
-        blk = gw < kTopK ? sel[bt * kTopK + gw] : -1;
+        blk = sel[bt * kTopK + gw / kWPB];
     }
     if (blk >= nvis) {
         if (lane == 0) set_status(p.status, MSA_STATUS_SELECT);
@@ -109,8 +112,9 @@ __global__ void __cluster_dims__(kAttCluster, 1, 1) __launch_bounds__(kAttThread
     int nk = 0, nq = 0;
     int64_t vec0 = 0;
     if (blk >= 0) {
-        const int64_t kbase = (int64_t)blk * kBlock;
-        nk = (int)min64(kBlock, pos + 1 - kbase);
+        // this warp's part of the block: keys [part * 32 kQPW, (part + 1) * 32 kQPW)
+        const int64_t kbase = (int64_t)blk * kBlock + (gw % kWPB) * (kQPW * kAttQuarter);
+        nk = (int)max64(0, min64(kQPW * kAttQuarter, pos + 1 - kbase));
         nq = (nk + kAttQuarter - 1) / kAttQuarter;
         vec0 = ((int64_t)b * p.Hkv + kvh) * p.lmax + kbase;
     }
@@ -188,15 +192,15 @@ __global__ void __cluster_dims__(kAttCluster, 1, 1) __launch_bounds__(kAttThread
     }
     cluster.sync();
 
-    // ---- merge the 4 CTAs of the cluster: CTA r finalises dim pairs [16r, 16r + 16) — float2
-    // slot 128 r + t of the (pair, head) array: head t % 8, pair 16 r + t / 8
-    {
-        const int e = 128 * crank + threadIdx.x;
+    // ---- merge the CL CTAs of the cluster: CTA r finalises float2 slots [512 r / CL,
+    // 512 (r + 1) / CL) of the (pair, head) array; slot e holds head e % 8 of dim pair e / 8
+    if (threadIdx.x < 512 / CL) {
+        const int e = (512 / CL) * crank + threadIdx.x;
         const int q = e & 7, pi = e >> 3;
-        float Mr[kAttCluster], Lr[kAttCluster];
-        float2 Or[kAttCluster];
+        float Mr[CL], Lr[CL];
+        float2 Or[CL];
 #pragma unroll
-        for (int r = 0; r < kAttCluster; ++r) {
+        for (int r = 0; r < CL; ++r) {
             const float* pm = cluster.map_shared_rank(cM, r);
             const float* pl = cluster.map_shared_rank(cL, r);
             const float2* po = reinterpret_cast<const float2*>(cluster.map_shared_rank(sO0, r));
@@ -206,10 +210,10 @@ __global__ void __cluster_dims__(kAttCluster, 1, 1) __launch_bounds__(kAttThread
         }
         float M = -INFINITY;
 #pragma unroll
-        for (int r = 0; r < kAttCluster; ++r) M = fmaxf(M, Mr[r]);
+        for (int r = 0; r < CL; ++r) M = fmaxf(M, Mr[r]);
         float Lt = 0.0f, a0 = 0.0f, a1 = 0.0f;
 #pragma unroll
-        for (int r = 0; r < kAttCluster; ++r) {
+        for (int r = 0; r < CL; ++r) {
             const float f = Mr[r] == -INFINITY ? 0.0f : exp2f(Mr[r] - M);
             Lt += f * Lr[r];
             a0 += f * Or[r].x;
@@ -226,20 +230,20 @@ __global__ void __cluster_dims__(kAttCluster, 1, 1) __launch_bounds__(kAttThread
     cluster.sync();  // keep this CTA's shared memory alive until every peer has read it
 }
 
-template <int G, bool FUSED>
+template <int G, bool FUSED, int CL>
 int launch_g(const Problem& p, const int32_t* sel, const float* bs, int32_t* sel_out, float* out, float* lse,
              bool pdl, cudaStream_t st) {
     const int64_t units = (int64_t)p.B * p.Tq * p.Hkv;
     static int configured_dev = -1;
     const DeviceInfo& di = device_info();
     if (configured_dev != di.device) {
-        if (cudaFuncSetAttribute(attend_kernel<G, FUSED>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(attend_kernel<G, FUSED, CL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)kAttSmem) != cudaSuccess)
             return MSA_ECUDA;
         configured_dev = di.device;
     }
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(units * kAttCluster));
+    cfg.gridDim = dim3((unsigned)(units * CL));
     cfg.blockDim = dim3(kAttThreads);
     cfg.dynamicSmemBytes = kAttSmem;
     cfg.stream = st;
@@ -248,9 +252,19 @@ int launch_g(const Problem& p, const int32_t* sel, const float* bs, int32_t* sel
     attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, attend_kernel<G, FUSED>, p, sel, bs, sel_out, out, lse) != cudaSuccess)
+    if (cudaLaunchKernelEx(&cfg, attend_kernel<G, FUSED, CL>, p, sel, bs, sel_out, out, lse) != cudaSuccess)
         return MSA_ECUDA;
     return MSA_OK;
+}
+
+// Few (row, KV head) units (at most half the SM count): clusters of 8 CTAs, two warps per
+// selected block, so each warp's serial chain is half as long; otherwise clusters of 4.
+template <int G, bool FUSED>
+int launch_cl(const Problem& p, const int32_t* sel, const float* bs, int32_t* sel_out, float* out, float* lse,
+              bool pdl, cudaStream_t st) {
+    const int64_t units = (int64_t)p.B * p.Tq * p.Hkv;
+    if (2 * units <= device_info().num_sms) return launch_g<G, FUSED, 8>(p, sel, bs, sel_out, out, lse, pdl, st);
+    return launch_g<G, FUSED, 4>(p, sel, bs, sel_out, out, lse, pdl, st);
 }
 
 template <bool FUSED>
@@ -258,12 +272,12 @@ int launch_any(const Problem& p, const int32_t* sel, const float* bs, int32_t* s
                bool pdl, cudaStream_t st) {
     if (p.D != kD) return MSA_EUNSUPPORTED;
     const int64_t units = (int64_t)p.B * p.Tq * p.Hkv;
-    if (units * kAttCluster > 0x7FFFFFFFll) return MSA_EUNSUPPORTED;
+    if (units * 8 > 0x7FFFFFFFll) return MSA_EUNSUPPORTED;
     switch (p.Hq / p.Hkv) {
-        case 1: return launch_g<1, FUSED>(p, sel, bs, sel_out, out, lse, pdl, st);
-        case 2: return launch_g<2, FUSED>(p, sel, bs, sel_out, out, lse, pdl, st);
-        case 4: return launch_g<4, FUSED>(p, sel, bs, sel_out, out, lse, pdl, st);
-        case 8: return launch_g<8, FUSED>(p, sel, bs, sel_out, out, lse, pdl, st);
+        case 1: return launch_cl<1, FUSED>(p, sel, bs, sel_out, out, lse, pdl, st);
+        case 2: return launch_cl<2, FUSED>(p, sel, bs, sel_out, out, lse, pdl, st);
+        case 4: return launch_cl<4, FUSED>(p, sel, bs, sel_out, out, lse, pdl, st);
+        case 8: return launch_cl<8, FUSED>(p, sel, bs, sel_out, out, lse, pdl, st);
         default: return MSA_EUNSUPPORTED;
     }
 }

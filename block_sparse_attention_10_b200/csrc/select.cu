@@ -27,13 +27,12 @@ constexpr int kPer = 16;  // candidates per thread held in registers (rows of <=
 // Rows of <= 4,096 blocks: one CTA of 8 warps per (sequence, query token), two levels.
 constexpr int kCtaPer = 16;  // 8 warps x 32 lanes x 16 candidates
 constexpr int kCtaMaxBlocks = kSelWarps * 32 * kCtaPer;
-constexpr int kCand = kTopK - 1;  // candidates kept per chunk
 
 __global__ void __launch_bounds__(kSelThreads)
     select_cta_kernel(const Problem p, const float* __restrict__ block_scores, int32_t* __restrict__ sel,
                       int32_t* __restrict__ sel_copy) {
-    __shared__ uint32_t ckey[kSelWarps * kCand];
-    __shared__ int32_t cid[kSelWarps * kCand];
+    __shared__ uint32_t ckey[kSelWarps * (kTopK - 1)];
+    __shared__ int32_t cid[kSelWarps * (kTopK - 1)];
     __shared__ int32_t res[kTopK];
     pdl_wait();
     pdl_launch_dependents();
@@ -42,48 +41,8 @@ __global__ void __launch_bounds__(kSelThreads)
     const int b = (int)(row / p.Tq), t = (int)(row % p.Tq);
     const int64_t L = clamp_len(p.seq_lens[b], p.Tq, p.lmax, nullptr);
     const int64_t r = (L - p.Tq + t) / kBlock;  // forced block
-    const int64_t nvis = r + 1;
-    const float* s = block_scores + row * p.nbmax;
-
-    // level 1: the best 15 of this warp's chunk, in ascending block order
-    const int base = warp * 32 * kCtaPer;
-    uint32_t k[kCtaPer];
-    int cnt = 0;
-#pragma unroll
-    for (int j = 0; j < kCtaPer; ++j) {
-        const int64_t n = base + j * 32 + lane;
-        k[j] = (n < nvis && n != r) ? score_key(__ldg(s + n)) : 0u;
-        cnt += k[j] != 0u ? 1 : 0;
-    }
-    cnt = (int)__reduce_add_sync(0xffffffffu, (unsigned)cnt);
-    const int want_w = min(kCand, cnt);
-    if (want_w > 0) {
-        int n_gt;
-        const uint32_t T = warp_kth_key(k, want_w, n_gt);
-        warp_compact(k, T, want_w - n_gt, lane, [&](int slot, int j) {
-            ckey[warp * kCand + slot] = k[j];
-            cid[warp * kCand + slot] = base + j * 32 + lane;
-        });
-    }
-    if (lane >= want_w && lane < kCand) ckey[warp * kCand + lane] = 0u;
-    __syncthreads();
-
-    // level 2: the row's best 15 among the 120 candidates
+    select_row_cta<kSelWarps, kCtaPer>(block_scores + row * p.nbmax, r + 1, r, warp, lane, ckey, cid, res);
     if (warp != 0) return;
-    const int want = (int)min64(kCand, nvis - 1);
-    if (want > 0) {
-        uint32_t kk[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int c = j * 32 + lane;
-            kk[j] = c < kSelWarps * kCand ? ckey[c] : 0u;
-        }
-        int n_gt;
-        const uint32_t T = warp_kth_key(kk, want, n_gt);
-        warp_compact(kk, T, want - n_gt, lane, [&](int slot, int j) { res[slot] = cid[j * 32 + lane]; });
-    }
-    if (lane == want) res[want] = (int32_t)r;
-    if (lane > want && lane < kTopK) res[lane] = -1;
     __syncwarp();
     if (lane < kTopK) {
         sel[row * kTopK + lane] = res[lane];

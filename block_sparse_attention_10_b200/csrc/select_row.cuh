@@ -113,6 +113,55 @@ __device__ __forceinline__ void select_row_warp(const float* __restrict__ s, int
     if (lane > want && lane < kTopK) out[lane] = -1;
 }
 
+// Rows of <= WARPS * 32 * PER blocks, selected by the WARPS warps of a CTA: warp w keeps the
+// best 15 of blocks [32 PER w, 32 PER (w + 1)) in shared memory (ckey/cid, WARPS * 15
+// entries each), in ascending block order; then warp 0 selects the row's best 15 from those
+// candidates (they contain it), which sit in ascending block order, so the index tie-break
+// carries over, and writes out[0..15].  Every thread of the CTA calls it (one barrier).
+template <int WARPS, int PER, bool kCoherent = false>
+__device__ __forceinline__ void select_row_cta(const float* __restrict__ s, int64_t nvis, int64_t r, int warp,
+                                               int lane, uint32_t* ckey, int32_t* cid, int32_t* out) {
+    constexpr int kCand = kTopK - 1;
+    const int base = warp * 32 * PER;
+    uint32_t k[PER];
+    int cnt = 0;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+        const int64_t n = base + j * 32 + lane;
+        k[j] = (n < nvis && n != r) ? score_key(kCoherent ? __ldcg(s + n) : __ldg(s + n)) : 0u;
+        cnt += k[j] != 0u ? 1 : 0;
+    }
+    cnt = (int)__reduce_add_sync(0xffffffffu, (unsigned)cnt);
+    const int want_w = min(kCand, cnt);
+    if (want_w > 0) {
+        int n_gt;
+        const uint32_t T = warp_kth_key(k, want_w, n_gt);
+        warp_compact(k, T, want_w - n_gt, lane, [&](int slot, int j) {
+            ckey[warp * kCand + slot] = k[j];
+            cid[warp * kCand + slot] = base + j * 32 + lane;
+        });
+    }
+    if (lane >= want_w && lane < kCand) ckey[warp * kCand + lane] = 0u;
+    __syncthreads();
+    if (warp != 0) return;
+    constexpr int kC = WARPS * kCand;
+    constexpr int kPer2 = (kC + 31) / 32;
+    const int want = (int)min64(kCand, nvis - 1);
+    if (want > 0) {
+        uint32_t kk[kPer2];
+#pragma unroll
+        for (int j = 0; j < kPer2; ++j) {
+            const int cc = j * 32 + lane;
+            kk[j] = cc < kC ? ckey[cc] : 0u;
+        }
+        int n_gt;
+        const uint32_t T = warp_kth_key(kk, want, n_gt);
+        warp_compact(kk, T, want - n_gt, lane, [&](int slot, int j) { out[slot] = cid[j * 32 + lane]; });
+    }
+    if (lane == want) out[want] = (int32_t)r;
+    if (lane > want && lane < kTopK) out[lane] = -1;
+}
+
 // Any row length: chunks of 32 * PER blocks, the best keys so far carried along.  Returns,
 // in lane i < 16, the i-th selected block id in ascending order (or -1).
 template <int PER, bool kCoherent = false>

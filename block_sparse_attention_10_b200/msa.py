@@ -108,9 +108,10 @@ def _stream(stream=None):
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-@dataclass
+@dataclass(frozen=True)
 class Nvfp4Cache:
-    """An NVFP4 cache tensor: data uint8 [B, H, lmax, dim/2], scale uint8 [B, H, lmax, dim/16], fp32 scale."""
+    """An NVFP4 cache tensor: data uint8 [B, H, lmax, dim/2], scale uint8 [B, H, lmax, dim/16], fp32 scale.
+    Immutable (a new cache is a new object), so a problem's cached parameter block stays valid."""
     data: torch.Tensor
     scale: torch.Tensor
     tensor_scale: float
@@ -138,7 +139,22 @@ class MsaProblem:
     pool_mode: int = 0
     status: Optional[torch.Tensor] = None  # int32/uint32 [1]
 
+    def __setattr__(self, name, value):
+        # any change of a field invalidates the cached parameter block
+        object.__setattr__(self, name, value)
+        if name != "_prm":
+            object.__setattr__(self, "_prm", None)
+
     def params(self) -> _Params:
+        """The ``msa_params_t`` of this problem, built once and reused while no field is
+        reassigned (tensors changed in place keep their addresses)."""
+        prm = getattr(self, "_prm", None)
+        if prm is None:
+            prm = self._build_params()
+            object.__setattr__(self, "_prm", prm)
+        return prm
+
+    def _build_params(self) -> _Params:
         B, Tq, Hq, D = self.q.shape
         HI, DI = self.q_idx.shape[2], self.q_idx.shape[3]
         Hkv = self.k.data.shape[1]

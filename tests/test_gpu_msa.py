@@ -2,7 +2,8 @@
 
 Sizes span several tiles and a ragged tail; edge cases: one key, a context that
 fits in 16 blocks (dense), partial last blocks, multi-token causal queries, GQA
-groups 1..8, indexer heads 1..8, DI 64/128, max pooling, head weights.
+groups 1..8, indexer heads 1..8, DI 64/128, max pooling, head weights, rows of more
+than 1,024 blocks (separate two-level selection launch).
 """
 import numpy as np
 import pytest
@@ -38,6 +39,8 @@ CASES = {
     "tq32_hi1": lambda: _custom("e", 1, 32, 8, 2, 1, 128, [6000], 6016),
     "tq2_hi8_dense": lambda: _custom("f", 2, 2, 16, 2, 8, 128, [2048, 1100], 2048),
     "g4_hi4_tq4": lambda: _custom("g", 3, 4, 16, 4, 4, 64, [20000, 128, 129], 20096, needles=6),
+    # rows of > 1,024 blocks: msa_decode selects in its own launch (two-level CTA kernel)
+    "long_rows_tq2": lambda: _custom("h", 2, 2, 8, 1, 4, 64, [150000, 133333], 150016, needles=4),
 }
 
 
