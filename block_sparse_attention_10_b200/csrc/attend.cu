@@ -8,9 +8,9 @@
 //
 // Design (B200): one thread-block cluster of 4 CTAs x 4 warps per
 // (sequence, query token, KV head): each of the 16 warps takes one selected
-// block (split-K over the <= 16 blocks); grids of few such units (at most half
-// the SM count) use clusters of 8 CTAs, two warps per block, to halve each
-// warp's serial chain.  Each warp streams its keys as 32-key quarters
+// block (split-K over the <= 16 blocks); grids of few such units use clusters
+// of 8 CTAs (two warps per block) or 16 (four, one 32-key quarter each) to
+// shorten each warp's serial chain.  Each warp streams its keys as 32-key quarters
 // (K and V nibbles + scales, 4.5 KB each) through a private
 // 2-stage shared-memory ring with untiled bulk copies (cp.async.bulk, no
 // multicast), so the next quarter lands while the current one is computed;
@@ -257,13 +257,49 @@ int launch_g(const Problem& p, const int32_t* sel, const float* bs, int32_t* sel
     return MSA_OK;
 }
 
-// Few (row, KV head) units (at most half the SM count): clusters of 8 CTAs, two warps per
-// selected block, so each warp's serial chain is half as long; otherwise clusters of 4.
+// Clusters of 16 CTAs (a non-portable size: used only where the device accepts it) with 4
+// warps per selected block, one quarter each
+template <int G, bool FUSED>
+bool cluster16_ok() {
+    static int ok_dev = -2, ok = 0;
+    const DeviceInfo& di = device_info();
+    if (ok_dev != di.device) {
+        ok = 0;
+        auto kern = attend_kernel<G, FUSED, 16>;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttSmem) == cudaSuccess) {
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(16);
+            cfg.blockDim = dim3(kAttThreads);
+            cfg.dynamicSmemBytes = kAttSmem;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 16;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int clusters = 0;
+            if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) == cudaSuccess && clusters > 0) ok = 1;
+        }
+        cudaGetLastError();  // a refused query leaves no sticky error behind
+        ok_dev = di.device;
+    }
+    return ok != 0;
+}
+
+// Few (row, KV head) units: clusters of 16 CTAs (one quarter-block per warp) when 16 CTAs per
+// unit still fit in one wave of one CTA per SM, clusters of 8 (two warps per block) when the
+// units are at most half the SM count, else clusters of 4 (one warp per block).  Smaller
+// pieces per warp shorten each warp's serial chain where the grid leaves SMs idle.
 template <int G, bool FUSED>
 int launch_cl(const Problem& p, const int32_t* sel, const float* bs, int32_t* sel_out, float* out, float* lse,
               bool pdl, cudaStream_t st) {
     const int64_t units = (int64_t)p.B * p.Tq * p.Hkv;
-    if (2 * units <= device_info().num_sms) return launch_g<G, FUSED, 8>(p, sel, bs, sel_out, out, lse, pdl, st);
+    const int sms = device_info().num_sms;
+    if (16 * units <= sms && cluster16_ok<G, FUSED>())
+        return launch_g<G, FUSED, 16>(p, sel, bs, sel_out, out, lse, pdl, st);
+    if (2 * units <= sms) return launch_g<G, FUSED, 8>(p, sel, bs, sel_out, out, lse, pdl, st);
     return launch_g<G, FUSED, 4>(p, sel, bs, sel_out, out, lse, pdl, st);
 }
 
