@@ -94,8 +94,9 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(kAttThreads, 4)
     if constexpr (FUSED) {
         const float* srow = block_scores + bt * p.nbmax;
         const int64_t r = nvis - 1;
-        if (warp == 0) {
-            if (nvis <= 512) select_row_warp<16>(srow, nvis, r, lane, sh_sel);
+        if (warp == 0) {  // as few candidate registers per lane as the row needs
+            if (nvis <= 128) select_row_warp<4>(srow, nvis, r, lane, sh_sel);
+            else if (nvis <= 512) select_row_warp<16>(srow, nvis, r, lane, sh_sel);
             else select_row_warp<32>(srow, nvis, r, lane, sh_sel);
         }
         __syncthreads();

@@ -46,7 +46,7 @@ constexpr int kFThreads = 32 * kFWarps;
 constexpr int kFRing = 3;
 constexpr int kFStage = kIdxStageBytes;
 static_assert(kIdxStageBytes == kAttStageBytes, "index and attention stages share the ring");
-constexpr int kItemStages = 4;  // stages per IDX item: 2 blocks at DI = 128, 4 at DI = 64
+constexpr int kItemStages = 8;  // stages per IDX item: 4 blocks at DI = 128, 8 at DI = 64
 constexpr int kAttBlocksPerItem = 2;
 constexpr int kAttItemsPerRow = kTopK / kAttBlocksPerItem;  // partials per (row, KV head)
 constexpr int kPartFloats = 64 * 8 * 2 + 16;                // O [64 dim pairs][8 heads][2], m[8], l[8]

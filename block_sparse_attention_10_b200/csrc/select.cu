@@ -167,6 +167,7 @@ int launch_select(const Problem& p, const float* block_scores, int32_t* sel, int
     if (!short_rows && p.nbmax <= kCtaMaxBlocks)
         e = cudaLaunchKernelEx(&cfg, select_cta_kernel, p, block_scores, sel, sel_copy);
     else if (!short_rows) e = cudaLaunchKernelEx(&cfg, select_kernel, p, block_scores, sel, sel_copy);
+    else if (p.nbmax <= 32 * 4) e = cudaLaunchKernelEx(&cfg, select_warp_kernel<4>, p, block_scores, sel, sel_copy);
     else if (p.nbmax <= 32 * 16) e = cudaLaunchKernelEx(&cfg, select_warp_kernel<16>, p, block_scores, sel, sel_copy);
     else e = cudaLaunchKernelEx(&cfg, select_warp_kernel<32>, p, block_scores, sel, sel_copy);
     if (e != cudaSuccess) return MSA_ECUDA;

@@ -45,25 +45,37 @@ __device__ __forceinline__ uint32_t score_key(float s) {
 
 // T = the want-th largest of the warp's non-zero keys counted with multiplicity, and
 // n_gt = how many keys exceed it.  Needs 1 <= want <= the number of non-zero keys.
+// Each round's multiplicity count and the next round's maximum are independent, so both
+// reductions are in flight together (the last round computes one maximum it does not use).
 template <int PER>
 __device__ __forceinline__ uint32_t warp_kth_key(const uint32_t (&k)[PER], int want, int& n_gt) {
-    uint32_t prev = 0xFFFFFFFFu;  // above every finite score's key
-    int taken = 0;
-    for (;;) {
-        uint32_t m = 0u;
+    auto max_below = [&](uint32_t prev) -> uint32_t {
+        uint32_t m[PER];
 #pragma unroll
-        for (int j = 0; j < PER; ++j) m = max(m, k[j] < prev ? k[j] : 0u);
-        const uint32_t v = __reduce_max_sync(0xffffffffu, m);
+        for (int j = 0; j < PER; ++j) m[j] = k[j] < prev ? k[j] : 0u;
+#pragma unroll
+        for (int w = PER / 2; w >= 1; w >>= 1)
+#pragma unroll
+            for (int j = 0; j < w; ++j) m[j] = max(m[j], m[j + w]);
+        return __reduce_max_sync(0xffffffffu, m[0]);
+    };
+    auto count_eq = [&](uint32_t v) -> int {
         int c = 0;
 #pragma unroll
         for (int j = 0; j < PER; ++j) c += k[j] == v ? 1 : 0;
-        c = (int)__reduce_add_sync(0xffffffffu, (unsigned)c);
+        return (int)__reduce_add_sync(0xffffffffu, (unsigned)c);
+    };
+    int taken = 0;
+    uint32_t v = max_below(0xFFFFFFFFu);  // above every finite score's key
+    for (;;) {
+        const int c = count_eq(v);
+        const uint32_t next = max_below(v);
         if (taken + c >= want) {
             n_gt = taken;
             return v;
         }
         taken += c;
-        prev = v;
+        v = next;
     }
 }
 
