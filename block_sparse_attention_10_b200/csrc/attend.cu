@@ -114,10 +114,11 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(kAttThreads, 4)
     int64_t vec0 = 0;
     if (blk >= 0) {
         // this warp's part of the block: keys [part * 32 kQPW, (part + 1) * 32 kQPW)
-        const int64_t kbase = (int64_t)blk * kBlock + (gw % kWPB) * (kQPW * kAttQuarter);
+        const int part0 = (gw % kWPB) * (kQPW * kAttQuarter);
+        const int64_t kbase = (int64_t)blk * kBlock + part0;
         nk = (int)max64(0, min64(kQPW * kAttQuarter, pos + 1 - kbase));
         nq = (nk + kAttQuarter - 1) / kAttQuarter;
-        vec0 = ((int64_t)b * p.Hkv + kvh) * p.lmax + kbase;
+        vec0 = block_vec(p, b, blk, kvh, p.Hkv) + part0;
     }
     // quarter j of the block -> stage j & 1 (rows rounded up to 16; the cache holds whole blocks)
     auto issue = [&](int j) {

@@ -553,7 +553,8 @@ FusedLayout fused_layout(const Problem& p) {
 }
 
 bool fused_supported(const Problem& p) {
-    return p.B <= kMaxB && (int64_t)p.Tq * p.HI <= 16 && (p.DI == 64 || p.DI == 128) && p.D == kAttD;
+    return p.B <= kMaxB && (int64_t)p.Tq * p.HI <= 16 && (p.DI == 64 || p.DI == 128) && p.D == kAttD &&
+           p.block_table == nullptr;
 }
 
 int launch_decode_fused(const Problem& p, void* ws, float* out, float* lse, int32_t* sel_out, bool pdl,

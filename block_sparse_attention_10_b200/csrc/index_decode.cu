@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
                 if (lane == 0) {
                     const int rows = (min(valid, KPS) + 15) & ~15;
                     const int s = (int)(slot_issued % R);
-                    const int64_t row0 = (int64_t)ib * p.lmax + n * kBlock + is * KPS;
+                    const int64_t row0 = block_vec(p, ib, n, 0, 1) + is * KPS;
                     uint8_t* st = my_stages + s * kIdxStageBytes;
                     const uint32_t db = (uint32_t)(rows * (DI / 2)), sb = (uint32_t)(rows * (DI / 16));
                     mbar_arrive_expect_tx(&my_bars[s], db + sb);

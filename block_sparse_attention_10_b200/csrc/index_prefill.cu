@@ -239,7 +239,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     const int64_t key = k0 + j;
                     uint32_t w = 0u, sc = 0u;
                     if (key < L) {
-                        const int64_t vec = (int64_t)b * p.lmax + key;
+                        const int64_t vec = block_vec(p, b, key / kBlock, 0, 1) + key % kBlock;
                         w = *reinterpret_cast<const uint32_t*>(p.ik.data + vec * (DI / 2) + cr * 4);
                         sc = p.ik.scale[vec * (DI / 16) + (cr >> 1)];
                     }

@@ -39,7 +39,23 @@ struct Problem {
     float softmax_scale;
     int pool_mode;
     uint32_t* status;
+    const int32_t* block_table;  // [B][nbmax] page of each block, or nullptr (contiguous caches)
+    int64_t num_pages;
 };
+
+// First cache vector of block n of sequence b, head h of H: contiguous caches hold
+// [B][H][lmax][...]; paged caches hold pages [num_pages][H][128][...] found through the
+// block table.  A page id outside the pool is flagged and replaced by page 0, so every
+// copy stays inside the pool.
+__device__ __forceinline__ int64_t block_vec(const Problem& p, int b, int64_t n, int h, int H) {
+    if (p.block_table == nullptr) return ((int64_t)b * H + h) * p.lmax + n * kBlock;
+    int64_t page = __ldg(p.block_table + (int64_t)b * p.nbmax + n);
+    if (page < 0 || page >= p.num_pages) {
+        set_status(p.status, MSA_STATUS_PAGE);
+        page = 0;
+    }
+    return (page * H + h) * kBlock;
+}
 
 int launch_nvfp4_encode(const float* x, int64_t nvec, int dim, float s_t, uint8_t* data, uint8_t* scale,
                         cudaStream_t st);

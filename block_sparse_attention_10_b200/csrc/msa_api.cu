@@ -51,6 +51,7 @@ int check_params(const msa_params_t* p, bool need_index, bool need_attend) {
     if (p->lmax > (int64_t(1) << 31)) return MSA_EUNSUPPORTED;
     if (p->Tq > p->lmax) return MSA_EINVAL;
     if (p->pool_mode != 0 && p->pool_mode != 1) return MSA_EINVAL;
+    if (p->block_table != nullptr && p->num_pages <= 0) return MSA_EINVAL;
     if (need_index) {
         if (p->HI <= 0 || p->DI <= 0 || !p->q_idx) return MSA_EINVAL;
         if (int r = check_cache(p->ik)) return r;
@@ -94,6 +95,8 @@ Problem to_problem(const msa_params_t* p) {
     q.softmax_scale = p->softmax_scale > 0.0f ? p->softmax_scale : 1.0f / sqrtf((float)p->D);
     q.pool_mode = p->pool_mode;
     q.status = p->status;
+    q.block_table = p->block_table;
+    q.num_pages = p->block_table != nullptr ? p->num_pages : 0;
     return q;
 }
 

@@ -47,7 +47,8 @@ class _Params(ctypes.Structure):
                 ("D", ctypes.c_int), ("HI", ctypes.c_int), ("DI", ctypes.c_int), ("lmax", ctypes.c_int64),
                 ("seq_lens", ctypes.c_void_p), ("k", _Cache), ("v", _Cache), ("ik", _Cache),
                 ("q", ctypes.c_void_p), ("q_idx", ctypes.c_void_p), ("w_idx", ctypes.c_void_p),
-                ("softmax_scale", ctypes.c_float), ("pool_mode", ctypes.c_int), ("status", ctypes.c_void_p)]
+                ("softmax_scale", ctypes.c_float), ("pool_mode", ctypes.c_int), ("status", ctypes.c_void_p),
+                ("block_table", ctypes.c_void_p), ("num_pages", ctypes.c_int64)]
 
 
 _lib = None
@@ -138,6 +139,9 @@ class MsaProblem:
     softmax_scale: float = 0.0
     pool_mode: int = 0
     status: Optional[torch.Tensor] = None  # int32/uint32 [1]
+    # paged caches: int32 [B, lmax / 128] page of each block; k, v, ik are then page pools
+    # [num_pages, H, 128, dim/2] (+ scales)
+    block_table: Optional[torch.Tensor] = None
 
     def __setattr__(self, name, value):
         # any change of a field invalidates the cached parameter block
@@ -158,14 +162,18 @@ class MsaProblem:
         B, Tq, Hq, D = self.q.shape
         HI, DI = self.q_idx.shape[2], self.q_idx.shape[3]
         Hkv = self.k.data.shape[1]
-        lmax = self.ik.data.shape[2]  # every cache of a problem has the same capacity
-        return _Params(B, Tq, Hq, Hkv, D, HI, DI, lmax, self.seq_lens.data_ptr(), self.k._c(), self.v._c(),
-                       self.ik._c(), self.q.data_ptr(), self.q_idx.data_ptr(),
+        paged = self.block_table is not None
+        return _Params(B, Tq, Hq, Hkv, D, HI, DI, self.nbmax * MSA_BLOCK_TOKENS, self.seq_lens.data_ptr(),
+                       self.k._c(), self.v._c(), self.ik._c(), self.q.data_ptr(), self.q_idx.data_ptr(),
                        None if self.w_idx is None else self.w_idx.data_ptr(), self.softmax_scale, self.pool_mode,
-                       None if self.status is None else self.status.data_ptr())
+                       None if self.status is None else self.status.data_ptr(),
+                       self.block_table.data_ptr() if paged else None, self.ik.data.shape[0] if paged else 0)
 
     @property
     def nbmax(self) -> int:
+        """Blocks per sequence: the cache capacity (contiguous) or the block-table width (paged)."""
+        if self.block_table is not None:
+            return self.block_table.shape[1]
         return self.ik.data.shape[2] // MSA_BLOCK_TOKENS
 
 

@@ -71,6 +71,7 @@ typedef enum msa_status {
 #define MSA_STATUS_SEQLEN 1u   /* some seq_lens[b] < Tq or > lmax: clamped */
 #define MSA_STATUS_SELECT 2u   /* a selected block id >= the visible block count: skipped */
 #define MSA_STATUS_TIMEOUT 4u  /* a bounded wait inside a kernel gave up (results invalid) */
+#define MSA_STATUS_PAGE 8u     /* a block-table page id outside the pool: page 0 read (results invalid) */
 /* With MSA_STATUS_TIMEOUT, which wait gave up: */
 #define MSA_STATUS_AT_INDEX_PRODUCER 0x100u /* indexer: producer waiting for a free stage */
 #define MSA_STATUS_AT_INDEX_DRAIN 0x200u    /* indexer: producer draining its last copies */
@@ -80,7 +81,9 @@ typedef enum msa_status {
 #define MSA_STATUS_AT_DECODE_WAIT 0x2000u   /* single-launch decode: warp waiting for another warp's
                                                pooled scores or selection */
 
-/* One NVFP4 cache tensor (K, V or index-K); the layout is given above. */
+/* One NVFP4 cache tensor (K, V or index-K); the layout is given above.  With a
+ * block table (msa_params_t.block_table) the planes are page pools instead:
+ * data [num_pages][heads][128][dim/2], scale [num_pages][heads][128][dim/16]. */
 typedef struct msa_nvfp4_cache {
     const uint8_t* data;  /* [B][heads][lmax][dim/2], 16-byte aligned */
     const uint8_t* scale; /* [B][heads][lmax][dim/16], 16-byte aligned */
@@ -107,6 +110,12 @@ typedef struct msa_nvfp4_cache {
  *   pool_mode 0 = mean, 1 = max
  *   status    device uint32 status word (bits MSA_STATUS_*), or NULL; kernels
  *             only OR bits into it, the caller clears it
+ *   block_table  NULL for contiguous caches; else a paged cache: device int32
+ *             [B][lmax/128] mapping block n of sequence b to a page of the k, v
+ *             and ik pools (one page = one 128-token MSA block of every head).
+ *             A page id outside [0, num_pages) sets MSA_STATUS_PAGE and page 0
+ *             is read in its place (results invalid)
+ *   num_pages pages in each pool (> 0 with a block table)
  */
 typedef struct msa_params {
     int B, Tq, Hq, Hkv, D, HI, DI;
@@ -119,6 +128,8 @@ typedef struct msa_params {
     float softmax_scale;
     int pool_mode;
     uint32_t* status;
+    const int32_t* block_table;
+    int64_t num_pages;
 } msa_params_t;
 
 /* Human-readable name of an msa_status code (static string, never NULL). */
@@ -202,9 +213,9 @@ int msa_decode(const msa_params_t* p, void* ws, size_t ws_bytes, float* out, flo
  * alternative, not used by msa_decode.
  * ------------------------------------------------------------------------- */
 
-/* Scratch for msa_decode_single_launch (0 if the shape is not supported:
- * it needs Tq * HI <= 16): counters, pooled scores, selection and per-block
- * attention partials. */
+/* Scratch for msa_decode_single_launch (0 if the problem is not supported:
+ * it needs Tq * HI <= 16 and contiguous caches): counters, pooled scores,
+ * selection and per-block attention partials. */
 size_t msa_workspace_size_single_launch(const msa_params_t* p);
 
 /* As msa_decode, in one launch (plus one cudaMemsetAsync that clears the
@@ -212,7 +223,7 @@ size_t msa_workspace_size_single_launch(const msa_params_t* p);
  *   ws, ws_bytes  at least msa_workspace_size_single_launch(p) bytes,
  *                 256-byte aligned; contents on entry are ignored; one call
  *                 at a time may use it
- * Returns MSA_EUNSUPPORTED for Tq * HI > 16.  A wait inside the kernel for
+ * Returns MSA_EUNSUPPORTED for Tq * HI > 16 or a block table.  A wait inside the kernel for
  * another warp's result that exceeds 2 s (all CTAs of the grid must be
  * resident: another kernel holding SMs for that long) sets MSA_STATUS_TIMEOUT
  * | MSA_STATUS_AT_DECODE_WAIT and ends the launch. */

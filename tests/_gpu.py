@@ -22,7 +22,7 @@ def run_steps(p):
     """msa_index -> msa_select -> msa_attend as separate calls."""
     B, Tq = p.q.shape[:2]
     bs = torch.full((B, Tq, p.nbmax), float("nan"), dtype=torch.float32, device=p.q.device)
-    lmax = p.k.data.shape[2]
+    lmax = p.nbmax * 128
     ts = torch.full((B, Tq, lmax), float("nan"), dtype=torch.float32, device=p.q.device)
     msa.msa_index(p, bs, ts)
     sel = torch.empty(B, Tq, 16, dtype=torch.int32, device=p.q.device)
@@ -45,3 +45,29 @@ def run_decode(p, single_launch=False, ws=None):
 
 def status_of(p):
     return 0 if p.status is None else int(p.status.item())
+
+
+def paged_problem(p, extra_pages=7, seed=0, fill=0xAB):
+    """The same problem with its caches scattered into shuffled page pools (one page = one
+    128-token block of every head) and a block table; unused pages hold garbage."""
+    B, nb = p.q.shape[0], p.nbmax
+    g = torch.Generator().manual_seed(seed)
+    npages = B * nb + extra_pages
+    perm = torch.randperm(npages, generator=g)[:B * nb]
+    dev = p.q.device
+    idx = perm.to(dev)
+
+    def scatter(t):
+        H, x = t.shape[1], t.shape[-1]
+        blocks = t.view(B, H, nb, 128, x).permute(0, 2, 1, 3, 4).reshape(B * nb, H, 128, x)
+        out = torch.full((npages, H, 128, x), fill, dtype=torch.uint8, device=dev)
+        out[idx] = blocks
+        return out
+
+    def pool(c):
+        return msa.Nvfp4Cache(scatter(c.data), scatter(c.scale), c.tensor_scale)
+
+    return msa.MsaProblem(seq_lens=p.seq_lens, k=pool(p.k), v=pool(p.v), ik=pool(p.ik), q=p.q, q_idx=p.q_idx,
+                          w_idx=p.w_idx, softmax_scale=p.softmax_scale, pool_mode=p.pool_mode,
+                          status=torch.zeros(1, dtype=torch.int32, device=dev),
+                          block_table=perm.view(B, nb).to(torch.int32).to(dev))

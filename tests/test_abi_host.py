@@ -66,6 +66,27 @@ def test_workspace_size_host_only(L):
     assert L.msa_workspace_size_single_launch(ctypes.byref(bad)) == 0
 
 
+def test_block_table_arguments(L):
+    # a block table needs a positive page count; the single launch does not take paged caches
+    p = _params(block_table=0xA000, num_pages=0)
+    assert L.msa_workspace_size(ctypes.byref(p)) == 0
+    r = L.msa_decode(ctypes.byref(p), ctypes.c_void_p(0x10000), 1 << 20, ctypes.c_void_p(0x20000), None, None, None)
+    assert r == 1
+    p = _params(block_table=0xA000, num_pages=64)
+    assert L.msa_workspace_size(ctypes.byref(p)) == L.msa_workspace_size(ctypes.byref(_params()))
+    assert L.msa_workspace_size_single_launch(ctypes.byref(p)) == 0
+    r = L.msa_decode_single_launch(ctypes.byref(p), ctypes.c_void_p(0x10000), 1 << 30, ctypes.c_void_p(0x20000),
+                                   None, None, None)
+    assert r == 2
+
+
+def test_params_struct_layout(L):
+    # the Python mirror of msa_params_t ends with the block table and the page count
+    names = [f[0] for f in msa._Params._fields_]
+    assert names[-3:] == ["status", "block_table", "num_pages"]
+    assert ctypes.sizeof(msa._Params) == msa._Params.num_pages.offset + 8
+
+
 def test_single_launch_rejects_before_enqueueing(L):
     out = ctypes.c_void_p(0x20000)
     r = L.msa_decode_single_launch(ctypes.byref(_params(Tq=8)), ctypes.c_void_p(0x10000), 1 << 30, out, None, None,
