@@ -118,7 +118,7 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(kAttThreads, 4)
         const int64_t kbase = (int64_t)blk * kBlock + part0;
         nk = (int)max64(0, min64(kQPW * kAttQuarter, pos + 1 - kbase));
         nq = (nk + kAttQuarter - 1) / kAttQuarter;
-        vec0 = block_vec(p, b, blk, kvh, p.Hkv) + part0;
+        vec0 = block_vec_any(p, b, blk, kvh, p.Hkv) + part0;
     }
     // quarter j of the block -> stage j & 1 (rows rounded up to 16; the cache holds whole blocks)
     auto issue = [&](int j) {
@@ -223,8 +223,7 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(kAttThreads, 4)
         }
         if (q < G) {
             const float inv = Lt > 0.0f ? p.v.s_t / Lt : 0.0f;
-            float* orow = out + ((bt * p.Hq) + (int64_t)kvh * G + q) * kD;
-            *reinterpret_cast<float2*>(orow + 2 * pi) = make_float2(a0 * inv, a1 * inv);
+            store_out2(p, out, ((bt * p.Hq) + (int64_t)kvh * G + q) * kD + 2 * pi, a0 * inv, a1 * inv);
             if (lse != nullptr && crank == 0 && threadIdx.x < 8)
                 lse[bt * p.Hq + (int64_t)kvh * G + q] = Lt > 0.0f ? (M + log2f(Lt)) * kLn2 : -INFINITY;
         }

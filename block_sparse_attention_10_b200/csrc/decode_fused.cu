@@ -446,13 +446,12 @@ __global__ void __launch_bounds__(kFThreads, 2) decode_fused_kernel(const Proble
                     const int h = h0 + e;
                     if (h < G) {
                         const float inv = Lt[e] > 0.0f ? p.v.s_t / Lt[e] : 0.0f;
-                        float* orow = fa.out + (row * p.Hq + (int64_t)cur.kvh * G + h) * kAttD;
+                        const int64_t orow = (row * p.Hq + (int64_t)cur.kvh * G + h) * kAttD;
 #pragma unroll
                         for (int k = 0; k < 8; ++k) {
                             const int pi = (lane >> 2) + 8 * k;
-                            const float2 v = e == 0 ? make_float2(o4[k].x * inv, o4[k].y * inv)
-                                                    : make_float2(o4[k].z * inv, o4[k].w * inv);
-                            *reinterpret_cast<float2*>(orow + 2 * pi) = v;
+                            if (e == 0) store_out2(p, fa.out, orow + 2 * pi, o4[k].x * inv, o4[k].y * inv);
+                            else store_out2(p, fa.out, orow + 2 * pi, o4[k].z * inv, o4[k].w * inv);
                         }
                         if (fa.lse != nullptr && lane < 4)
                             fa.lse[row * p.Hq + (int64_t)cur.kvh * G + h] =

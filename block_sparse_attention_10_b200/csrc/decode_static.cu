@@ -46,7 +46,7 @@ int static_scratch_address(void** out) {
 }  // namespace
 }  // namespace msa
 
-extern "C" int msa_decode_static(const msa_params_t* p, float* out, float* lse, int32_t* sel_out,
+extern "C" int msa_decode_static(const msa_params_t* p, void* out, float* lse, int32_t* sel_out,
                                  cudaStream_t stream) {
     // Argument checks of msa_decode: with no workspace it validates everything else
     // and returns MSA_EWORKSPACE without enqueueing any work.

@@ -41,7 +41,7 @@ constexpr size_t idx_smem_bytes(int B) {
     return (size_t)kIdxWarps * kIdxRing * (kIdxStageBytes + sizeof(uint64_t)) + (size_t)(2 * B + 2) * sizeof(int);
 }
 
-template <int DI, int HI, int NT>
+template <int DI, int HI, int NT, bool PAGED>
 __global__ void __launch_bounds__(kIdxThreads, 2)
     index_decode_kernel(const Problem p, float* __restrict__ block_scores, float* __restrict__ token_scores) {
     constexpr int R = kIdxRing;
@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
                 if (lane == 0) {
                     const int rows = (min(valid, KPS) + 15) & ~15;
                     const int s = (int)(slot_issued % R);
-                    const int64_t row0 = block_vec(p, ib, n, 0, 1) + is * KPS;
+                    const int64_t row0 = block_vec<PAGED>(p, ib, n, 0, 1) + is * KPS;
                     uint8_t* st = my_stages + s * kIdxStageBytes;
                     const uint32_t db = (uint32_t)(rows * (DI / 2)), sb = (uint32_t)(rows * (DI / 16));
                     mbar_arrive_expect_tx(&my_bars[s], db + sb);
@@ -164,9 +164,9 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
         }
 }
 
-template <int DI, int HI, int NT>
+template <int DI, int HI, int NT, bool PAGED>
 int launch_t(const Problem& p, float* bs, float* ts, bool pdl, cudaStream_t st) {
-    auto kern = index_decode_kernel<DI, HI, NT>;
+    auto kern = index_decode_kernel<DI, HI, NT, PAGED>;
     const size_t smem = idx_smem_bytes(p.B);
     static int configured_dev = -1;
     const DeviceInfo& di = device_info();
@@ -193,10 +193,11 @@ int launch_t(const Problem& p, float* bs, float* ts, bool pdl, cudaStream_t st) 
 template <int DI, int HI>
 int launch_nt(const Problem& p, float* bs, float* ts, bool pdl, cudaStream_t st) {
     const int nq = p.Tq * HI;
-    if (nq <= 8) return launch_t<DI, HI, 1>(p, bs, ts, pdl, st);
-    if (nq <= 16) return launch_t<DI, HI, 2>(p, bs, ts, pdl, st);
-    if (nq <= 24) return launch_t<DI, HI, 3>(p, bs, ts, pdl, st);
-    return launch_t<DI, HI, 4>(p, bs, ts, pdl, st);
+    const bool paged = p.block_table != nullptr;
+    if (nq <= 8) return paged ? launch_t<DI, HI, 1, true>(p, bs, ts, pdl, st) : launch_t<DI, HI, 1, false>(p, bs, ts, pdl, st);
+    if (nq <= 16) return paged ? launch_t<DI, HI, 2, true>(p, bs, ts, pdl, st) : launch_t<DI, HI, 2, false>(p, bs, ts, pdl, st);
+    if (nq <= 24) return paged ? launch_t<DI, HI, 3, true>(p, bs, ts, pdl, st) : launch_t<DI, HI, 3, false>(p, bs, ts, pdl, st);
+    return paged ? launch_t<DI, HI, 4, true>(p, bs, ts, pdl, st) : launch_t<DI, HI, 4, false>(p, bs, ts, pdl, st);
 }
 
 template <int DI>

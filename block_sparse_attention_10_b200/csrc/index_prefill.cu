@@ -80,7 +80,7 @@ __device__ __forceinline__ bool pf_tile_live(int qt, int64_t k0, int64_t L, int 
     return k0 < L && k0 <= L - Tq + tb - 1;
 }
 
-template <int DI, int HI>
+template <int DI, int HI, bool PAGED>
 __global__ void __launch_bounds__(kPfThreads, 1)
     index_prefill_kernel(const Problem p, float* __restrict__ block_scores, const __grid_constant__ CUtensorMap tmap) {
     using G = PfGeom<DI>;
@@ -239,7 +239,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     const int64_t key = k0 + j;
                     uint32_t w = 0u, sc = 0u;
                     if (key < L) {
-                        const int64_t vec = block_vec(p, b, key / kBlock, 0, 1) + key % kBlock;
+                        const int64_t vec = block_vec<PAGED>(p, b, key / kBlock, 0, 1) + key % kBlock;
                         w = *reinterpret_cast<const uint32_t*>(p.ik.data + vec * (DI / 2) + cr * 4);
                         sc = p.ik.scale[vec * (DI / 16) + (cr >> 1)];
                     }
@@ -334,7 +334,7 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-template <int DI, int HI>
+template <int DI, int HI, bool PAGED>
 int launch_pf(const Problem& p, float* bs, bool pdl, cudaStream_t st) {
     using G = PfGeom<DI>;
     auto enc = tensor_map_encoder();
@@ -349,7 +349,7 @@ int launch_pf(const Problem& p, float* bs, bool pdl, cudaStream_t st) {
             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         return MSA_ECUDA;
-    auto kern = index_prefill_kernel<DI, HI>;
+    auto kern = index_prefill_kernel<DI, HI, PAGED>;
     static int configured_dev = -1;
     const DeviceInfo& di = device_info();
     if (configured_dev != di.device) {
@@ -374,10 +374,10 @@ int launch_pf(const Problem& p, float* bs, bool pdl, cudaStream_t st) {
 template <int DI>
 int launch_pf_hi(const Problem& p, float* bs, bool pdl, cudaStream_t st) {
     switch (p.HI) {
-        case 1: return launch_pf<DI, 1>(p, bs, pdl, st);
-        case 2: return launch_pf<DI, 2>(p, bs, pdl, st);
-        case 4: return launch_pf<DI, 4>(p, bs, pdl, st);
-        case 8: return launch_pf<DI, 8>(p, bs, pdl, st);
+        case 1: return p.block_table ? launch_pf<DI, 1, true>(p, bs, pdl, st) : launch_pf<DI, 1, false>(p, bs, pdl, st);
+        case 2: return p.block_table ? launch_pf<DI, 2, true>(p, bs, pdl, st) : launch_pf<DI, 2, false>(p, bs, pdl, st);
+        case 4: return p.block_table ? launch_pf<DI, 4, true>(p, bs, pdl, st) : launch_pf<DI, 4, false>(p, bs, pdl, st);
+        case 8: return p.block_table ? launch_pf<DI, 8, true>(p, bs, pdl, st) : launch_pf<DI, 8, false>(p, bs, pdl, st);
         default: return MSA_EUNSUPPORTED;
     }
 }

@@ -41,20 +41,38 @@ struct Problem {
     uint32_t* status;
     const int32_t* block_table;  // [B][nbmax] page of each block, or nullptr (contiguous caches)
     int64_t num_pages;
+    int out_bf16;                // attention output as bf16 (else fp32)
 };
 
 // First cache vector of block n of sequence b, head h of H: contiguous caches hold
 // [B][H][lmax][...]; paged caches hold pages [num_pages][H][128][...] found through the
 // block table.  A page id outside the pool is flagged and replaced by page 0, so every
-// copy stays inside the pool.
+// copy stays inside the pool.  PAGED is a compile-time choice in the indexers' stream
+// loops (the contiguous path then carries no table lookup); block_vec_any decides at run
+// time where it is called once per warp.
+template <bool PAGED>
 __device__ __forceinline__ int64_t block_vec(const Problem& p, int b, int64_t n, int h, int H) {
-    if (p.block_table == nullptr) return ((int64_t)b * H + h) * p.lmax + n * kBlock;
-    int64_t page = __ldg(p.block_table + (int64_t)b * p.nbmax + n);
-    if (page < 0 || page >= p.num_pages) {
-        set_status(p.status, MSA_STATUS_PAGE);
-        page = 0;
+    if constexpr (!PAGED) {
+        return ((int64_t)b * H + h) * p.lmax + n * kBlock;
+    } else {
+        int64_t page = __ldg(p.block_table + (int64_t)b * p.nbmax + n);
+        if (page < 0 || page >= p.num_pages) {
+            set_status(p.status, MSA_STATUS_PAGE);
+            page = 0;
+        }
+        return (page * H + h) * kBlock;
     }
-    return (page * H + h) * kBlock;
+}
+__device__ __forceinline__ int64_t block_vec_any(const Problem& p, int b, int64_t n, int h, int H) {
+    return p.block_table != nullptr ? block_vec<true>(p, b, n, h, H) : block_vec<false>(p, b, n, h, H);
+}
+
+// Stores two adjacent output elements (index i, i + 1) as fp32 or, with out_bf16, bf16 (RNE).
+__device__ __forceinline__ void store_out2(const Problem& p, float* out, int64_t i, float a, float b) {
+    if (p.out_bf16)
+        *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(out) + i) = __floats2bfloat162_rn(a, b);
+    else
+        *reinterpret_cast<float2*>(out + i) = make_float2(a, b);
 }
 
 int launch_nvfp4_encode(const float* x, int64_t nvec, int dim, float s_t, uint8_t* data, uint8_t* scale,

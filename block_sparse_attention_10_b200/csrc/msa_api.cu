@@ -52,6 +52,7 @@ int check_params(const msa_params_t* p, bool need_index, bool need_attend) {
     if (p->Tq > p->lmax) return MSA_EINVAL;
     if (p->pool_mode != 0 && p->pool_mode != 1) return MSA_EINVAL;
     if (p->block_table != nullptr && p->num_pages <= 0) return MSA_EINVAL;
+    if (p->out_bf16 != 0 && p->out_bf16 != 1) return MSA_EINVAL;
     if (need_index) {
         if (p->HI <= 0 || p->DI <= 0 || !p->q_idx) return MSA_EINVAL;
         if (int r = check_cache(p->ik)) return r;
@@ -97,6 +98,7 @@ Problem to_problem(const msa_params_t* p) {
     q.status = p->status;
     q.block_table = p->block_table;
     q.num_pages = p->block_table != nullptr ? p->num_pages : 0;
+    q.out_bf16 = p->out_bf16;
     return q;
 }
 
@@ -197,15 +199,17 @@ int msa_select(const msa_params_t* p, const float* block_scores, int32_t* sel, c
     return launch_select(to_problem(p), block_scores, sel, nullptr, false, stream);
 }
 
-int msa_attend(const msa_params_t* p, const int32_t* sel, float* out, float* lse, cudaStream_t stream) {
+int msa_attend(const msa_params_t* p, const int32_t* sel, void* out_, float* lse, cudaStream_t stream) {
+    float* out = static_cast<float*>(out_);  // bf16 elements when out_bf16
     if (int r = check_params(p, false, true)) return r;
     if (!sel || !out) return MSA_EINVAL;
     if (!aligned16(out)) return MSA_EALIGN;
     return launch_attend(to_problem(p), sel, out, lse, false, stream);
 }
 
-int msa_decode(const msa_params_t* p, void* ws, size_t ws_bytes, float* out, float* lse, int32_t* sel_out,
+int msa_decode(const msa_params_t* p, void* ws, size_t ws_bytes, void* out_, float* lse, int32_t* sel_out,
                cudaStream_t stream) {
+    float* out = static_cast<float*>(out_);  // bf16 elements when out_bf16
     if (int r = check_params(p, true, true)) return r;
     if (!out) return MSA_EINVAL;
     if (!aligned16(out)) return MSA_EALIGN;
@@ -222,8 +226,9 @@ int msa_decode(const msa_params_t* p, void* ws, size_t ws_bytes, float* out, flo
     return launch_attend(q, sel, out, lse, pdl, stream);
 }
 
-int msa_decode_single_launch(const msa_params_t* p, void* ws, size_t ws_bytes, float* out, float* lse,
+int msa_decode_single_launch(const msa_params_t* p, void* ws, size_t ws_bytes, void* out_, float* lse,
                              int32_t* sel_out, cudaStream_t stream) {
+    float* out = static_cast<float*>(out_);  // bf16 elements when out_bf16
     if (int r = check_params(p, true, true)) return r;
     if (!out) return MSA_EINVAL;
     if (!aligned16(out)) return MSA_EALIGN;

@@ -48,7 +48,7 @@ class _Params(ctypes.Structure):
                 ("seq_lens", ctypes.c_void_p), ("k", _Cache), ("v", _Cache), ("ik", _Cache),
                 ("q", ctypes.c_void_p), ("q_idx", ctypes.c_void_p), ("w_idx", ctypes.c_void_p),
                 ("softmax_scale", ctypes.c_float), ("pool_mode", ctypes.c_int), ("status", ctypes.c_void_p),
-                ("block_table", ctypes.c_void_p), ("num_pages", ctypes.c_int64)]
+                ("block_table", ctypes.c_void_p), ("num_pages", ctypes.c_int64), ("out_bf16", ctypes.c_int)]
 
 
 _lib = None
@@ -142,6 +142,7 @@ class MsaProblem:
     # paged caches: int32 [B, lmax / 128] page of each block; k, v, ik are then page pools
     # [num_pages, H, 128, dim/2] (+ scales)
     block_table: Optional[torch.Tensor] = None
+    out_bf16: bool = False  # attention output as bf16 instead of fp32
 
     def __setattr__(self, name, value):
         # any change of a field invalidates the cached parameter block
@@ -167,7 +168,8 @@ class MsaProblem:
                        self.k._c(), self.v._c(), self.ik._c(), self.q.data_ptr(), self.q_idx.data_ptr(),
                        None if self.w_idx is None else self.w_idx.data_ptr(), self.softmax_scale, self.pool_mode,
                        None if self.status is None else self.status.data_ptr(),
-                       self.block_table.data_ptr() if paged else None, self.ik.data.shape[0] if paged else 0)
+                       self.block_table.data_ptr() if paged else None, self.ik.data.shape[0] if paged else 0,
+                       1 if self.out_bf16 else 0)
 
     @property
     def nbmax(self) -> int:
@@ -275,8 +277,9 @@ def alloc_workspace(p: MsaProblem) -> torch.Tensor:
 
 
 def outputs(p: MsaProblem):
+    """(out [B, Tq, Hq, D] fp32 or bf16 per p.out_bf16, lse fp32 [B, Tq, Hq], sel int32 [B, Tq, 16])."""
     B, Tq, Hq, D = p.q.shape
     dev = p.q.device
-    return (torch.empty(B, Tq, Hq, D, dtype=torch.float32, device=dev),
+    return (torch.empty(B, Tq, Hq, D, dtype=torch.bfloat16 if p.out_bf16 else torch.float32, device=dev),
             torch.empty(B, Tq, Hq, dtype=torch.float32, device=dev),
             torch.empty(B, Tq, MSA_TOPK_BLOCKS, dtype=torch.int32, device=dev))

@@ -116,6 +116,8 @@ typedef struct msa_nvfp4_cache {
  *             A page id outside [0, num_pages) sets MSA_STATUS_PAGE and page 0
  *             is read in its place (results invalid)
  *   num_pages pages in each pool (> 0 with a block table)
+ *   out_bf16  0: attention output fp32; 1: bf16 (the fp32 result rounded to
+ *             nearest even, for the next layer); lse stays fp32
  */
 typedef struct msa_params {
     int B, Tq, Hq, Hkv, D, HI, DI;
@@ -130,6 +132,7 @@ typedef struct msa_params {
     uint32_t* status;
     const int32_t* block_table;
     int64_t num_pages;
+    int out_bf16;
 } msa_params_t;
 
 /* Human-readable name of an msa_status code (static string, never NULL). */
@@ -184,9 +187,9 @@ int msa_select(const msa_params_t* p, const float* block_scores, int32_t* sel,
 /* Exact softmax attention over the selected blocks (split over the blocks,
  * combined in on-chip memory):
  *   sel  int32 [B][Tq][16] (ids < 0 are skipped)
- *   out  fp32 [B][Tq][Hq][D]; lse fp32 [B][Tq][Hq] (natural log of the
+ *   out  [B][Tq][Hq][D], fp32 (bf16 with out_bf16); lse fp32 [B][Tq][Hq] (natural log of the
  *        softmax denominator of the scaled scores) or NULL */
-int msa_attend(const msa_params_t* p, const int32_t* sel, float* out, float* lse,
+int msa_attend(const msa_params_t* p, const int32_t* sel, void* out, float* lse,
                cudaStream_t stream);
 
 /* The whole MSA decode step: msa_index -> msa_select -> msa_attend (two
@@ -196,7 +199,7 @@ int msa_attend(const msa_params_t* p, const int32_t* sel, float* out, float* lse
  *                 256-byte aligned; contents on entry are ignored
  *   out, lse      as for msa_attend
  *   sel_out       int32 [B][Tq][16] copy of the selection, or NULL */
-int msa_decode(const msa_params_t* p, void* ws, size_t ws_bytes, float* out, float* lse,
+int msa_decode(const msa_params_t* p, void* ws, size_t ws_bytes, void* out, float* lse,
                int32_t* sel_out, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
@@ -227,7 +230,7 @@ size_t msa_workspace_size_single_launch(const msa_params_t* p);
  * another warp's result that exceeds 2 s (all CTAs of the grid must be
  * resident: another kernel holding SMs for that long) sets MSA_STATUS_TIMEOUT
  * | MSA_STATUS_AT_DECODE_WAIT and ends the launch. */
-int msa_decode_single_launch(const msa_params_t* p, void* ws, size_t ws_bytes, float* out,
+int msa_decode_single_launch(const msa_params_t* p, void* ws, size_t ws_bytes, void* out,
                              float* lse, int32_t* sel_out, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
@@ -256,7 +259,7 @@ int msa_decode_single_launch(const msa_params_t* p, void* ws, size_t ws_bytes, f
  *   - all calls share the one array, which keeps the last call's contents:
  *     calls that overlap on the GPU (other streams, other host threads) race
  *     and must be serialised by the caller. */
-int msa_decode_static(const msa_params_t* p, float* out, float* lse, int32_t* sel_out,
+int msa_decode_static(const msa_params_t* p, void* out, float* lse, int32_t* sel_out,
                       cudaStream_t stream);
 
 #ifdef __cplusplus

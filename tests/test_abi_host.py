@@ -81,10 +81,18 @@ def test_block_table_arguments(L):
 
 
 def test_params_struct_layout(L):
-    # the Python mirror of msa_params_t ends with the block table and the page count
+    # the Python mirror of msa_params_t ends with the block table, the page count and the
+    # output type (int, padded to the struct's 8-byte alignment)
     names = [f[0] for f in msa._Params._fields_]
-    assert names[-3:] == ["status", "block_table", "num_pages"]
-    assert ctypes.sizeof(msa._Params) == msa._Params.num_pages.offset + 8
+    assert names[-4:] == ["status", "block_table", "num_pages", "out_bf16"]
+    assert msa._Params.out_bf16.offset == msa._Params.num_pages.offset + 8
+    assert ctypes.sizeof(msa._Params) == msa._Params.out_bf16.offset + 8
+
+
+def test_out_type_argument(L):
+    p = _params(out_bf16=2)
+    r = L.msa_decode(ctypes.byref(p), ctypes.c_void_p(0x10000), 1 << 20, ctypes.c_void_p(0x20000), None, None, None)
+    assert r == 1
 
 
 def test_single_launch_rejects_before_enqueueing(L):

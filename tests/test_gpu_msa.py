@@ -10,7 +10,7 @@ import pytest
 import torch
 
 import oracle
-from block_sparse_attention_10_b200 import configs, synth
+from block_sparse_attention_10_b200 import configs, msa, synth
 from tests._common import (bf16_values, check_attention, check_selection, oracle_caches)
 from tests._gpu import problem_from_inputs, run_decode, run_steps, status_of
 
@@ -99,3 +99,31 @@ def test_tiny_needles_found():
     p = problem_from_inputs(inp)
     d = run_decode(p)
     assert set(inp.needles[0]) <= set(d["sel"][0, 0].tolist())
+
+
+def test_bf16_output_is_the_rounded_fp32_output(case):
+    name, inp, _ = case
+    p = problem_from_inputs(inp)
+    ws = msa.alloc_workspace(p)
+    out32, lse32, sel32 = msa.outputs(p)
+    msa.msa_decode(p, ws, out32, lse32, sel32)
+    p.out_bf16 = True
+    out16, lse16, sel16 = msa.outputs(p)
+    assert out16.dtype == torch.bfloat16
+    msa.msa_decode(p, ws, out16, lse16, sel16)
+    a16 = torch.empty_like(out16)
+    msa.msa_attend(p, sel16, a16, None)
+    torch.cuda.synchronize()
+    assert status_of(p) == 0
+    assert torch.equal(sel16, sel32) and torch.equal(lse16, lse32)
+    assert torch.equal(out16.view(torch.int16), out32.to(torch.bfloat16).view(torch.int16))
+    assert torch.equal(a16.view(torch.int16), out16.view(torch.int16))
+    if msa.msa_workspace_size_single_launch(p) > 0:
+        o1, _, _ = msa.outputs(p)
+        msa.msa_decode_single_launch(p, msa.alloc_workspace_single_launch(p), o1)
+        torch.cuda.synchronize()
+        p.out_bf16 = False
+        o2, _, _ = msa.outputs(p)
+        msa.msa_decode_single_launch(p, msa.alloc_workspace_single_launch(p), o2)
+        torch.cuda.synchronize()
+        assert torch.equal(o1.view(torch.int16), o2.to(torch.bfloat16).view(torch.int16))
