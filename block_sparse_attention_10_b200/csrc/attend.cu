@@ -22,7 +22,7 @@
 // The partial (m, l, O) of the 4 warps are merged in shared memory, then the
 // CTAs of the cluster merge through distributed shared memory (each CTA
 // finalises 128 / CL of the 128 dims).  With the selection fused in (rows of
-// <= 1,024 blocks), warp 0 of every CTA first selects the row's blocks.  No global scratch,
+// <= 1,024 blocks), every CTA first selects the row's blocks.  No global scratch,
 // no second launch, a fixed merge order (bitwise deterministic).
 #include <cooperative_groups.h>
 
@@ -44,8 +44,9 @@ constexpr int64_t kFusedSelectMaxBlocks = 1024;  // rows one warp selects from r
 constexpr int kWarpSmem = 2 * kAttStageBytes;  // 9 KB: also holds the warp's partial O (4 KB) at the end
 constexpr size_t kAttSmem = (size_t)kAttWarps * kWarpSmem + 2 * kAttWarps * sizeof(uint64_t) + 2 * 8 * sizeof(float);
 
-// FUSED: the CTA first selects its row's blocks from the pooled scores (warp 0, rows of
-// <= 1,024 blocks) instead of reading a selection written by select.cu.
+// FUSED: the CTA first selects its row's blocks from the pooled scores (rows of <= 1,024
+// blocks: warp 0 alone up to 128, else all 4 warps in two levels) instead of reading a
+// selection written by select.cu.
 template <int G, bool FUSED, int CL>
 __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(kAttThreads, 4)
     attend_kernel(const Problem p, const int32_t* __restrict__ sel, const float* __restrict__ block_scores,
@@ -94,10 +95,13 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(kAttThreads, 4)
     if constexpr (FUSED) {
         const float* srow = block_scores + bt * p.nbmax;
         const int64_t r = nvis - 1;
-        if (warp == 0) {  // as few candidate registers per lane as the row needs
-            if (nvis <= 128) select_row_warp<4>(srow, nvis, r, lane, sh_sel);
-            else if (nvis <= 512) select_row_warp<16>(srow, nvis, r, lane, sh_sel);
-            else select_row_warp<32>(srow, nvis, r, lane, sh_sel);
+        if (nvis <= 128) {
+            if (warp == 0) select_row_warp<4>(srow, nvis, r, lane, sh_sel);
+        } else {  // the CTA's 4 warps: 128 or 256 blocks each, then warp 0 over the 60 candidates
+            __shared__ uint32_t ckey[kAttWarps * (kTopK - 1)];
+            __shared__ int32_t cid[kAttWarps * (kTopK - 1)];
+            if (nvis <= 512) select_row_cta<kAttWarps, 4>(srow, nvis, r, warp, lane, ckey, cid, sh_sel);
+            else select_row_cta<kAttWarps, 8>(srow, nvis, r, warp, lane, ckey, cid, sh_sel);
         }
         __syncthreads();
         if (warp == 0 && lane < kTopK && sel_out != nullptr && crank == 0 && kvh == 0)
