@@ -99,3 +99,36 @@ def test_unsupported_shape_is_refused():
     with pytest.raises(msa.MsaError) as e:
         msa.msa_decode_single_launch(p, torch.empty(1 << 20, dtype=torch.uint8, device="cuda"), out)
     assert e.value.code == 2
+
+
+def test_maximum_batch():
+    # B = 4096 (the library's limit): 4,096 ragged short sequences; per-CTA prefix arrays of
+    # 2 x 4,097 ints (one CTA per SM for the indexers), a 16,384-CTA attention grid.  The
+    # inputs are generated on the GPU (the same bits as on the host) and copied back for
+    # the oracle.
+    B = 4096
+    rng = np.random.default_rng(4096)
+    lens = [int(x) for x in rng.integers(1, 641, B)]
+    w = synth.Workload("maxb", B=B, Tq=1, Hq=8, Hkv=1, D=128, HI=4, DI=64, seq_len=max(lens), lmax=640,
+                       needles=0, seed=41)
+    inp = synth.make_inputs(w, device="cuda")
+    inp.seq_lens = lens
+    for name in ("k", "v", "ik"):  # zero past each sequence's own length, then to the host
+        t = getattr(inp, name)
+        mask = torch.arange(640, device="cuda")[None, :] < torch.tensor(lens, device="cuda")[:, None]
+        t.mul_(mask[:, None, :, None])
+        setattr(inp, name, t.cpu())
+    inp.q, inp.q_idx = inp.q.cpu(), inp.q_idx.cpu()
+    p = problem_from_inputs(inp)
+    d = run_decode(p)
+    assert status_of(p) == 0
+    k, v, ik = oracle_caches(inp)
+    bs, _ = oracle.index(bf16_values(inp.q_idx), ik, inp.seq_lens)
+    check_selection(d["sel"], oracle.select(bs, inp.seq_lens), bs, inp.seq_lens, 1)
+    o, l = oracle.attend(bf16_values(inp.q), k, v, d["sel"], inp.seq_lens)
+    check_attention(d["out"], o)
+    np.testing.assert_allclose(d["lse"], l, rtol=1e-4, atol=1e-4)
+    s = run_decode(p, single_launch=True)
+    assert status_of(p) == 0
+    assert np.array_equal(s["sel"], d["sel"])
+    check_attention(s["out"], o)
