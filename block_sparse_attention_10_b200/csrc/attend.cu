@@ -1,10 +1,10 @@
 // attend.cu — exact softmax attention over the selected NVFP4 blocks (decode).
 //
-// "Main attention then runs exactly, but only over the top 16 blocks ... That
-// caps each query at 2,048 keys" ("vLLM Adds Day-0 Support for
-// MiniMax-M3.1-Flash", ainewsbites.com, "A model built for efficient
-// inference").  Query head h reads KV head h / (Hq/Hkv); keys j > pos are
-// masked; K and V are NVFP4 and dequantised in registers.
+// Method ("vLLM Adds Day-0 Support for MiniMax-M3.1-Flash", ainewsbites.com,
+// section "A model built for efficient inference"): softmax attention is computed
+// exactly, but only over the 16 selected blocks of 128 tokens, so no query reads
+// more than 2,048 keys.  Query head h reads KV head h / (Hq/Hkv); keys j > pos
+// are masked; K and V are NVFP4 and dequantised in registers.
 //
 // Design (B200): one thread-block cluster of 4 CTAs x 4 warps per
 // (sequence, query token, KV head): each of the 16 warps takes one selected

@@ -1,8 +1,8 @@
 // attend_quarter.cuh — one warp's exact-attention step over 32 keys of one KV head.
 //
-// "Main attention then runs exactly, but only over the top 16 blocks"
-// ("vLLM Adds Day-0 Support for MiniMax-M3.1-Flash", ainewsbites.com, "A model built for
-// efficient inference").  A warp computes the G query heads of one KV head against the
+// Method ("vLLM Adds Day-0 Support for MiniMax-M3.1-Flash", ainewsbites.com, section "A
+// model built for efficient inference"): attention over the selected blocks is exact
+// softmax attention, not an approximation.  A warp computes the G query heads of one KV head against the
 // keys of a 32-key quarter of a selected block and folds them into its running
 // (max, sum, output) with the online softmax:
 //   S^T = K Q^T    mma m16n8k16, A = dequantised K (exact f16, 16 keys), B = the G

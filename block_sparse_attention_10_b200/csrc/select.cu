@@ -1,9 +1,9 @@
 // select.cu — top-16 block selection with the most recent block forced.
 //
-// "Main attention then runs exactly, but only over the top 16 blocks, and the
-// most recent block is always kept" ("vLLM Adds Day-0 Support for
-// MiniMax-M3.1-Flash", ainewsbites.com, "A model built for efficient
-// inference").  Reading: the query's own block r = pos div 128 plus the best
+// Method ("vLLM Adds Day-0 Support for MiniMax-M3.1-Flash", ainewsbites.com,
+// section "A model built for efficient inference"): 16 blocks per query are
+// attended, and the block that holds the query is always among them.
+// Reading: the query's own block r = pos div 128 plus the best
 // min(15, r) other blocks under the total order (score desc, index asc); the
 // list is written ascending and padded with -1.
 //

@@ -1,10 +1,10 @@
 // select_row.cuh — top-16 block selection of one (sequence, query token) row by one warp.
 //
-// "Main attention then runs exactly, but only over the top 16 blocks, and the most recent
-// block is always kept" ("vLLM Adds Day-0 Support for MiniMax-M3.1-Flash",
-// ainewsbites.com, "A model built for efficient inference").  Reading: the query's own
-// block r plus the best min(15, r) other blocks under the total order (score desc,
-// index asc), written ascending and padded with -1.  r = nvis - 1 is the last visible
+// Method ("vLLM Adds Day-0 Support for MiniMax-M3.1-Flash", ainewsbites.com, section
+// "A model built for efficient inference"): exact attention is restricted to 16 blocks
+// per query, and the block holding the query itself is never dropped.  Reading: the
+// query's own block r plus the best min(15, r) other blocks under the total order
+// (score desc, index asc), written ascending and padded with -1.  r = nvis - 1 is the last visible
 // block, so it always comes last in the ascending list.
 //
 // Threshold selection (select_row_warp): every candidate becomes a 32-bit key whose

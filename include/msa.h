@@ -245,8 +245,8 @@ int msa_decode_single_launch(const msa_params_t* p, void* ws, size_t ws_bytes, v
  * array of MSA_STATIC_SCRATCH_BYTES owned by the library, for callers that
  * cannot call cudaMalloc: a plugin handed only its inputs and outputs by a host
  * framework that owns all device memory, or a hot loop that must not risk the
- * device-wide synchronisation an allocation can cause.  Allocates and frees
- * nothing, on the device or the host.
+ * device-wide synchronisation an allocation can cause.  Calls no allocation
+ * routine, on the device or the host (but see the first-call note below).
  *   p, out, lse, sel_out, stream   as for msa_decode
  * Returns the msa_decode argument errors, or MSA_EWORKSPACE when
  * msa_workspace_size(p) exceeds MSA_STATIC_SCRATCH_BYTES (e.g. B * Tq *
@@ -255,7 +255,13 @@ int msa_decode_single_launch(const msa_params_t* p, void* ws, size_t ws_bytes, v
  * Notes:
  *   - every GPU that loads libmsa.so holds the array until the process exits;
  *   - the first call on each device looks up the array's address (once, with
- *     that device current); make that first call before any stream capture;
+ *     that device current).  With lazy module loading (the CUDA default) the
+ *     driver only loads the library's module, and so places the array in
+ *     device memory, at that lookup: the first call may therefore allocate on
+ *     the driver's side and synchronise.  Treat it as the warm-up call, and
+ *     make it before any stream capture and outside latency-critical code;
+ *   - after cudaDeviceReset the next call looks the address up again (the
+ *     device then has a new context and the array a new address);
  *   - all calls share the one array, which keeps the last call's contents:
  *     calls that overlap on the GPU (other streams, other host threads) race
  *     and must be serialised by the caller. */

@@ -40,7 +40,7 @@ def run_decode(p, single_launch=False, ws=None):
     out, lse, sel = msa.outputs(p)
     (msa.msa_decode_single_launch if single_launch else msa.msa_decode)(p, ws, out, lse, sel)
     torch.cuda.synchronize()
-    return dict(sel=sel.cpu().numpy(), out=out.cpu().numpy(), lse=lse.cpu().numpy())
+    return dict(sel=sel.cpu().numpy(), out=out.float().cpu().numpy(), lse=lse.cpu().numpy())
 
 
 def status_of(p):

@@ -70,9 +70,9 @@ def _check_sequence(w, p, meta, b, sel_gpu, out_gpu):
 
 
 @pytest.mark.parametrize("w,samples", [
-    (configs.DECODE_B32_64K, [0, 17, 31]),
-    (configs.LONG_RAGGED_256K, [0, 5, 7]),
-    (configs.SPEC_VERIFY_512K, [1, 3]),
+    (configs.DECODE_B32_64K, [0, 5, 9, 14, 17, 22, 27, 31]),
+    (configs.LONG_RAGGED_256K, list(range(8))),
+    (configs.SPEC_VERIFY_512K, list(range(4))),
 ])
 def test_full_size_decode_sampled(w, samples):
     p, meta = _gpu_problem(w)

@@ -11,7 +11,7 @@ import torch
 
 import oracle
 from block_sparse_attention_10_b200 import configs, msa, synth
-from tests._common import (bf16_values, check_attention, check_selection, oracle_caches)
+from tests._common import (bf16_values, check_attention, check_attention_bf16, check_selection, oracle_caches)
 from tests._gpu import problem_from_inputs, run_decode, run_steps, status_of
 
 pytestmark = pytest.mark.gpu
@@ -127,3 +127,14 @@ def test_bf16_output_is_the_rounded_fp32_output(case):
         msa.msa_decode_single_launch(p, msa.alloc_workspace_single_launch(p), o2)
         torch.cuda.synchronize()
         assert torch.equal(o1.view(torch.int16), o2.to(torch.bfloat16).view(torch.int16))
+
+
+def test_bf16_output_matches_oracle(case):
+    """bf16 attention output of msa_decode against the oracle rounded to bf16."""
+    name, inp, (k, v, ik) = case
+    p = problem_from_inputs(inp)
+    p.out_bf16 = True
+    d = run_decode(p)
+    assert status_of(p) == 0
+    out, _ = oracle.attend(bf16_values(inp.q), k, v, d["sel"], inp.seq_lens)
+    check_attention_bf16(d["out"], out)

@@ -3,12 +3,16 @@ against the same problem with contiguous caches: identical arithmetic, so every 
 bitwise equal — pooled scores, token scores, selection, attention, lse — for decode (warp
 and CTA selection, clusters of 4/8/16), multi-token causal rows and chunked prefill (the
 tensor-core indexer).  Unused pages hold garbage, so a read of a wrong page would show.
-A page id outside the pool sets MSA_STATUS_PAGE and reads page 0 instead (no fault)."""
+A page id outside the pool sets MSA_STATUS_PAGE and reads page 0 instead (no fault).
+The paged path is also checked against the oracle directly (selection, fp32 and bf16
+attention output), so a block-table error shared by both layouts would still show."""
 import numpy as np
 import pytest
 import torch
 
+import oracle
 from block_sparse_attention_10_b200 import msa, synth
+from tests._common import bf16_values, check_attention, check_attention_bf16, check_selection, oracle_caches
 from tests._gpu import paged_problem, problem_from_inputs, run_decode, run_steps, status_of
 
 pytestmark = pytest.mark.gpu
@@ -49,6 +53,26 @@ def test_paged_equals_contiguous(name):
     assert status_of(p) == 0 and status_of(pp) == 0
     for key in ("sel", "out", "lse"):
         assert np.array_equal(d[key].view(np.uint32), e[key].view(np.uint32)), key
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_paged_matches_oracle(name):
+    inp = CASES[name]()
+    k, v, ik = oracle_caches(inp)
+    pp = paged_problem(problem_from_inputs(inp), seed=len(name) + 3)
+    d = run_decode(pp)
+    assert status_of(pp) == 0
+    Tq = inp.w.Tq
+    bs, _ = oracle.index(bf16_values(inp.q_idx), ik, inp.seq_lens)
+    check_selection(d["sel"], oracle.select(bs, inp.seq_lens), bs, inp.seq_lens, Tq)
+    out, lse = oracle.attend(bf16_values(inp.q), k, v, d["sel"], inp.seq_lens)
+    check_attention(d["out"], out)
+    np.testing.assert_allclose(d["lse"], lse, rtol=1e-4, atol=1e-4)
+    pp.out_bf16 = True
+    d16 = run_decode(pp)
+    assert status_of(pp) == 0
+    assert np.array_equal(d16["sel"], d["sel"])
+    check_attention_bf16(d16["out"], out)
 
 
 def test_page_outside_pool_is_flagged():

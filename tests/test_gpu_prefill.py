@@ -3,9 +3,10 @@ msa_decode step against the oracle.
 
 Small cases span several 128-row query tiles, a partial last tile, ragged
 lengths, causal diagonals, HI 1..8, DI 64/128 and head weights; the full-size
-workload (2 sequences, 4,096-token chunk on a 128K context) is checked on
-sampled query tokens, each of which the oracle scores as a one-token step at its
-own position (causal truncation; pinned in test_oracle_msa).
+workload (2 sequences, 4,096-token chunk on a 128K context) is checked on 256
+sampled query tokens (chunk start and end, every block-boundary class, random),
+each of which the oracle scores as a one-token step at its own position (causal
+truncation; pinned in test_oracle_msa).
 """
 import numpy as np
 import pytest
@@ -13,7 +14,8 @@ import torch
 
 import oracle
 from block_sparse_attention_10_b200 import configs, msa, synth
-from tests._common import bf16_values, check_attention, check_selection, oracle_caches
+from tests._common import (bf16_values, check_attention, check_selection, oracle_attend_rows,
+                           oracle_caches, oracle_index_rows)
 from tests._gpu import problem_from_inputs, run_decode
 
 pytestmark = pytest.mark.gpu
@@ -88,7 +90,24 @@ def test_prefill_rejects_max_pooling_and_token_scores():
     assert e.value.code == 2
 
 
+def _sample_tokens(Tq, L, n, seed):
+    """n query tokens of the chunk: its first and last three, every token whose position is
+    the first, second or last of a 128-token block, then seeded random tokens."""
+    pos0 = L - Tq
+    toks = {0, 1, 2, Tq - 3, Tq - 2, Tq - 1}
+    toks |= {t for t in range(Tq) if (pos0 + t) % 128 in (0, 1, 127)}
+    rng = np.random.default_rng(seed)
+    while len(toks) < n:
+        toks.add(int(rng.integers(0, Tq)))
+    return sorted(toks)
+
+
 def test_prefill_full_size_sampled_tokens():
+    """The full-size chunked-prefill workload in bench.py's launch configuration (one
+    msa_decode over both sequences), checked on 128 sampled query tokens of each sequence
+    (256 rows): pooled-score selection and attention against the oracle, which regenerates
+    each sequence's caches on the CPU from the counter-based generator and encodes them with
+    its own encoder."""
     w = configs.PREFILL_4K_ON_128K
     inp = synth.make_inputs(w, device="cuda")
     p = msa.MsaProblem(seq_lens=torch.tensor(inp.seq_lens, dtype=torch.int32, device="cuda"),
@@ -103,35 +122,38 @@ def test_prefill_full_size_sampled_tokens():
     msa.msa_decode(p, ws, out, lse, sel)
     torch.cuda.synchronize()
     assert int(p.status.item()) == 0
-    sel_h, out_h = sel.cpu().numpy(), out.cpu().numpy()
+    sel_h, out_h, lse_h = sel.cpu().numpy(), out.cpu().numpy(), lse.cpu().numpy()
     assert np.isfinite(out_h).all()
     L = w.seq_len
-    tokens = [0, 1, 127, 128, 2047, 2048, 4000, 4095]
+    rows = 0
     for b in range(w.B):
-        qi = bf16_values(p.q_idx[b])                      # [Tq, HI, DI]
-        ik32 = torch.zeros(1, 1, w.lmax, w.DI)
-        ik32[0, :, :L] = synth.kv_tokens(w, synth.TID_IK, b, 1, w.DI, 0, L)
-        ik = oracle.nvfp4_encode(ik32.numpy(), s_ik)
-        assert np.array_equal(ik.data[0, 0], p.ik.data[b, 0].cpu().numpy())
-        n = len(tokens)
-        ikb = oracle.Nvfp4(np.repeat(ik.data, n, 0), np.repeat(ik.scale, n, 0), s_ik)
+        tokens = _sample_tokens(w.Tq, L, 128, seed=100 + b)
+        assert len(tokens) == 128
         pos = [L - w.Tq + t for t in tokens]
-        obs, _ = oracle.index(qi[tokens][:, None], ikb, [x + 1 for x in pos])
-        osel = oracle.select(obs, [x + 1 for x in pos])
-        check_selection(sel_h[b, tokens][:, None], osel, obs, [x + 1 for x in pos], 1)
-        # attention for the sampled tokens on the GPU's selection
-        blocks = sorted({int(x) for t in tokens for x in sel_h[b, t] if x >= 0})
-        kd = np.zeros((1, w.Hkv, w.lmax, w.D // 2), np.uint8)
-        ksc = np.zeros((1, w.Hkv, w.lmax, w.D // 16), np.uint8)
-        vd, vsc = kd.copy(), ksc.copy()
-        for nblk in blocks:
-            t0, t1 = nblk * 128, min(L, (nblk + 1) * 128)
-            kb = oracle.nvfp4_encode(synth.kv_tokens(w, synth.TID_K, b, w.Hkv, w.D, t0, t1).numpy(), s_k)
-            vb = oracle.nvfp4_encode(synth.kv_tokens(w, synth.TID_V, b, w.Hkv, w.D, t0, t1).numpy(), s_v)
-            kd[0, :, t0:t1], ksc[0, :, t0:t1] = kb.data, kb.scale
-            vd[0, :, t0:t1], vsc[0, :, t0:t1] = vb.data, vb.scale
-        K = oracle.Nvfp4(np.repeat(kd, n, 0), np.repeat(ksc, n, 0), s_k)
-        V = oracle.Nvfp4(np.repeat(vd, n, 0), np.repeat(vsc, n, 0), s_v)
-        q = bf16_values(p.q[b])[tokens][:, None]
-        o, _ = oracle.attend(q, K, V, sel_h[b, tokens][:, None], [x + 1 for x in pos])
-        check_attention(out_h[b, tokens][:, None], o)
+        q, qi, _ = synth.queries(w, [b])
+        assert torch.equal(q[0], p.q[b].cpu()) and torch.equal(qi[0], p.q_idx[b].cpu())
+        # the sequence's caches, generated and encoded on the CPU
+        ik32 = np.zeros((1, 1, w.lmax, w.DI), np.float32)
+        ik32[0, :, :L] = synth.kv_tokens(w, synth.TID_IK, b, 1, w.DI, 0, L).numpy()
+        ik = oracle.nvfp4_encode(ik32, s_ik)
+        del ik32
+        assert np.array_equal(ik.data[0, 0], p.ik.data[b, 0].cpu().numpy())
+        kv = []
+        for tid, s in ((synth.TID_K, s_k), (synth.TID_V, s_v)):
+            x = np.zeros((1, w.Hkv, w.lmax, w.D), np.float32)
+            x[0, :, :L] = synth.kv_tokens(w, tid, b, w.Hkv, w.D, 0, L).numpy()
+            kv.append(oracle.nvfp4_encode(x, s))
+            del x
+        K, V = kv
+        assert np.array_equal(K.scale[0, :, :L], p.k.scale[b, :, :L].cpu().numpy())
+        assert np.array_equal(V.data[0, :, L - 4096:L], p.v.data[b, :, L - 4096:L].cpu().numpy())
+        # selection of every sampled row against the oracle's own pooled scores
+        obs = oracle_index_rows(bf16_values(qi[0])[tokens], ik, pos)
+        osel = oracle.select(obs[:, None], [x + 1 for x in pos])
+        check_selection(sel_h[b, tokens][:, None], osel, obs[:, None], [x + 1 for x in pos], 1)
+        # attention of every sampled row over the GPU's selection
+        o, l = oracle_attend_rows(bf16_values(q[0])[tokens], K, V, sel_h[b, tokens], pos)
+        check_attention(out_h[b, tokens], o)
+        np.testing.assert_allclose(lse_h[b, tokens], l, rtol=1e-4, atol=1e-4)
+        rows += len(tokens)
+    assert rows >= 256

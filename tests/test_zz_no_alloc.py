@@ -1,8 +1,10 @@
 """msa_decode_static: the decode step for callers that cannot allocate device memory
 (e.g. a plugin that a host framework hands only its inputs and outputs).  Its scratch
 is a fixed device array inside libmsa.so; this checks it against msa_decode, which
-takes caller scratch, on two calls in a row (the second call must not be disturbed by
-what the first left in the shared array), and that oversized problems are refused.
+takes caller scratch, on calls in a row (a call must not be disturbed by what an earlier
+call left in the shared array; one problem has rows of more than 1,024 blocks, so its
+selection goes through the array's selection region), and that oversized problems are
+refused.
 
 Collected last on purpose, so a stop-at-first-failure run has already run every
 other test before this one."""
@@ -38,11 +40,29 @@ def _ragged_case():
     return inp
 
 
+def _long_rows_case():
+    # rows of more than 1,024 blocks: msa_decode runs the selection as its own launch, which
+    # writes the selected ids into the second region of the scratch (after the block scores)
+    w = synth.Workload("noalloc_long", B=2, Tq=1, Hq=8, Hkv=1, D=128, HI=4, DI=64, seq_len=163000,
+                       lmax=163840, needles=6, seed=4243)
+    inp = synth.make_inputs(w, device="cuda")
+    inp.seq_lens = [163000, 140001]
+    L = inp.seq_lens[1]
+    inp.k[1, :, L:] = 0
+    inp.v[1, :, L:] = 0
+    inp.ik[1, :, L:] = 0
+    return inp
+
+
 def test_static_scratch_matches_msa_decode_twice():
     torch.cuda.set_device(0)
-    # a larger problem first, then a smaller one: stale scratch from call 1 must not matter
-    for inp in (_ragged_case(), synth.make_inputs(configs.TINY)):
+    # calls in a row over problems of different shapes (the long-row problem twice, the
+    # second time after two other problems overwrote the shared array): stale scratch
+    # from an earlier call must not matter
+    for make in (_long_rows_case, _ragged_case, lambda: synth.make_inputs(configs.TINY), _long_rows_case):
+        inp = make()
         p = problem_from_inputs(inp)
+        assert msa.msa_workspace_size(p) <= msa.MSA_STATIC_SCRATCH_BYTES
         ref = run_decode(p)
         got = _static(p)
         assert int(p.status.item()) == 0
