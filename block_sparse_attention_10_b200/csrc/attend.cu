@@ -114,6 +114,7 @@ __global__ void __cluster_dims__(CL, 1, 1) __launch_bounds__(kAttThreads, 4)
         if (lane == 0) set_status(p.status, MSA_STATUS_SELECT);
         blk = -1;
     }
+    if (blk < p.blk_lo || blk >= p.blk_hi) blk = -1;  // another rank's block (context-parallel decode)
     int nk = 0, nq = 0;
     int64_t vec0 = 0;
     if (blk >= 0) {

@@ -68,7 +68,8 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
             if (b < B) {
                 const int64_t L = clamp_len(p.seq_lens[b], Tq, p.lmax, blockIdx.x == 0 ? p.status : nullptr);
                 lens[b] = (int)L;
-                nb = (int)((L + kBlock - 1) / kBlock);
+                // the sequence's blocks inside [blk_lo, blk_hi)
+                nb = (int)max64(0, min64((L + kBlock - 1) / kBlock, p.blk_hi) - p.blk_lo);
             }
             int x = nb;
 #pragma unroll
@@ -87,14 +88,14 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
     __syncthreads();
     pdl_launch_dependents();
 
-    // blocks past a sequence's length score -inf (no unit covers them)
+    // blocks past a sequence's length, or outside [blk_lo, blk_hi), score -inf (no unit covers them)
     {
         const int64_t total = (int64_t)B * Tq * p.nbmax;
         const int64_t stride = (int64_t)gridDim.x * kIdxThreads;
         for (int64_t i = (int64_t)blockIdx.x * kIdxThreads + threadIdx.x; i < total; i += stride) {
-            const int64_t n = i % p.nbmax;
+            const int64_t n = i % p.nbmax - p.blk_lo;
             const int b = (int)(i / (p.nbmax * Tq));
-            if (n >= prefix[b + 1] - prefix[b]) block_scores[i] = -INFINITY;
+            if (n < 0 || n >= prefix[b + 1] - prefix[b]) block_scores[i] = -INFINITY;
         }
     }
 
@@ -111,7 +112,7 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
     auto issue_upto = [&](uint32_t limit) {
         while (slot_issued < limit && iu < u_end) {
             while (prefix[ib + 1] <= iu) ++ib;
-            const int64_t n = iu - prefix[ib];
+            const int64_t n = p.blk_lo + (iu - prefix[ib]);
             const int valid = (int)min64(kBlock, lens[ib] - n * kBlock) - is * KPS;
             if (valid > 0) {
                 if (lane == 0) {
@@ -154,7 +155,9 @@ __global__ void __launch_bounds__(kIdxThreads, 2)
             cur_b = b;
             idx_load_query<DI, HI, NT>(p, b, g, c, q);
         }
-        if (!idx_block<DI, HI, NT>(p, b, u - prefix[b], lens[b], q, acquire, block_scores, token_scores, g, c)) break;
+        if (!idx_block<DI, HI, NT>(p, b, p.blk_lo + (u - prefix[b]), lens[b], q, acquire, block_scores, token_scores,
+                                   g, c))
+            break;
     }
     // never leave with copies in flight into this warp's stages
     for (uint32_t j = slot; j < slot_issued; ++j)

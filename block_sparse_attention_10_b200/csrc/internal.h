@@ -42,6 +42,11 @@ struct Problem {
     const int32_t* block_table;  // [B][nbmax] page of each block, or nullptr (contiguous caches)
     int64_t num_pages;
     int out_bf16;                // attention output as bf16 (else fp32)
+    // Blocks [blk_lo, blk_hi) of every sequence are the ones this call covers (the whole
+    // context, [0, nbmax), except for the context-parallel entry points, where each rank
+    // holds one contiguous range): the indexer scores only these blocks and attention
+    // skips selected blocks outside them.
+    int64_t blk_lo, blk_hi;
 };
 
 // First cache vector of block n of sequence b, head h of H: contiguous caches hold
@@ -95,6 +100,17 @@ int launch_attend(const Problem& p, const int32_t* sel, float* out, float* lse, 
 // Selection fused into the attention kernel (rows of <= 1,024 blocks; else MSA_EUNSUPPORTED).
 int launch_select_attend(const Problem& p, const float* block_scores, int32_t* sel_out, float* out, float* lse,
                          bool pdl, cudaStream_t st);
+
+// Context-parallel decode (dcp.cu).  Candidates: this rank's best 15 blocks of [blk_lo,
+// blk_hi) per row, from block scores written by the range indexer; merge: G ranks'
+// candidates -> the selection; combine: G attention partials -> the output.
+constexpr int kDcpMaxRanks = 32;
+int launch_dcp_candidates(const Problem& p, const float* block_scores, float* cand_score, int32_t* cand_id, bool pdl,
+                          cudaStream_t st);
+int launch_dcp_merge(const Problem& p, int G, const float* cand_score, const int32_t* cand_id, int32_t* sel,
+                     bool pdl, cudaStream_t st);
+int launch_dcp_combine(const Problem& p, int G, const float* part_out, const float* part_lse, float* out, float* lse,
+                       bool pdl, cudaStream_t st);
 
 // The whole decode step in one persistent launch (decode_fused.cu).  Workspace: byte
 // offsets of its regions; the counter region [0, ctr_bytes) is cleared by the launcher.

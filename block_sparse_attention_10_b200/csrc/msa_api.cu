@@ -99,6 +99,8 @@ Problem to_problem(const msa_params_t* p) {
     q.block_table = p->block_table;
     q.num_pages = p->block_table != nullptr ? p->num_pages : 0;
     q.out_bf16 = p->out_bf16;
+    q.blk_lo = 0;
+    q.blk_hi = q.nbmax;
     return q;
 }
 
@@ -237,6 +239,63 @@ int msa_decode_single_launch(const msa_params_t* p, void* ws, size_t ws_bytes, v
     if (!ws || ws_bytes < fused_layout(q).total || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0)
         return MSA_EWORKSPACE;
     return launch_decode_fused(q, ws, out, lse, sel_out, pdl_enabled(), stream);
+}
+
+// ---------------------------------------------------------------- context-parallel decode
+
+size_t msa_dcp_workspace_size(const msa_params_t* p) {
+    if (check_params(p, true, false) != MSA_OK) return 0;
+    return ws_block_scores_bytes(p);
+}
+
+int msa_dcp_candidates(const msa_params_t* p, int64_t n0, int64_t n1, void* ws, size_t ws_bytes,
+                       float* cand_score, int32_t* cand_id, cudaStream_t stream) {
+    if (int r = check_params(p, true, false)) return r;
+    if (!cand_score || !cand_id) return MSA_EINVAL;
+    Problem q = to_problem(p);
+    if (n0 < 0 || n1 <= n0 || n1 > q.nbmax) return MSA_EINVAL;
+    if ((int64_t)p->Tq * p->HI > 32) return MSA_EUNSUPPORTED;  // decode indexer only
+    if (!ws || ws_bytes < ws_block_scores_bytes(p) || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0)
+        return MSA_EWORKSPACE;
+    q.blk_lo = n0;
+    q.blk_hi = n1;
+    float* bs = static_cast<float*>(ws);
+    const bool pdl = pdl_enabled();
+    if (int r = launch_index_decode(q, bs, nullptr, pdl, stream)) return r;
+    return launch_dcp_candidates(q, bs, cand_score, cand_id, pdl, stream);
+}
+
+int msa_dcp_merge(const msa_params_t* p, int G, const float* cand_score, const int32_t* cand_id, int32_t* sel,
+                  cudaStream_t stream) {
+    if (int r = check_params(p, false, false)) return r;
+    if (!cand_score || !cand_id || !sel) return MSA_EINVAL;
+    if (G < 1) return MSA_EINVAL;
+    if (G > kDcpMaxRanks) return MSA_EUNSUPPORTED;
+    return launch_dcp_merge(to_problem(p), G, cand_score, cand_id, sel, false, stream);
+}
+
+int msa_dcp_attend(const msa_params_t* p, int64_t n0, int64_t n1, const int32_t* sel, float* out, float* lse,
+                   cudaStream_t stream) {
+    if (int r = check_params(p, false, true)) return r;
+    if (!sel || !out || !lse) return MSA_EINVAL;
+    if (!aligned16(out)) return MSA_EALIGN;
+    Problem q = to_problem(p);
+    if (n0 < 0 || n1 <= n0 || n1 > q.nbmax) return MSA_EINVAL;
+    q.blk_lo = n0;
+    q.blk_hi = n1;
+    q.out_bf16 = 0;  // partials stay fp32 until the combine
+    return launch_attend(q, sel, out, lse, false, stream);
+}
+
+int msa_dcp_combine(const msa_params_t* p, int G, const float* part_out, const float* part_lse, void* out_,
+                    float* lse, cudaStream_t stream) {
+    float* out = static_cast<float*>(out_);  // bf16 elements when out_bf16
+    if (int r = check_params(p, false, true)) return r;
+    if (!part_out || !part_lse || !out) return MSA_EINVAL;
+    if (!aligned16(part_out) || !aligned16(out)) return MSA_EALIGN;
+    if (G < 1) return MSA_EINVAL;
+    if (G > kDcpMaxRanks) return MSA_EUNSUPPORTED;
+    return launch_dcp_combine(to_problem(p), G, part_out, part_lse, out, lse, false, stream);
 }
 
 }  // extern "C"

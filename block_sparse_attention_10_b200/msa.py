@@ -28,7 +28,8 @@ MSA_STATUS_TIMEOUT = 4
 # names exported by the C ABI (include/msa.h)
 EXPORTS = ("msa_status_string", "msa_version", "msa_nvfp4_encode", "msa_nvfp4_decode", "msa_nvfp4_amax",
            "msa_workspace_size", "msa_index", "msa_select", "msa_attend", "msa_decode", "msa_decode_static",
-           "msa_workspace_size_single_launch", "msa_decode_single_launch")
+           "msa_workspace_size_single_launch", "msa_decode_single_launch", "msa_dcp_workspace_size",
+           "msa_dcp_candidates", "msa_dcp_merge", "msa_dcp_attend", "msa_dcp_combine")
 MSA_STATIC_SCRATCH_BYTES = 4 << 20
 
 
@@ -80,9 +81,15 @@ def lib() -> ctypes.CDLL:
         L.msa_workspace_size_single_launch.argtypes = [P]
         L.msa_decode_single_launch.argtypes = [P, vp, ctypes.c_size_t, vp, vp, vp, vp]
         L.msa_decode_static.argtypes = [P, vp, vp, vp, vp]
+        L.msa_dcp_workspace_size.restype = ctypes.c_size_t
+        L.msa_dcp_workspace_size.argtypes = [P]
+        L.msa_dcp_candidates.argtypes = [P, i64, i64, vp, ctypes.c_size_t, vp, vp, vp]
+        L.msa_dcp_merge.argtypes = [P, i32, vp, vp, vp, vp]
+        L.msa_dcp_attend.argtypes = [P, i64, i64, vp, vp, vp, vp]
+        L.msa_dcp_combine.argtypes = [P, i32, vp, vp, vp, vp, vp]
         for name in (n for n in EXPORTS
                      if n not in ("msa_status_string", "msa_version", "msa_workspace_size",
-                                  "msa_workspace_size_single_launch")):
+                                  "msa_workspace_size_single_launch", "msa_dcp_workspace_size")):
             getattr(L, name).restype = i32
         _lib = L
     return _lib
@@ -283,3 +290,41 @@ def outputs(p: MsaProblem):
     return (torch.empty(B, Tq, Hq, D, dtype=torch.bfloat16 if p.out_bf16 else torch.float32, device=dev),
             torch.empty(B, Tq, Hq, dtype=torch.float32, device=dev),
             torch.empty(B, Tq, MSA_TOPK_BLOCKS, dtype=torch.int32, device=dev))
+
+
+# --------------------------------------------------------------------------- context-parallel decode
+
+def msa_dcp_workspace_size(p: MsaProblem) -> int:
+    prm = p.params()
+    return int(lib().msa_dcp_workspace_size(ctypes.byref(prm)))
+
+
+def msa_dcp_candidates(p: MsaProblem, n0: int, n1: int, ws: torch.Tensor, cand_score: torch.Tensor,
+                       cand_id: torch.Tensor, stream=None):
+    """This rank's candidates from blocks [n0, n1): fp32 / int32 [B, Tq, 16] (see msa.h)."""
+    prm = p.params()
+    _check(lib().msa_dcp_candidates(ctypes.byref(prm), n0, n1, _ptr(ws), ws.numel() * ws.element_size(),
+                                    _ptr(cand_score), _ptr(cand_id), _stream(stream)), "msa_dcp_candidates")
+
+
+def msa_dcp_merge(p: MsaProblem, cand_score: torch.Tensor, cand_id: torch.Tensor, sel: torch.Tensor, stream=None):
+    """Merge of the G ranks' candidates [G, B, Tq, 16] into the selection [B, Tq, 16]."""
+    prm = p.params()
+    _check(lib().msa_dcp_merge(ctypes.byref(prm), cand_score.shape[0], _ptr(cand_score), _ptr(cand_id), _ptr(sel),
+                               _stream(stream)), "msa_dcp_merge")
+
+
+def msa_dcp_attend(p: MsaProblem, n0: int, n1: int, sel: torch.Tensor, part_out: torch.Tensor,
+                   part_lse: torch.Tensor, stream=None):
+    """Attention over the selected blocks in [n0, n1): fp32 partial out [B, Tq, Hq, D] and lse [B, Tq, Hq]."""
+    prm = p.params()
+    _check(lib().msa_dcp_attend(ctypes.byref(prm), n0, n1, _ptr(sel), _ptr(part_out), _ptr(part_lse),
+                                _stream(stream)), "msa_dcp_attend")
+
+
+def msa_dcp_combine(p: MsaProblem, part_out: torch.Tensor, part_lse: torch.Tensor, out: torch.Tensor,
+                    lse: Optional[torch.Tensor] = None, stream=None):
+    """Combine of G partials [G, B, Tq, Hq, D] / [G, B, Tq, Hq] into out (fp32 or bf16) and lse."""
+    prm = p.params()
+    _check(lib().msa_dcp_combine(ctypes.byref(prm), part_out.shape[0], _ptr(part_out), _ptr(part_lse), _ptr(out),
+                                 _ptr(lse), _stream(stream)), "msa_dcp_combine")

@@ -203,6 +203,72 @@ int msa_decode(const msa_params_t* p, void* ws, size_t ws_bytes, void* out, floa
                int32_t* sel_out, cudaStream_t stream);
 
 /* ---------------------------------------------------------------------------
+ * Indexer decode context parallelism (the pages' "DCP": "vLLM delivers day-0
+ * support for MiniMax-M3.1-Flash", readmex.ai, TL;DR; "vLLM Adds Day-0 Support
+ * for MiniMax-M3.1-Flash on NVIDIA and AMD GPUs", ainewsbites.com, "Kernel and
+ * serving optimizations": the indexer of a long decode context is split over
+ * GPUs).  The pages give no algorithm; this library's reading keeps the
+ * single-GPU result:
+ *
+ *   G ranks split the blocks of every sequence into G contiguous ranges that
+ *   cover [0, lmax/128) without overlap; rank g holds blocks [n0, n1) of the K,
+ *   V and index-K caches (contiguous caches of full capacity of which only the
+ *   range is read, or a paged cache whose block table names pages only for the
+ *   range: entries outside it are never read).  One decode step is
+ *     msa_dcp_candidates (own range) -> all-gather of the candidates ->
+ *     msa_dcp_merge (same result on every rank) -> msa_dcp_attend (own range)
+ *     -> all-gather of the partials -> msa_dcp_combine.
+ *   The merged selection equals msa_decode's bit for bit (every block's pooled
+ *   score is computed by the same arithmetic; the best 15 blocks of the context
+ *   are among the ranks' best 15); the combined output matches msa_decode's
+ *   within the attention tolerance (the partials are merged in another order).
+ *   Exchanged bytes per query row: G x 16 x 8 (candidates) and
+ *   G x Hq x (D + 1) x 4 (partials).  The exchange itself is the caller's (NCCL
+ *   all-gather in the package's Python layer); these calls only compute.
+ *   Decode indexer only: Tq * HI <= 32.  Results are bitwise deterministic.
+ * ------------------------------------------------------------------------- */
+
+/* Scratch for msa_dcp_candidates: the pooled block scores [B][Tq][lmax/128] fp32. */
+size_t msa_dcp_workspace_size(const msa_params_t* p);
+
+/* The indexer and block pooling over blocks [n0, n1) only (0 <= n0 < n1 <= lmax/128),
+ * then, per (sequence, query token), this rank's candidates: its best min(15, c)
+ * blocks other than the query's own block r (c = the visible blocks of the range
+ * other than r), by (score desc, block index asc):
+ *   ws, ws_bytes  at least msa_dcp_workspace_size(p) bytes, 256-byte aligned
+ *   cand_score    fp32 [B][Tq][16], cand_id int32 [B][Tq][16]: the candidates in
+ *                 that order, then (-inf, -1) padding (slot 15 is always padding)
+ * Returns MSA_EINVAL for an empty or out-of-bounds range, MSA_EUNSUPPORTED for
+ * Tq * HI > 32. */
+int msa_dcp_candidates(const msa_params_t* p, int64_t n0, int64_t n1, void* ws, size_t ws_bytes,
+                       float* cand_score, int32_t* cand_id, cudaStream_t stream);
+
+/* Merge of G ranks' candidates (1 <= G <= 32), every rank the same way:
+ *   cand_score fp32 [G][B][Tq][16], cand_id int32 [G][B][Tq][16] (rank g's
+ *   msa_dcp_candidates output at index g)
+ *   sel        int32 [B][Tq][16]: the query's own block plus the best min(15, r)
+ *              pairs by (score desc, id asc), ascending, -1 padded.  Pairs whose id
+ *              is not a visible block other than r are ignored; a pair received
+ *              twice counts once. */
+int msa_dcp_merge(const msa_params_t* p, int G, const float* cand_score, const int32_t* cand_id,
+                  int32_t* sel, cudaStream_t stream);
+
+/* Attention of every query over those of its selected blocks that lie in [n0, n1):
+ *   out  fp32 [B][Tq][Hq][D], normalised over this rank's keys (zeros when the
+ *        rank holds none of the query's selected blocks); out_bf16 is ignored
+ *   lse  fp32 [B][Tq][Hq] (required): natural log of the softmax denominator over
+ *        this rank's keys, -inf when it holds none of them */
+int msa_dcp_attend(const msa_params_t* p, int64_t n0, int64_t n1, const int32_t* sel, float* out, float* lse,
+                   cudaStream_t stream);
+
+/* Combine of G partials (1 <= G <= 32) in rank order:
+ *   part_out fp32 [G][B][Tq][Hq][D], part_lse fp32 [G][B][Tq][Hq]
+ *   out      [B][Tq][Hq][D], fp32 (bf16 with out_bf16): sum_g exp(lse_g - lse) out_g
+ *   lse      fp32 [B][Tq][Hq] or NULL: log sum_g exp(lse_g) */
+int msa_dcp_combine(const msa_params_t* p, int G, const float* part_out, const float* part_lse, void* out,
+                    float* lse, cudaStream_t stream);
+
+/* ---------------------------------------------------------------------------
  * The decode step as one persistent launch.  Prior art: the single-launch
  * "mono" decode path of "vLLM turns MiniMax's day-zero promise into
  * GPU-specific serving code" (upstreambeat.ai, "What changed").  Same results
