@@ -361,7 +361,13 @@ def step_work(w, seq_lens, sel):
 
 def launches_per_step(p):
     """Kernels of ours that one msa_decode call launches: the indexer, then the selection
-    fused into the attention kernel (rows of <= 1,024 blocks) or select + attend."""
+    fused into the attention kernel (rows of <= 1,024 blocks) or select + attend; chunked
+    prefill with 8 query heads per KV head: indexer, select, the three selection-inversion
+    kernels, the block-major attention and the merge of the slot partials."""
+    B, Tq, Hq, _ = p.q.shape
+    HI, Hkv = p.q_idx.shape[2], p.k.data.shape[1]
+    if Tq * HI > 32 and Hq == 8 * Hkv:
+        return 7
     return 2 if p.nbmax <= 1024 else 3
 
 

@@ -1,0 +1,737 @@
+// attend_prefill.cu — exact sparse attention for a chunk of many query tokens (chunked
+// prefill) on the fifth-generation tensor cores.
+//
+// Method ("vLLM Adds Day-0 Support for MiniMax-M3.1-Flash", ainewsbites.com, section "A
+// model built for efficient inference"): every query token attends, with exact softmax,
+// to the keys of its own 16 selected 128-token blocks that it can see; query head h reads
+// KV head h / (Hq/Hkv).  The pages' prefill path fuses its steps ("Kernel and serving
+// optimizations", same page); the design below is this library's.
+//
+// Decode attention gathers, per (token, KV head), its 16 blocks and dequantises them for
+// that token alone.  With thousands of tokens in a chunk, each block is selected by tens
+// of them, so this file turns the work around and goes block by block:
+//   1. ap_count / ap_scan / ap_fill invert the selection: for every (sequence, block) the
+//      list of (token, slot) pairs that selected it (slot = its place in the token's 16);
+//   2. ap_attend_kernel: one persistent CTA per SM walks items (sequence, KV head, block)
+//      cut into tiles of 16 listed tokens x 8 query heads = 128 rows, the tiles spread
+//      evenly over the CTAs.  Per item the 4 compute warps dequantise the block once: K as
+//      bf16 [128 keys x 128 dims] and V transposed as f16 [128 dims x 128 keys], both in the
+//      K-major 128-byte-swizzle layout the tensor cores read (e2m1 x e4m3 is exact in both
+//      types); one warp streams the raw block (bulk copies) and each tile's query rows
+//      (TMA, 128-byte swizzle, one 8-row atom per token, no multicast); one thread issues
+//        S = Q K^T   tcgen05.mma kind::f16, bf16, 128 x 128 x 128, fp32 in TMEM,
+//        O = P V     tcgen05.mma kind::f16, f16,  128 x 128 x 128, fp32 in TMEM,
+//      with S and O double-buffered (4 x 128 TMEM columns) so that the softmax of one tile
+//      overlaps the MMAs of the next; the compute warps (one TMEM lane = one row each) read
+//      S with tcgen05.ld, mask keys past the token's position, take the row max, write
+//      P = 2^(S c - m c) as f16 into shared memory for the second MMA, and finally write
+//      the row's output normalised by its own sum (f16, unscaled by the V tensor scale)
+//      and its log-sum-exp to the token's slot;
+//   3. ap_merge_kernel combines each token's (up to) 16 slot partials in slot order:
+//      lse = log sum_s exp(lse_s), out = s_V * sum_s exp(lse_s - lse) o_s.
+// Every output row's arithmetic is independent of the tile row it occupies and the merge
+// order is fixed, so results are bitwise reproducible although the lists are filled with
+// atomics.  Every wait is bounded (MSA_STATUS_TIMEOUT | MSA_STATUS_AT_ATTEND).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "internal.h"
+#include "tcgen05.cuh"
+
+namespace msa {
+namespace {
+
+constexpr int kApG = 8;                // query heads per KV head on this path
+constexpr int kApTok = 128 / kApG;     // listed tokens per 128-row tile
+constexpr int kApComputeWarps = 4;
+constexpr int kApMmaWarp = 4;
+constexpr int kApTmaWarp = 5;
+constexpr int kApThreads = 32 * 6;
+constexpr int kApTile = 32768;         // 128 rows x 128 16-bit elements: two 16 KB K-blocks
+constexpr int kApKB = 16384;           // one K-block (64 elements of 128 rows)
+constexpr int kOffK = 0;               // K, bf16 [key][dim]
+constexpr int kOffV = kApTile;         // V^T, f16 [dim][key]
+constexpr int kOffQ = 2 * kApTile;     // 2 query stages
+constexpr int kOffP = 4 * kApTile;     // 2 P buffers, f16 [row][key]
+constexpr int kOffRaw = 6 * kApTile;   // the raw NVFP4 block: K nibbles, K scales, V nibbles, V scales
+constexpr int kRawK = 0, kRawKs = 8192, kRawV = 9216, kRawVs = 17408, kRawBytes = 18432;
+constexpr int kOffBar = kOffRaw + kRawBytes;
+constexpr size_t kApSmem = 1024 + kOffBar + 256;
+constexpr uint32_t kApTmemCols = 512;  // S at columns 0 / 128, O at 256 / 384
+constexpr float kApLog2e = 1.4426950408889634f;
+constexpr float kApLn2 = 0.6931471805599453f;
+
+struct ApWork {
+    const int32_t* sel;         // [B][Tq][16]
+    int32_t* cnt;               // [B * nbmax] tokens that selected block n of sequence b
+    int32_t* cursor;            // [B * nbmax] fill positions
+    int32_t* list_off;          // [B * nbmax] start of each list
+    int32_t* tile_start;        // [items + 1] first tile of item (b, kvh, n); last entry = total
+    int32_t* list;              // [B * Tq * 16] entries t * 16 + slot, grouped by (b, n)
+    float* part_lse;            // [B][Tq][16][Hq]
+    __half* part_o;             // [B][Tq][16][Hq][D]
+};
+
+// ------------------------------------------------------------------ selection inversion
+
+__device__ __forceinline__ bool ap_valid_entry(const Problem& p, const int32_t* sel, int64_t e, int& b, int& t,
+                                               int& n) {
+    const int64_t bt = e / kTopK;
+    b = (int)(bt / p.Tq);
+    t = (int)(bt % p.Tq);
+    n = sel[e];
+    const int64_t L = clamp_len(p.seq_lens[b], p.Tq, p.lmax, nullptr);
+    const int64_t nvis = (L - p.Tq + t) / kBlock + 1;
+    if (n >= nvis) set_status(p.status, MSA_STATUS_SELECT);
+    return n >= 0 && n < nvis;
+}
+
+__global__ void ap_count_kernel(const Problem p, const ApWork w) {
+    pdl_wait();
+    pdl_launch_dependents();
+    const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= (int64_t)p.B * p.Tq * kTopK) return;
+    int b, t, n;
+    if (ap_valid_entry(p, w.sel, e, b, t, n)) atomicAdd(&w.cnt[(int64_t)b * p.nbmax + n], 1);
+}
+
+// Exclusive scan of `count(i)` for i < N into out[0..N] (out[N] = total) by one CTA of 1024 threads.
+template <class Count>
+__device__ __forceinline__ void ap_block_scan(int64_t N, Count&& count, int32_t* out, int32_t* warp_sums) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int32_t carry = 0;
+    for (int64_t base = 0; base < N; base += 1024) {
+        const int64_t i = base + tid;
+        const int32_t x = i < N ? count(i) : 0;
+        int32_t v = x;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t y = __shfl_up_sync(0xffffffffu, v, o);
+            if (lane >= o) v += y;
+        }
+        if (lane == 31) warp_sums[warp] = v;
+        __syncthreads();
+        if (warp == 0) {
+            int32_t s = warp_sums[lane];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int32_t y = __shfl_up_sync(0xffffffffu, s, o);
+                if (lane >= o) s += y;
+            }
+            warp_sums[lane] = s;  // inclusive sums of the warps
+        }
+        __syncthreads();
+        const int32_t before = carry + (warp > 0 ? warp_sums[warp - 1] : 0) + v - x;
+        if (i < N) out[i] = before;
+        const int32_t total = warp_sums[31];
+        __syncthreads();  // warp_sums is rewritten by the next chunk
+        carry += total;
+    }
+    if (tid == 0) out[N] = carry;
+}
+
+__global__ void __launch_bounds__(1024) ap_scan_kernel(const Problem p, const ApWork w) {
+    __shared__ int32_t warp_sums[32];
+    pdl_wait();
+    pdl_launch_dependents();
+    const int64_t lists = (int64_t)p.B * p.nbmax;
+    ap_block_scan(lists, [&](int64_t i) { return w.cnt[i]; }, w.list_off, warp_sums);
+    for (int64_t i = threadIdx.x; i < lists; i += 1024) w.cursor[i] = 0;
+    // tiles of item (b, kvh, n): ceil(cnt[b][n] / 16)
+    const int64_t items = lists * p.Hkv;
+    ap_block_scan(
+        items,
+        [&](int64_t i) {
+            const int64_t n = i % p.nbmax, b = i / (p.nbmax * p.Hkv);
+            return (w.cnt[b * p.nbmax + n] + kApTok - 1) / kApTok;
+        },
+        w.tile_start, warp_sums);
+}
+
+__global__ void ap_fill_kernel(const Problem p, const ApWork w) {
+    pdl_wait();
+    pdl_launch_dependents();
+    const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= (int64_t)p.B * p.Tq * kTopK) return;
+    int b, t, n;
+    if (ap_valid_entry(p, w.sel, e, b, t, n)) {
+        const int64_t ln = (int64_t)b * p.nbmax + n;
+        const int at = atomicAdd(&w.cursor[ln], 1);
+        w.list[w.list_off[ln] + at] = t * kTopK + (int)(e % kTopK);
+    }
+}
+
+// ------------------------------------------------------------------ block-major attention
+
+// The CTA's walk over its tiles: item = (b * Hkv + kvh) * nbmax + n, tiles
+// [tile_start[item], tile_start[item + 1]).
+struct ApWalk {
+    int64_t item;
+    __device__ __forceinline__ void seek(const int32_t* ts, int64_t items, int tau) {
+        int64_t lo = 0, hi = items;  // ts[0] = 0 <= tau < ts[items]
+        while (hi - lo > 1) {
+            const int64_t mid = (lo + hi) >> 1;
+            if (ts[mid] <= tau) lo = mid;
+            else hi = mid;
+        }
+        item = lo;
+    }
+    __device__ __forceinline__ void advance(const int32_t* ts, int tau) {
+        while (ts[item + 1] <= tau) ++item;
+    }
+};
+
+__device__ __forceinline__ uint32_t f16x2_to_bf16x2(uint32_t h) {
+    const __half2 v = *reinterpret_cast<const __half2*>(&h);
+    const __nv_bfloat162 b = __floats2bfloat162_rn(__low2float(v), __high2float(v));
+    return *reinterpret_cast<const uint32_t*>(&b);
+}
+
+// The raw NVFP4 block (keys kbase .. kbase + 127 of one KV head) -> K (bf16 [key][dim]) and
+// V^T (f16 [dim][key]), 128-byte swizzle, K-major; keys at or past L become zeros.
+__device__ __forceinline__ void ap_dequant(uint8_t* smem, int64_t kbase, int64_t L, int tid) {
+    const uint8_t* raw = smem + kOffRaw;
+    const int nvalid = (int)min64(kBlock, max64(0, L - kbase));
+    uint8_t* kt = smem + kOffK;
+#pragma unroll 4
+    for (int k = 0; k < 16; ++k) {
+        const int q = tid + 128 * k;
+        const int j = q >> 4, cr = q & 15;  // key j, dims 8 cr .. 8 cr + 7
+        uint32_t w = *reinterpret_cast<const uint32_t*>(raw + kRawK + j * 64 + cr * 4);
+        uint32_t sc = raw[kRawKs + j * 8 + (cr >> 1)];
+        if (j >= nvalid) w = sc = 0u;
+        uint32_t h[4];
+        e2m1x8_to_f16x8(w, h[0], h[1], h[2], h[3]);
+        const uint32_t s2 = e4m3_bcast_f16x2(sc);
+        uint4 o;
+        o.x = f16x2_to_bf16x2(hmul2(h[0], s2));
+        o.y = f16x2_to_bf16x2(hmul2(h[1], s2));
+        o.z = f16x2_to_bf16x2(hmul2(h[2], s2));
+        o.w = f16x2_to_bf16x2(hmul2(h[3], s2));
+        *reinterpret_cast<uint4*>(kt + (cr >> 3) * kApKB + j * 128 + (((cr & 7) ^ (j & 7)) << 4)) = o;
+    }
+    // V^T: thread = (dims 16 w16 .. 16 w16 + 15, keys 8 kg .. 8 kg + 7) -> 16 rows x one 16-byte chunk
+    uint8_t* vt = smem + kOffV;
+    const int w16 = tid & 7, kg = tid >> 3;
+    uint2 x[8];
+    uint32_t s[8];
+#pragma unroll
+    for (int a = 0; a < 8; ++a) {
+        const int key = kg * 8 + a;
+        x[a] = *reinterpret_cast<const uint2*>(raw + kRawV + key * 64 + w16 * 8);
+        s[a] = raw[kRawVs + key * 8 + w16];
+        if (key >= nvalid) {
+            x[a] = make_uint2(0u, 0u);
+            s[a] = 0u;
+        }
+    }
+    uint32_t rows[16][4];  // [dim 16 w16 + r][key pair i]
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t sc = e4m3x2_to_f16x2(s[2 * i] | (s[2 * i + 1] << 8));  // (key 2i, key 2i+1)
+#pragma unroll
+        for (int hw = 0; hw < 2; ++hw) {
+            const uint32_t A = hw ? x[2 * i].y : x[2 * i].x, Bw = hw ? x[2 * i + 1].y : x[2 * i + 1].x;
+            const uint32_t ev = (A & 0x0F0F0F0Fu) | ((Bw << 4) & 0xF0F0F0F0u);  // byte k: dim 8 hw + 2k
+            const uint32_t od = ((A >> 4) & 0x0F0F0F0Fu) | (Bw & 0xF0F0F0F0u);  // byte k: dim 8 hw + 2k + 1
+            uint32_t e[4], o[4];
+            e2m1x8_to_f16x8(ev, e[0], e[1], e[2], e[3]);
+            e2m1x8_to_f16x8(od, o[0], o[1], o[2], o[3]);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                rows[8 * hw + 2 * k][i] = hmul2(e[k], sc);
+                rows[8 * hw + 2 * k + 1][i] = hmul2(o[k], sc);
+            }
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+        const int d = 16 * w16 + r;
+        *reinterpret_cast<uint4*>(vt + (kg >> 3) * kApKB + d * 128 + (((kg & 7) ^ (d & 7)) << 4)) =
+            make_uint4(rows[r][0], rows[r][1], rows[r][2], rows[r][3]);
+    }
+}
+
+template <bool PAGED>
+__global__ void __launch_bounds__(kApThreads, 1)
+    ap_attend_kernel(const Problem p, const ApWork w, const __grid_constant__ CUtensorMap tmap) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kOffBar);
+    uint64_t* raw_full = bar + 0;
+    uint64_t* raw_empty = bar + 1;
+    uint64_t* kv_full = bar + 2;
+    uint64_t* kv_empty = bar + 3;
+    uint64_t* q_full = bar + 4;    // [2]
+    uint64_t* q_empty = bar + 6;   // [2]
+    uint64_t* s_full = bar + 8;    // [2]
+    uint64_t* s_empty = bar + 10;  // [2]
+    uint64_t* p_full = bar + 12;   // [2]
+    uint64_t* p_empty = bar + 14;  // [2]
+    uint64_t* o_full = bar + 16;   // [2]
+    uint64_t* o_empty = bar + 18;  // [2]
+    uint64_t* done = bar + 20;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 21);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_wait();
+    if (threadIdx.x == 0) {
+        mbar_init(raw_full, 1);
+        mbar_init(raw_empty, kApComputeWarps);
+        mbar_init(kv_full, kApComputeWarps);
+        mbar_init(kv_empty, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&q_full[s], 1);
+            mbar_init(&q_empty[s], 1);
+            mbar_init(&s_full[s], 1);
+            mbar_init(&s_empty[s], kApComputeWarps);
+            mbar_init(&p_full[s], kApComputeWarps);
+            mbar_init(&p_empty[s], 1);
+            mbar_init(&o_full[s], 1);
+            mbar_init(&o_empty[s], kApComputeWarps);
+        }
+        mbar_init(done, 1);
+        fence_mbar_init();
+    }
+    if (warp == kApMmaWarp) {
+        tmem_alloc(tmem_slot, kApTmemCols);
+        tmem_relinquish();
+    }
+    tcgen05_fence_before();
+    __syncthreads();
+    tcgen05_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    pdl_launch_dependents();
+
+    const int64_t items = (int64_t)p.B * p.Hkv * p.nbmax;
+    const int total = w.tile_start[items];
+    const int t0 = (int)((int64_t)total * blockIdx.x / gridDim.x);
+    const int t1 = (int)((int64_t)total * (blockIdx.x + 1) / gridDim.x);
+    const int Tq = p.Tq;
+    auto fail = [&]() { set_status(p.status, MSA_STATUS_TIMEOUT | MSA_STATUS_AT_ATTEND); };
+
+    if (warp == kApTmaWarp) {
+        // ------------------------------------------------------------ producer: raw blocks, query tiles
+        if (lane == 0 && t0 < t1) {
+            ApWalk wk;
+            wk.seek(w.tile_start, items, t0);
+            int64_t cur = -1;
+            int it = -1, issued = 0;
+            bool ok = true;
+            for (int tau = t0; tau < t1 && ok; ++tau) {
+                const int i = tau - t0, sb = i & 1;
+                wk.advance(w.tile_start, tau);
+                const int64_t n = wk.item % p.nbmax, bk = wk.item / p.nbmax;
+                const int kvh = (int)(bk % p.Hkv), b = (int)(bk / p.Hkv);
+                if (wk.item != cur) {
+                    cur = wk.item;
+                    ++it;
+                    if (it >= 1 && !mbar_wait(raw_empty, (it - 1) & 1)) {
+                        fail();
+                        ok = false;
+                        break;
+                    }
+                    const int64_t vec = block_vec<PAGED>(p, b, n, kvh, p.Hkv);
+                    uint8_t* raw = smem + kOffRaw;
+                    mbar_arrive_expect_tx(raw_full, 2 * (8192 + 1024));
+                    bulk_g2s(raw + kRawK, p.k.data + vec * 64, 8192, raw_full);
+                    bulk_g2s(raw + kRawKs, p.k.scale + vec * 8, 1024, raw_full);
+                    bulk_g2s(raw + kRawV, p.v.data + vec * 64, 8192, raw_full);
+                    bulk_g2s(raw + kRawVs, p.v.scale + vec * 8, 1024, raw_full);
+                }
+                const int64_t ln = (int64_t)b * p.nbmax + n;
+                const int j = tau - w.tile_start[wk.item];
+                const int ntok = min(kApTok, w.cnt[ln] - j * kApTok);
+                if (i >= 2 && !mbar_wait(&q_empty[sb], ((i >> 1) - 1) & 1)) {
+                    fail();
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(&q_full[sb], (uint32_t)(ntok * 2 * 1024));
+                const int32_t* lst = w.list + w.list_off[ln] + j * kApTok;
+                uint8_t* qs = smem + kOffQ + sb * kApTile;
+                for (int k = 0; k < ntok; ++k) {
+                    const int t = lst[k] / kTopK;
+                    tma_load_4d(qs + k * 1024, &tmap, 0, kvh * kApG, t, b, &q_full[sb]);
+                    tma_load_4d(qs + kApKB + k * 1024, &tmap, 64, kvh * kApG, t, b, &q_full[sb]);
+                }
+                issued = i + 1;
+            }
+            // never leave with copies in flight into this CTA's shared memory
+            for (int i = max(0, issued - 2); i < issued; ++i)
+                if (!mbar_wait(&q_full[i & 1], (i >> 1) & 1)) {
+                    fail();
+                    break;
+                }
+            if (it >= 0 && !mbar_wait(raw_full, it & 1)) fail();
+        }
+    } else if (warp == kApMmaWarp) {
+        // ------------------------------------------------------------ MMA issuer (one thread)
+        if (lane == 0 && t0 < t1) {
+            constexpr uint32_t idesc_s = umma_idesc_bf16_f32(128, 128);
+            constexpr uint32_t idesc_o = umma_idesc_f16_f32(128, 128);
+            const uint32_t kt = smem_u32(smem + kOffK), vt = smem_u32(smem + kOffV);
+            auto pv = [&](int i) -> bool {
+                const int sb = i & 1;
+                if (!mbar_wait(&p_full[sb], (i >> 1) & 1)) return false;
+                if (i >= 2 && !mbar_wait(&o_empty[sb], ((i >> 1) - 1) & 1)) return false;
+                tcgen05_fence_after();
+                const uint32_t pa = smem_u32(smem + kOffP + sb * kApTile);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    umma_bf16_ss(tmem + 256 + sb * 128, umma_desc_k_sw128(pa + (k >> 2) * kApKB + (k & 3) * 32),
+                                 umma_desc_k_sw128(vt + (k >> 2) * kApKB + (k & 3) * 32), idesc_o, k > 0 ? 1u : 0u);
+                umma_commit(&p_empty[sb]);
+                umma_commit(&o_full[sb]);
+                return true;
+            };
+            ApWalk wk;
+            wk.seek(w.tile_start, items, t0);
+            int64_t cur = -1;
+            int it = -1;
+            bool ok = true, pending = false;
+            for (int tau = t0; tau < t1 && ok; ++tau) {
+                const int i = tau - t0, sb = i & 1;
+                wk.advance(w.tile_start, tau);
+                if (wk.item != cur) {
+                    if (pending && !pv(i - 1)) {
+                        ok = false;
+                        break;
+                    }
+                    pending = false;
+                    if (it >= 0) umma_commit(kv_empty);  // every MMA reading this item's K and V
+                    cur = wk.item;
+                    ++it;
+                    if (!mbar_wait(kv_full, it & 1)) {
+                        ok = false;
+                        break;
+                    }
+                    tcgen05_fence_after();
+                }
+                if (!mbar_wait(&q_full[sb], (i >> 1) & 1) || (i >= 2 && !mbar_wait(&s_empty[sb], ((i >> 1) - 1) & 1))) {
+                    ok = false;
+                    break;
+                }
+                tcgen05_fence_after();
+                const uint32_t qa = smem_u32(smem + kOffQ + sb * kApTile);
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    umma_bf16_ss(tmem + sb * 128, umma_desc_k_sw128(qa + (k >> 2) * kApKB + (k & 3) * 32),
+                                 umma_desc_k_sw128(kt + (k >> 2) * kApKB + (k & 3) * 32), idesc_s, k > 0 ? 1u : 0u);
+                umma_commit(&q_empty[sb]);
+                umma_commit(&s_full[sb]);
+                if (pending && !pv(i - 1)) {
+                    ok = false;
+                    break;
+                }
+                pending = true;
+            }
+            if (ok && pending && !pv(t1 - t0 - 1)) ok = false;
+            if (!ok) fail();
+            // every MMA issued has completed before the CTA releases its tensor memory
+            umma_commit(done);
+            if (!mbar_wait(done, 0)) fail();
+        }
+    } else {
+        // ------------------------------------------------------------ compute warps: dequant, softmax, output
+        const int row = threadIdx.x;  // TMEM lane and tile row: token slot row / 8, head row % 8
+        const int tslot = row >> 3, hq = row & 7;
+        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+        const float c = p.softmax_scale * p.k.s_t * kApLog2e;
+        // the previous tile's row state, for its output step
+        float prev_mc = 0.0f, prev_l = 0.0f;
+        int64_t prev_row = -1;
+        auto wait_all = [&](uint64_t* b_, uint32_t parity) -> bool {
+            return __all_sync(0xffffffffu, mbar_wait(b_, parity)) != 0;
+        };
+        auto output = [&](int i, float mc, float l, int64_t orow) -> bool {
+            const int sb = i & 1;
+            if (!wait_all(&o_full[sb], (i >> 1) & 1)) return false;
+            tcgen05_fence_after();
+            const float inv = l > 0.0f ? 1.0f / l : 0.0f;
+#pragma unroll
+            for (int c4 = 0; c4 < 4; ++c4) {
+                float o[32];
+                tmem_ld32(lane_base + 256 + sb * 128 + c4 * 32, o);
+                tmem_wait_ld();
+                if (orow >= 0) {
+                    uint4* dst = reinterpret_cast<uint4*>(w.part_o + orow * 128 + c4 * 32);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        dst[q] = make_uint4(pack_f16x2(o[8 * q] * inv, o[8 * q + 1] * inv),
+                                            pack_f16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
+                                            pack_f16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv),
+                                            pack_f16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
+                }
+            }
+            tcgen05_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&o_empty[sb]);
+            if (orow >= 0) w.part_lse[orow] = (mc + log2f(l)) * kApLn2;
+            return true;
+        };
+        bool ok = true;
+        if (t0 < t1) {
+            ApWalk wk;
+            wk.seek(w.tile_start, items, t0);
+            int64_t cur = -1;
+            int it = -1;
+            for (int tau = t0; tau < t1; ++tau) {
+                const int i = tau - t0, sb = i & 1;
+                wk.advance(w.tile_start, tau);
+                const int64_t n = wk.item % p.nbmax, bk = wk.item / p.nbmax;
+                const int kvh = (int)(bk % p.Hkv), b = (int)(bk / p.Hkv);
+                const int64_t L = clamp_len(p.seq_lens[b], Tq, p.lmax, nullptr);
+                if (wk.item != cur) {
+                    cur = wk.item;
+                    ++it;
+                    if (!wait_all(raw_full, it & 1) || (it >= 1 && !wait_all(kv_empty, (it - 1) & 1))) {
+                        ok = false;
+                        break;
+                    }
+                    ap_dequant(smem, n * kBlock, L, row);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        mbar_arrive(raw_empty);
+                        mbar_arrive(kv_full);
+                    }
+                }
+                // ---- softmax of tile i
+                const int64_t ln = (int64_t)b * p.nbmax + n;
+                const int j = tau - w.tile_start[wk.item];
+                const int ntok = min(kApTok, w.cnt[ln] - j * kApTok);
+                int kvis = 0;
+                int64_t orow = -1;
+                if (tslot < ntok) {
+                    const int e = w.list[w.list_off[ln] + j * kApTok + tslot];
+                    const int t = e / kTopK, slot = e % kTopK;
+                    kvis = (int)min64(kBlock, L - Tq + t - n * kBlock + 1);
+                    orow = (((int64_t)b * Tq + t) * kTopK + slot) * p.Hq + kvh * kApG + hq;
+                }
+                if (!wait_all(&s_full[sb], (i >> 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                tcgen05_fence_after();
+                float v[4][32];  // S row: key k in v[k / 32][k % 32]
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(lane_base + sb * 128 + c4 * 32, v[c4]);
+                tmem_wait_ld();
+                tcgen05_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&s_empty[sb]);
+                float m = -INFINITY;
+#pragma unroll
+                for (int k = 0; k < 128; ++k)
+                    if (k < kvis) m = fmaxf(m, v[k >> 5][k & 31]);
+                const float mc = kvis > 0 ? m * c : 0.0f;
+                if (i >= 2 && !wait_all(&p_empty[sb], ((i >> 1) - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                uint8_t* prow = smem + kOffP + sb * kApTile + row * 128;
+                float l = 0.0f;
+#pragma unroll
+                for (int cc = 0; cc < 16; ++cc) {
+                    float e8[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int k = cc * 8 + u;
+                        e8[u] = k < kvis ? ex2_approx(fmaf(v[k >> 5][k & 31], c, -mc)) : 0.0f;
+                        l += e8[u];
+                    }
+                    *reinterpret_cast<uint4*>(prow + (cc >> 3) * kApKB + (((cc & 7) ^ (row & 7)) << 4)) =
+                        make_uint4(pack_f16x2(e8[0], e8[1]), pack_f16x2(e8[2], e8[3]), pack_f16x2(e8[4], e8[5]),
+                                   pack_f16x2(e8[6], e8[7]));
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&p_full[sb]);
+                // ---- output of tile i - 1 (its PV MMA ran while this tile's softmax did)
+                if (i >= 1 && !output(i - 1, prev_mc, prev_l, prev_row)) {
+                    ok = false;
+                    break;
+                }
+                prev_mc = mc;
+                prev_l = l;
+                prev_row = orow;
+            }
+            if (ok && !output(t1 - t0 - 1, prev_mc, prev_l, prev_row)) ok = false;
+            if (!ok && lane == 0) fail();
+        }
+    }
+
+    tcgen05_fence_before();
+    __syncthreads();
+    if (warp == kApMmaWarp) {
+        tcgen05_fence_after();
+        tmem_dealloc(tmem, kApTmemCols);
+    }
+}
+
+// ------------------------------------------------------------------ merge of the slot partials
+
+// One thread per (sequence, token, query head, 8 dims).
+__global__ void __launch_bounds__(256) ap_merge_kernel(const Problem p, const ApWork w, float* __restrict__ out,
+                                                       float* __restrict__ lse) {
+    pdl_wait();
+    pdl_launch_dependents();
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t heads = (int64_t)p.B * p.Tq * p.Hq;
+    if (i >= heads * 16) return;
+    const int g8 = (int)(i & 15);
+    const int64_t rh = i >> 4;
+    const int hq = (int)(rh % p.Hq);
+    const int64_t bt = rh / p.Hq;
+    const int b = (int)(bt / p.Tq), t = (int)(bt % p.Tq);
+    const int64_t L = clamp_len(p.seq_lens[b], p.Tq, p.lmax, nullptr);
+    const int64_t nvis = (L - p.Tq + t) / kBlock + 1;
+    float ls[kTopK];
+    float M = -INFINITY;
+#pragma unroll
+    for (int s = 0; s < kTopK; ++s) {
+        const int n = w.sel[bt * kTopK + s];
+        ls[s] = (n >= 0 && n < nvis) ? w.part_lse[(bt * kTopK + s) * p.Hq + hq] : -INFINITY;
+        M = fmaxf(M, ls[s]);
+    }
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    float W = 0.0f;
+    if (M != -INFINITY) {
+#pragma unroll
+        for (int s = 0; s < kTopK; ++s) {
+            if (ls[s] == -INFINITY) continue;
+            const float wt = expf(ls[s] - M);
+            W += wt;
+            const uint4 v = *reinterpret_cast<const uint4*>(w.part_o + ((bt * kTopK + s) * p.Hq + hq) * 128 + g8 * 8);
+            const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&vv[q]));
+                acc[2 * q] += wt * f.x;
+                acc[2 * q + 1] += wt * f.y;
+            }
+        }
+    }
+    const float inv = W > 0.0f ? p.v.s_t / W : 0.0f;
+    const int64_t o = (bt * p.Hq + hq) * 128 + g8 * 8;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) store_out2(p, out, o + 2 * q, acc[2 * q] * inv, acc[2 * q + 1] * inv);
+    if (g8 == 0 && lse != nullptr) lse[bt * p.Hq + hq] = W > 0.0f ? M + logf(W) : -INFINITY;
+}
+
+// ------------------------------------------------------------------ host side
+
+constexpr size_t kApAlign = 256;
+size_t ap_round(size_t x) { return (x + kApAlign - 1) / kApAlign * kApAlign; }
+
+struct ApLayout {
+    size_t cnt, cursor, off, tstart, list, lse, po, total;
+};
+
+ApLayout ap_layout(const Problem& p) {
+    ApLayout a;
+    const size_t lists = (size_t)p.B * p.nbmax, items = lists * p.Hkv, entries = (size_t)p.B * p.Tq * kTopK;
+    size_t at = 0;
+    a.cnt = at;
+    at += ap_round(lists * 4);
+    a.cursor = at;
+    at += ap_round(lists * 4);
+    a.off = at;
+    at += ap_round(lists * 4);
+    a.tstart = at;
+    at += ap_round((items + 1) * 4);
+    a.list = at;
+    at += ap_round(entries * 4);
+    a.lse = at;
+    at += ap_round(entries * p.Hq * 4);
+    a.po = at;
+    at += ap_round(entries * p.Hq * 128 * 2);
+    a.total = at;
+    return a;
+}
+
+cudaLaunchConfig_t ap_config(dim3 grid, dim3 block, size_t smem, bool pdl, cudaStream_t st,
+                             cudaLaunchAttribute* attr) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = pdl ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cfg;
+}
+
+template <bool PAGED>
+int launch_ap_attend(const Problem& p, const ApWork& w, bool pdl, cudaStream_t st) {
+    auto enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encode_entry());
+    if (enc == nullptr) return MSA_ECUDA;
+    // queries [B][Tq][Hq][128] bf16: boxes of 64 dims x 8 heads of one token, 128-byte swizzle
+    CUtensorMap tmap;
+    const cuuint64_t dims[4] = {128, (cuuint64_t)p.Hq, (cuuint64_t)p.Tq, (cuuint64_t)p.B};
+    const cuuint64_t strides[3] = {(cuuint64_t)128 * 2, (cuuint64_t)p.Hq * 128 * 2, (cuuint64_t)p.Tq * p.Hq * 128 * 2};
+    const cuuint32_t box[4] = {64, (cuuint32_t)kApG, 1, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    if (enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<__nv_bfloat16*>(p.q), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return MSA_ECUDA;
+    auto kern = ap_attend_kernel<PAGED>;
+    static int configured_dev = -1;
+    const DeviceInfo& di = device_info();
+    if (configured_dev != di.device) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kApSmem) != cudaSuccess)
+            return MSA_ECUDA;
+        configured_dev = di.device;
+    }
+    cudaLaunchAttribute attr[1];
+    cudaLaunchConfig_t cfg = ap_config(dim3((unsigned)di.num_sms), dim3(kApThreads), kApSmem, pdl, st, attr);
+    if (cudaLaunchKernelEx(&cfg, kern, p, w, tmap) != cudaSuccess) return MSA_ECUDA;
+    return MSA_OK;
+}
+
+}  // namespace
+
+bool attend_prefill_supported(const Problem& p) {
+    return (int64_t)p.Tq * p.HI > 32 && p.Hkv > 0 && p.Hq == kApG * p.Hkv && p.D == 128 &&
+           (int64_t)p.B * p.Tq * kTopK * p.Hkv < 0x7FFFFFFFll;
+}
+
+size_t attend_prefill_ws_bytes(const Problem& p) { return attend_prefill_supported(p) ? ap_layout(p).total : 0; }
+
+int launch_attend_prefill(const Problem& p, const int32_t* sel, void* ws, float* out, float* lse, bool pdl,
+                          cudaStream_t st) {
+    if (!attend_prefill_supported(p)) return MSA_EUNSUPPORTED;
+    const ApLayout a = ap_layout(p);
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    ApWork w;
+    w.sel = sel;
+    w.cnt = reinterpret_cast<int32_t*>(base + a.cnt);
+    w.cursor = reinterpret_cast<int32_t*>(base + a.cursor);
+    w.list_off = reinterpret_cast<int32_t*>(base + a.off);
+    w.tile_start = reinterpret_cast<int32_t*>(base + a.tstart);
+    w.list = reinterpret_cast<int32_t*>(base + a.list);
+    w.part_lse = reinterpret_cast<float*>(base + a.lse);
+    w.part_o = reinterpret_cast<__half*>(base + a.po);
+    const int64_t entries = (int64_t)p.B * p.Tq * kTopK;
+    if (cudaMemsetAsync(w.cnt, 0, (size_t)p.B * p.nbmax * 4, st) != cudaSuccess) return MSA_ECUDA;
+    cudaLaunchAttribute attr[1];
+    const dim3 eg((unsigned)((entries + 255) / 256));
+    cudaLaunchConfig_t cfg = ap_config(eg, dim3(256), 0, false, st, attr);
+    if (cudaLaunchKernelEx(&cfg, ap_count_kernel, p, w) != cudaSuccess) return MSA_ECUDA;
+    cfg = ap_config(dim3(1), dim3(1024), 0, pdl, st, attr);
+    if (cudaLaunchKernelEx(&cfg, ap_scan_kernel, p, w) != cudaSuccess) return MSA_ECUDA;
+    cfg = ap_config(eg, dim3(256), 0, pdl, st, attr);
+    if (cudaLaunchKernelEx(&cfg, ap_fill_kernel, p, w) != cudaSuccess) return MSA_ECUDA;
+    const int r = p.block_table != nullptr ? launch_ap_attend<true>(p, w, pdl, st) : launch_ap_attend<false>(p, w, pdl, st);
+    if (r != MSA_OK) return r;
+    const int64_t threads = (int64_t)p.B * p.Tq * p.Hq * 16;
+    cfg = ap_config(dim3((unsigned)((threads + 255) / 256)), dim3(256), 0, pdl, st, attr);
+    if (cudaLaunchKernelEx(&cfg, ap_merge_kernel, p, w, out, lse) != cudaSuccess) return MSA_ECUDA;
+    return MSA_OK;
+}
+
+}  // namespace msa

@@ -323,15 +323,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (fn == nullptr) {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
-    return fn;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encode_entry());
 }
 
 template <int DI, int HI, bool PAGED>
@@ -383,6 +375,18 @@ int launch_pf_hi(const Problem& p, float* bs, bool pdl, cudaStream_t st) {
 }
 
 }  // namespace
+
+void* tensor_map_encode_entry() {
+    static void* fn = nullptr;
+    if (fn == nullptr) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = ptr;
+    }
+    return fn;
+}
 
 int launch_index_prefill(const Problem& p, float* block_scores, bool pdl, cudaStream_t st) {
     if (p.pool_mode != 0) return MSA_EUNSUPPORTED;

@@ -101,6 +101,16 @@ int launch_attend(const Problem& p, const int32_t* sel, float* out, float* lse, 
 int launch_select_attend(const Problem& p, const float* block_scores, int32_t* sel_out, float* out, float* lse,
                          bool pdl, cudaStream_t st);
 
+// Sparse attention for chunked prefill (attend_prefill.cu): block-major tensor-core tiles.
+// Used by msa_decode when attend_prefill_supported(p) (Tq * HI > 32, Hq / Hkv = 8); its
+// workspace (selection inversion lists and per-slot partials) follows msa_decode's own.
+bool attend_prefill_supported(const Problem& p);
+size_t attend_prefill_ws_bytes(const Problem& p);
+int launch_attend_prefill(const Problem& p, const int32_t* sel, void* ws, float* out, float* lse, bool pdl,
+                          cudaStream_t st);
+// cuTensorMapEncodeTiled from the driver (nullptr if unavailable), looked up once.
+void* tensor_map_encode_entry();
+
 // Context-parallel decode (dcp.cu).  Candidates: this rank's best 15 blocks of [blk_lo,
 // blk_hi) per row, from block scores written by the range indexer; merge: G ranks'
 // candidates -> the selection; combine: G attention partials -> the output.

@@ -180,7 +180,7 @@ int msa_nvfp4_amax(const float* x, int64_t n, float* amax_out, cudaStream_t stre
 
 size_t msa_workspace_size(const msa_params_t* p) {
     if (check_params(p, true, true) != MSA_OK) return 0;
-    return ws_block_scores_bytes(p) + ws_sel_bytes(p);
+    return ws_block_scores_bytes(p) + ws_sel_bytes(p) + attend_prefill_ws_bytes(to_problem(p));
 }
 
 size_t msa_workspace_size_single_launch(const msa_params_t* p) {
@@ -215,13 +215,19 @@ int msa_decode(const msa_params_t* p, void* ws, size_t ws_bytes, void* out_, flo
     if (int r = check_params(p, true, true)) return r;
     if (!out) return MSA_EINVAL;
     if (!aligned16(out)) return MSA_EALIGN;
-    const size_t need = ws_block_scores_bytes(p) + ws_sel_bytes(p);
+    const Problem q = to_problem(p);
+    const size_t need = ws_block_scores_bytes(p) + ws_sel_bytes(p) + attend_prefill_ws_bytes(q);
     if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return MSA_EWORKSPACE;
     float* bs = static_cast<float*>(ws);
     int32_t* sel = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + ws_block_scores_bytes(p));
-    const Problem q = to_problem(p);
     const bool pdl = pdl_enabled();
     if (int r = launch_index(q, bs, nullptr, pdl, stream)) return r;
+    // chunked prefill: block-major tensor-core attention over the inverted selection
+    if (attend_prefill_supported(q)) {
+        if (int r = launch_select(q, bs, sel, sel_out, pdl, stream)) return r;
+        void* ws_ap = static_cast<uint8_t*>(ws) + ws_block_scores_bytes(p) + ws_sel_bytes(p);
+        return launch_attend_prefill(q, sel, ws_ap, out, lse, pdl, stream);
+    }
     // short rows: each attention CTA selects its own row's blocks (one launch fewer)
     if (q.nbmax <= 1024) return launch_select_attend(q, bs, sel_out, out, lse, pdl, stream);
     if (int r = launch_select(q, bs, sel, sel_out, pdl, stream)) return r;

@@ -35,6 +35,8 @@ def _custom(B, Tq, Hq, Hkv, HI, DI, lens, lmax, weights=False, seed=7):
 
 CASES = {
     "tq256_hi8_di128": lambda: _custom(2, 256, 32, 4, 8, 128, [2560, 1500], 2560),
+    # blocks chosen by more than 16 tokens (several tiles per block), ragged lengths
+    "tq1024_hi4_many_tiles": lambda: _custom(2, 1024, 16, 2, 4, 64, [3300, 1030], 3328),
     "tq100_hi4_di64_partial_tile": lambda: _custom(1, 100, 8, 1, 4, 64, [3000], 3072),
     "tq40_hi2_weights_ragged": lambda: _custom(3, 40, 16, 2, 2, 128, [5000, 40, 777], 5120, weights=True),
     "tq33_hi1_di64": lambda: _custom(2, 33, 8, 8, 1, 64, [129, 4100], 4224),
@@ -71,8 +73,15 @@ def test_prefill_index_select_attend(case):
     o, l = oracle.attend(bf16_values(inp.q), k, v, sel.cpu().numpy(), inp.seq_lens)
     check_attention(out.cpu().numpy(), o)
     np.testing.assert_allclose(lse.cpu().numpy(), l, rtol=1e-4, atol=1e-4)
+    # msa_decode: block-major tensor-core attention when Hq / Hkv = 8, else the gather kernel
     d = run_decode(p)
+    assert int(p.status.item()) == 0
     assert np.array_equal(d["sel"], sel.cpu().numpy())
+    check_attention(d["out"], o)
+    np.testing.assert_allclose(d["lse"], l, rtol=1e-4, atol=1e-4)
+    d2 = run_decode(p)
+    assert np.array_equal(d2["out"].view(np.uint32), d["out"].view(np.uint32))  # bitwise reproducible
+    assert np.array_equal(d2["lse"].view(np.uint32), d["lse"].view(np.uint32))
 
 
 def test_prefill_rejects_max_pooling_and_token_scores():
