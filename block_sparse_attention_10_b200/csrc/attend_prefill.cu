@@ -12,13 +12,16 @@
 // of them, so this file turns the work around and goes block by block:
 //   1. ap_count / ap_scan / ap_fill invert the selection: for every (sequence, block) the
 //      list of (token, slot) pairs that selected it (slot = its place in the token's 16);
+//      ap_tiles writes one record per tile (item, list offset, tokens, sequence length);
 //   2. ap_attend_kernel: one persistent CTA per SM walks items (sequence, KV head, block)
 //      cut into tiles of 16 listed tokens x 8 query heads = 128 rows, the tiles spread
 //      evenly over the CTAs.  Per item the 4 compute warps dequantise the block once: K as
 //      bf16 [128 keys x 128 dims] and V transposed as f16 [128 dims x 128 keys], both in the
 //      K-major 128-byte-swizzle layout the tensor cores read (e2m1 x e4m3 is exact in both
 //      types); one warp streams the raw block (bulk copies) and each tile's query rows
-//      (TMA, 128-byte swizzle, one 8-row atom per token, no multicast); one thread issues
+//      (TMA from 16 lanes, 128-byte swizzle, one 8-row atom per token, L2 evict-last, no
+//      multicast), prefetching the records and token ids of the next tiles and publishing
+//      each tile's record in a 4-slot shared-memory ring for the other warps; one thread issues
 //        S = Q K^T   tcgen05.mma kind::f16, bf16, 128 x 128 x 128, fp32 in TMEM,
 //        O = P V     tcgen05.mma kind::f16, f16,  128 x 128 x 128, fp32 in TMEM,
 //      with S and O double-buffered (4 x 128 TMEM columns) so that the softmax of one tile
@@ -55,8 +58,9 @@ constexpr int kOffQ = 2 * kApTile;     // 2 query stages
 constexpr int kOffP = 4 * kApTile;     // 2 P buffers, f16 [row][key]
 constexpr int kOffRaw = 6 * kApTile;   // the raw NVFP4 block: K nibbles, K scales, V nibbles, V scales
 constexpr int kRawK = 0, kRawKs = 8192, kRawV = 9216, kRawVs = 17408, kRawBytes = 18432;
-constexpr int kOffBar = kOffRaw + kRawBytes;
-constexpr size_t kApSmem = 1024 + kOffBar + 256;
+constexpr int kOffBar = kOffRaw + kRawBytes;  // 29 mbarriers + the TMEM address
+constexpr int kOffInfo = kOffBar + 256;       // 4 tile records
+constexpr size_t kApSmem = 1024 + kOffInfo + 4 * 96;
 constexpr uint32_t kApTmemCols = 512;  // S at columns 0 / 128, O at 256 / 384
 constexpr float kApLog2e = 1.4426950408889634f;
 constexpr float kApLn2 = 0.6931471805599453f;
@@ -68,6 +72,7 @@ struct ApWork {
     int32_t* list_off;          // [B * nbmax] start of each list
     int32_t* tile_start;        // [items + 1] first tile of item (b, kvh, n); last entry = total
     int32_t* list;              // [B * Tq * 16] entries t * 16 + slot, grouped by (b, n)
+    int4* tiles;                // [B * Tq * 16 * Hkv] per tile: item, list offset, tokens, clamped L
     float* part_lse;            // [B][Tq][16][Hq]
     __half* part_o;             // [B][Tq][16][Hq][D]
 };
@@ -161,25 +166,47 @@ __global__ void ap_fill_kernel(const Problem p, const ApWork w) {
     }
 }
 
+// One thread per item (b, kvh, n): its tiles' entries in the tile table, so that the
+// attention kernel reads one 16-byte record per tile instead of walking the prefix sums.
+__global__ void ap_tiles_kernel(const Problem p, const ApWork w) {
+    pdl_wait();
+    pdl_launch_dependents();
+    const int64_t item = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (item >= (int64_t)p.B * p.Hkv * p.nbmax) return;
+    const int64_t n = item % p.nbmax, b = item / (p.nbmax * p.Hkv);
+    const int64_t ln = b * p.nbmax + n;
+    const int cnt = w.cnt[ln], off = w.list_off[ln], t0 = w.tile_start[item];
+    const int L = (int)clamp_len(p.seq_lens[b], p.Tq, p.lmax, nullptr);
+    for (int j = 0; j * kApTok < cnt; ++j)
+        w.tiles[t0 + j] = make_int4((int)item, off + j * kApTok, min(kApTok, cnt - j * kApTok), L);
+}
+
 // ------------------------------------------------------------------ block-major attention
 
-// The CTA's walk over its tiles: item = (b * Hkv + kvh) * nbmax + n, tiles
-// [tile_start[item], tile_start[item + 1]).
-struct ApWalk {
-    int64_t item;
-    __device__ __forceinline__ void seek(const int32_t* ts, int64_t items, int tau) {
-        int64_t lo = 0, hi = items;  // ts[0] = 0 <= tau < ts[items]
-        while (hi - lo > 1) {
-            const int64_t mid = (lo + hi) >> 1;
-            if (ts[mid] <= tau) lo = mid;
-            else hi = mid;
-        }
-        item = lo;
-    }
-    __device__ __forceinline__ void advance(const int32_t* ts, int tau) {
-        while (ts[item + 1] <= tau) ++item;
-    }
+// One tile as the producer warp publishes it to the MMA thread and the compute warps.
+struct ApTileInfo {
+    int32_t item, b, kvh, n, ntok, L;
+    int32_t pad[2];
+    int32_t entry[kApTok];  // t * 16 + slot of the tile's tokens
 };
+constexpr int kApInfoSlots = 4;
+static_assert(sizeof(ApTileInfo) == 96, "tile record layout");
+
+// TMA load of a 4-D box with an L2 eviction-priority hint (no multicast).
+__device__ __forceinline__ void tma_load_4d_hint(void* dst, const void* tmap, int c0, int c1, int c2, int c3,
+                                                 uint64_t* bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], "
+        "[%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(smem_u32(dst)),
+        "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
 
 __device__ __forceinline__ uint32_t f16x2_to_bf16x2(uint32_t h) {
     const __half2 v = *reinterpret_cast<const __half2*>(&h);
@@ -262,16 +289,19 @@ __global__ void __launch_bounds__(kApThreads, 1)
     uint64_t* raw_empty = bar + 1;
     uint64_t* kv_full = bar + 2;
     uint64_t* kv_empty = bar + 3;
-    uint64_t* q_full = bar + 4;    // [2]
-    uint64_t* q_empty = bar + 6;   // [2]
-    uint64_t* s_full = bar + 8;    // [2]
-    uint64_t* s_empty = bar + 10;  // [2]
-    uint64_t* p_full = bar + 12;   // [2]
-    uint64_t* p_empty = bar + 14;  // [2]
-    uint64_t* o_full = bar + 16;   // [2]
-    uint64_t* o_empty = bar + 18;  // [2]
-    uint64_t* done = bar + 20;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 21);
+    uint64_t* q_full = bar + 4;       // [2]
+    uint64_t* q_empty = bar + 6;      // [2]
+    uint64_t* s_full = bar + 8;       // [2]
+    uint64_t* s_empty = bar + 10;     // [2]
+    uint64_t* p_full = bar + 12;      // [2]
+    uint64_t* p_empty = bar + 14;     // [2]
+    uint64_t* o_full = bar + 16;      // [2]
+    uint64_t* o_empty = bar + 18;     // [2]
+    uint64_t* info_full = bar + 20;   // [4]
+    uint64_t* info_empty = bar + 24;  // [4]
+    uint64_t* done = bar + 28;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 29);
+    ApTileInfo* info = reinterpret_cast<ApTileInfo*>(smem + kOffInfo);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     pdl_wait();
@@ -289,6 +319,10 @@ __global__ void __launch_bounds__(kApThreads, 1)
             mbar_init(&p_empty[s], 1);
             mbar_init(&o_full[s], 1);
             mbar_init(&o_empty[s], kApComputeWarps);
+        }
+        for (int s = 0; s < kApInfoSlots; ++s) {
+            mbar_init(&info_full[s], 1);
+            mbar_init(&info_empty[s], kApComputeWarps + 1);  // the compute warps and the MMA thread
         }
         mbar_init(done, 1);
         fence_mbar_init();
@@ -311,59 +345,85 @@ __global__ void __launch_bounds__(kApThreads, 1)
     auto fail = [&]() { set_status(p.status, MSA_STATUS_TIMEOUT | MSA_STATUS_AT_ATTEND); };
 
     if (warp == kApTmaWarp) {
-        // ------------------------------------------------------------ producer: raw blocks, query tiles
-        if (lane == 0 && t0 < t1) {
-            ApWalk wk;
-            wk.seek(w.tile_start, items, t0);
-            int64_t cur = -1;
-            int it = -1, issued = 0;
+        // ------------------------------------------------------------ producer warp: tile records, raw blocks,
+        // query rows.  The tile record of tile tau + 2 and the token ids of tile tau + 1 are loaded while
+        // tile tau is issued, so no global-load latency sits between two tiles.
+        if (t0 < t1) {
+            const uint64_t pol = l2_policy_evict_last();  // the queries are re-read by many tiles
+            int4 m0 = w.tiles[t0];
+            int4 m1 = t0 + 1 < t1 ? w.tiles[t0 + 1] : make_int4(0, 0, 0, 0);
+            int e0 = lane < m0.z ? w.list[m0.y + lane] : 0;
+            int cur = -1, it = -1, issued = 0;
             bool ok = true;
             for (int tau = t0; tau < t1 && ok; ++tau) {
-                const int i = tau - t0, sb = i & 1;
-                wk.advance(w.tile_start, tau);
-                const int64_t n = wk.item % p.nbmax, bk = wk.item / p.nbmax;
-                const int kvh = (int)(bk % p.Hkv), b = (int)(bk / p.Hkv);
-                if (wk.item != cur) {
-                    cur = wk.item;
+                const int i = tau - t0, sb = i & 1, s4 = i & (kApInfoSlots - 1);
+                // prefetch: token ids of the next tile, record of the one after
+                const int e1 = (tau + 1 < t1 && lane < m1.z) ? w.list[m1.y + lane] : 0;
+                const int4 m2 = tau + 2 < t1 ? w.tiles[tau + 2] : make_int4(0, 0, 0, 0);
+                const int item = m0.x, ntok = m0.z;
+                const int n = item % (int)p.nbmax, bk = item / (int)p.nbmax;
+                const int kvh = bk % p.Hkv, b = bk / p.Hkv;
+                if (item != cur) {
+                    cur = item;
                     ++it;
-                    if (it >= 1 && !mbar_wait(raw_empty, (it - 1) & 1)) {
-                        fail();
-                        ok = false;
-                        break;
+                    if (lane == 0) {
+                        if (it >= 1 && !mbar_wait(raw_empty, (it - 1) & 1)) ok = false;
+                        if (ok) {
+                            const int64_t vec = block_vec<PAGED>(p, b, n, kvh, p.Hkv);
+                            uint8_t* raw = smem + kOffRaw;
+                            mbar_arrive_expect_tx(raw_full, 2 * (8192 + 1024));
+                            bulk_g2s(raw + kRawK, p.k.data + vec * 64, 8192, raw_full);
+                            bulk_g2s(raw + kRawKs, p.k.scale + vec * 8, 1024, raw_full);
+                            bulk_g2s(raw + kRawV, p.v.data + vec * 64, 8192, raw_full);
+                            bulk_g2s(raw + kRawVs, p.v.scale + vec * 8, 1024, raw_full);
+                        }
                     }
-                    const int64_t vec = block_vec<PAGED>(p, b, n, kvh, p.Hkv);
-                    uint8_t* raw = smem + kOffRaw;
-                    mbar_arrive_expect_tx(raw_full, 2 * (8192 + 1024));
-                    bulk_g2s(raw + kRawK, p.k.data + vec * 64, 8192, raw_full);
-                    bulk_g2s(raw + kRawKs, p.k.scale + vec * 8, 1024, raw_full);
-                    bulk_g2s(raw + kRawV, p.v.data + vec * 64, 8192, raw_full);
-                    bulk_g2s(raw + kRawVs, p.v.scale + vec * 8, 1024, raw_full);
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (!ok) break;
                 }
-                const int64_t ln = (int64_t)b * p.nbmax + n;
-                const int j = tau - w.tile_start[wk.item];
-                const int ntok = min(kApTok, w.cnt[ln] - j * kApTok);
-                if (i >= 2 && !mbar_wait(&q_empty[sb], ((i >> 1) - 1) & 1)) {
-                    fail();
-                    ok = false;
-                    break;
+                if (lane == 0) {
+                    if (i >= kApInfoSlots && !mbar_wait(&info_empty[s4], ((i >> 2) - 1) & 1)) ok = false;
+                    if (ok && i >= 2 && !mbar_wait(&q_empty[sb], ((i >> 1) - 1) & 1)) ok = false;
                 }
-                mbar_arrive_expect_tx(&q_full[sb], (uint32_t)(ntok * 2 * 1024));
-                const int32_t* lst = w.list + w.list_off[ln] + j * kApTok;
-                uint8_t* qs = smem + kOffQ + sb * kApTile;
-                for (int k = 0; k < ntok; ++k) {
-                    const int t = lst[k] / kTopK;
-                    tma_load_4d(qs + k * 1024, &tmap, 0, kvh * kApG, t, b, &q_full[sb]);
-                    tma_load_4d(qs + kApKB + k * 1024, &tmap, 64, kvh * kApG, t, b, &q_full[sb]);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                // publish the tile record
+                if (lane < kApTok) info[s4].entry[lane] = e0;
+                if (lane == 0) {
+                    info[s4].item = item;
+                    info[s4].b = b;
+                    info[s4].kvh = kvh;
+                    info[s4].n = n;
+                    info[s4].ntok = ntok;
+                    info[s4].L = m0.w;
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(&info_full[s4]);
+                    mbar_arrive_expect_tx(&q_full[sb], (uint32_t)(ntok * 2 * 1024));
+                }
+                __syncwarp();
+                if (lane < ntok) {  // each lane gathers one token's 8 query heads
+                    const int t = e0 / kTopK;
+                    uint8_t* qs = smem + kOffQ + sb * kApTile + lane * 1024;
+                    tma_load_4d_hint(qs, &tmap, 0, kvh * kApG, t, b, &q_full[sb], pol);
+                    tma_load_4d_hint(qs + kApKB, &tmap, 64, kvh * kApG, t, b, &q_full[sb], pol);
                 }
                 issued = i + 1;
+                m0 = m1;
+                m1 = m2;
+                e0 = e1;
             }
+            if (!ok && lane == 0) fail();
             // never leave with copies in flight into this CTA's shared memory
-            for (int i = max(0, issued - 2); i < issued; ++i)
-                if (!mbar_wait(&q_full[i & 1], (i >> 1) & 1)) {
-                    fail();
-                    break;
-                }
-            if (it >= 0 && !mbar_wait(raw_full, it & 1)) fail();
+            if (lane == 0) {
+                for (int i = max(0, issued - 2); i < issued; ++i)
+                    if (!mbar_wait(&q_full[i & 1], (i >> 1) & 1)) {
+                        fail();
+                        break;
+                    }
+                if (it >= 0 && !mbar_wait(raw_full, it & 1)) fail();
+            }
         }
     } else if (warp == kApMmaWarp) {
         // ------------------------------------------------------------ MMA issuer (one thread)
@@ -385,22 +445,24 @@ __global__ void __launch_bounds__(kApThreads, 1)
                 umma_commit(&o_full[sb]);
                 return true;
             };
-            ApWalk wk;
-            wk.seek(w.tile_start, items, t0);
-            int64_t cur = -1;
-            int it = -1;
+            int cur = -1, it = -1;
             bool ok = true, pending = false;
             for (int tau = t0; tau < t1 && ok; ++tau) {
-                const int i = tau - t0, sb = i & 1;
-                wk.advance(w.tile_start, tau);
-                if (wk.item != cur) {
+                const int i = tau - t0, sb = i & 1, s4 = i & (kApInfoSlots - 1);
+                if (!mbar_wait(&info_full[s4], (i >> 2) & 1)) {
+                    ok = false;
+                    break;
+                }
+                const int item = info[s4].item;
+                mbar_arrive(&info_empty[s4]);
+                if (item != cur) {
                     if (pending && !pv(i - 1)) {
                         ok = false;
                         break;
                     }
                     pending = false;
                     if (it >= 0) umma_commit(kv_empty);  // every MMA reading this item's K and V
-                    cur = wk.item;
+                    cur = item;
                     ++it;
                     if (!mbar_wait(kv_full, it & 1)) {
                         ok = false;
@@ -458,38 +520,41 @@ __global__ void __launch_bounds__(kApThreads, 1)
                     uint4* dst = reinterpret_cast<uint4*>(w.part_o + orow * 128 + c4 * 32);
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
-                        dst[q] = make_uint4(pack_f16x2(o[8 * q] * inv, o[8 * q + 1] * inv),
-                                            pack_f16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
-                                            pack_f16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv),
-                                            pack_f16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
+                        __stcs(dst + q, make_uint4(pack_f16x2(o[8 * q] * inv, o[8 * q + 1] * inv),
+                                                   pack_f16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
+                                                   pack_f16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv),
+                                                   pack_f16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv)));
                 }
             }
             tcgen05_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&o_empty[sb]);
-            if (orow >= 0) w.part_lse[orow] = (mc + log2f(l)) * kApLn2;
+            if (orow >= 0) __stcs(w.part_lse + orow, (mc + log2f(l)) * kApLn2);
             return true;
         };
         bool ok = true;
         if (t0 < t1) {
-            ApWalk wk;
-            wk.seek(w.tile_start, items, t0);
-            int64_t cur = -1;
-            int it = -1;
+            int cur = -1, it = -1;
             for (int tau = t0; tau < t1; ++tau) {
-                const int i = tau - t0, sb = i & 1;
-                wk.advance(w.tile_start, tau);
-                const int64_t n = wk.item % p.nbmax, bk = wk.item / p.nbmax;
-                const int kvh = (int)(bk % p.Hkv), b = (int)(bk / p.Hkv);
-                const int64_t L = clamp_len(p.seq_lens[b], Tq, p.lmax, nullptr);
-                if (wk.item != cur) {
-                    cur = wk.item;
+                const int i = tau - t0, sb = i & 1, s4 = i & (kApInfoSlots - 1);
+                if (!wait_all(&info_full[s4], (i >> 2) & 1)) {
+                    ok = false;
+                    break;
+                }
+                const ApTileInfo& ti = info[s4];
+                const int item = ti.item, n = ti.n, b = ti.b, kvh = ti.kvh, ntok = ti.ntok;
+                const int64_t L = ti.L;
+                const int e = tslot < ntok ? ti.entry[tslot] : 0;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&info_empty[s4]);
+                if (item != cur) {
+                    cur = item;
                     ++it;
                     if (!wait_all(raw_full, it & 1) || (it >= 1 && !wait_all(kv_empty, (it - 1) & 1))) {
                         ok = false;
                         break;
                     }
-                    ap_dequant(smem, n * kBlock, L, row);
+                    ap_dequant(smem, (int64_t)n * kBlock, L, row);
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
@@ -498,15 +563,11 @@ __global__ void __launch_bounds__(kApThreads, 1)
                     }
                 }
                 // ---- softmax of tile i
-                const int64_t ln = (int64_t)b * p.nbmax + n;
-                const int j = tau - w.tile_start[wk.item];
-                const int ntok = min(kApTok, w.cnt[ln] - j * kApTok);
                 int kvis = 0;
                 int64_t orow = -1;
                 if (tslot < ntok) {
-                    const int e = w.list[w.list_off[ln] + j * kApTok + tslot];
                     const int t = e / kTopK, slot = e % kTopK;
-                    kvis = (int)min64(kBlock, L - Tq + t - n * kBlock + 1);
+                    kvis = (int)min64(kBlock, L - Tq + t - (int64_t)n * kBlock + 1);
                     orow = (((int64_t)b * Tq + t) * kTopK + slot) * p.Hq + kvh * kApG + hq;
                 }
                 if (!wait_all(&s_full[sb], (i >> 1) & 1)) {
@@ -572,7 +633,8 @@ __global__ void __launch_bounds__(kApThreads, 1)
 
 // ------------------------------------------------------------------ merge of the slot partials
 
-// One thread per (sequence, token, query head, 8 dims).
+// One thread per (sequence, token, query head, 8 dims).  All of the row's slot partials are
+// requested before any is combined (they are read once: streaming loads).
 __global__ void __launch_bounds__(256) ap_merge_kernel(const Problem p, const ApWork w, float* __restrict__ out,
                                                        float* __restrict__ lse) {
     pdl_wait();
@@ -587,12 +649,25 @@ __global__ void __launch_bounds__(256) ap_merge_kernel(const Problem p, const Ap
     const int b = (int)(bt / p.Tq), t = (int)(bt % p.Tq);
     const int64_t L = clamp_len(p.seq_lens[b], p.Tq, p.lmax, nullptr);
     const int64_t nvis = (L - p.Tq + t) / kBlock + 1;
+    const int4* selv = reinterpret_cast<const int4*>(w.sel + bt * kTopK);
+    int ids[kTopK];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int4 x = __ldg(selv + q);
+        ids[4 * q] = x.x;
+        ids[4 * q + 1] = x.y;
+        ids[4 * q + 2] = x.z;
+        ids[4 * q + 3] = x.w;
+    }
     float ls[kTopK];
+    uint4 ov[kTopK];
     float M = -INFINITY;
 #pragma unroll
     for (int s = 0; s < kTopK; ++s) {
-        const int n = w.sel[bt * kTopK + s];
-        ls[s] = (n >= 0 && n < nvis) ? w.part_lse[(bt * kTopK + s) * p.Hq + hq] : -INFINITY;
+        const bool valid = ids[s] >= 0 && ids[s] < nvis;
+        const int64_t r = (bt * kTopK + s) * p.Hq + hq;
+        ls[s] = valid ? __ldcs(w.part_lse + r) : -INFINITY;
+        ov[s] = valid ? __ldcs(reinterpret_cast<const uint4*>(w.part_o + r * 128 + g8 * 8)) : make_uint4(0, 0, 0, 0);
         M = fmaxf(M, ls[s]);
     }
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -600,11 +675,9 @@ __global__ void __launch_bounds__(256) ap_merge_kernel(const Problem p, const Ap
     if (M != -INFINITY) {
 #pragma unroll
         for (int s = 0; s < kTopK; ++s) {
-            if (ls[s] == -INFINITY) continue;
-            const float wt = expf(ls[s] - M);
+            const float wt = ls[s] == -INFINITY ? 0.0f : expf(ls[s] - M);
             W += wt;
-            const uint4 v = *reinterpret_cast<const uint4*>(w.part_o + ((bt * kTopK + s) * p.Hq + hq) * 128 + g8 * 8);
-            const uint32_t vv[4] = {v.x, v.y, v.z, v.w};
+            const uint32_t vv[4] = {ov[s].x, ov[s].y, ov[s].z, ov[s].w};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&vv[q]));
@@ -626,7 +699,7 @@ constexpr size_t kApAlign = 256;
 size_t ap_round(size_t x) { return (x + kApAlign - 1) / kApAlign * kApAlign; }
 
 struct ApLayout {
-    size_t cnt, cursor, off, tstart, list, lse, po, total;
+    size_t cnt, cursor, off, tstart, list, tiles, lse, po, total;
 };
 
 ApLayout ap_layout(const Problem& p) {
@@ -643,6 +716,8 @@ ApLayout ap_layout(const Problem& p) {
     at += ap_round((items + 1) * 4);
     a.list = at;
     at += ap_round(entries * 4);
+    a.tiles = at;
+    at += ap_round(entries * p.Hkv * sizeof(int4));
     a.lse = at;
     at += ap_round(entries * p.Hq * 4);
     a.po = at;
@@ -697,7 +772,7 @@ int launch_ap_attend(const Problem& p, const ApWork& w, bool pdl, cudaStream_t s
 
 bool attend_prefill_supported(const Problem& p) {
     return (int64_t)p.Tq * p.HI > 32 && p.Hkv > 0 && p.Hq == kApG * p.Hkv && p.D == 128 &&
-           (int64_t)p.B * p.Tq * kTopK * p.Hkv < 0x7FFFFFFFll;
+           (int64_t)p.B * p.Tq * kTopK * p.Hkv < 0x7FFFFFFFll && (int64_t)p.B * p.Hkv * p.nbmax < 0x7FFFFFFFll;
 }
 
 size_t attend_prefill_ws_bytes(const Problem& p) { return attend_prefill_supported(p) ? ap_layout(p).total : 0; }
@@ -714,6 +789,7 @@ int launch_attend_prefill(const Problem& p, const int32_t* sel, void* ws, float*
     w.list_off = reinterpret_cast<int32_t*>(base + a.off);
     w.tile_start = reinterpret_cast<int32_t*>(base + a.tstart);
     w.list = reinterpret_cast<int32_t*>(base + a.list);
+    w.tiles = reinterpret_cast<int4*>(base + a.tiles);
     w.part_lse = reinterpret_cast<float*>(base + a.lse);
     w.part_o = reinterpret_cast<__half*>(base + a.po);
     const int64_t entries = (int64_t)p.B * p.Tq * kTopK;
@@ -726,6 +802,9 @@ int launch_attend_prefill(const Problem& p, const int32_t* sel, void* ws, float*
     if (cudaLaunchKernelEx(&cfg, ap_scan_kernel, p, w) != cudaSuccess) return MSA_ECUDA;
     cfg = ap_config(eg, dim3(256), 0, pdl, st, attr);
     if (cudaLaunchKernelEx(&cfg, ap_fill_kernel, p, w) != cudaSuccess) return MSA_ECUDA;
+    const int64_t items = (int64_t)p.B * p.Hkv * p.nbmax;
+    cfg = ap_config(dim3((unsigned)((items + 255) / 256)), dim3(256), 0, pdl, st, attr);
+    if (cudaLaunchKernelEx(&cfg, ap_tiles_kernel, p, w) != cudaSuccess) return MSA_ECUDA;
     const int r = p.block_table != nullptr ? launch_ap_attend<true>(p, w, pdl, st) : launch_ap_attend<false>(p, w, pdl, st);
     if (r != MSA_OK) return r;
     const int64_t threads = (int64_t)p.B * p.Tq * p.Hq * 16;

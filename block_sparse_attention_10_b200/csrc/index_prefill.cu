@@ -207,15 +207,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     } else {
         // ------------------------------------------------------------------ epilogue warps
         const int et = threadIdx.x;  // 0..255
-        // blocks past each sequence's length score -inf
-        {
-            const int64_t total = (int64_t)p.B * Tq * p.nbmax;
-            for (int64_t i = (int64_t)blockIdx.x * 256 + et; i < total; i += (int64_t)gridDim.x * 256) {
-                const int64_t n = i % p.nbmax;
-                const int b = (int)(i / (p.nbmax * Tq));
-                const int64_t L = clamp_len(p.seq_lens[b], Tq, p.lmax, blockIdx.x == 0 && i < 256 ? p.status : nullptr);
-                if (n >= (L + kBlock - 1) / kBlock) block_scores[i] = -INFINITY;
-            }
+        // blocks past each sequence's length score -inf: one (sequence, token) row per thread
+        // of the grid, each writing only its row's blocks past the sequence's length
+        for (int64_t r = (int64_t)blockIdx.x * 256 + et; r < (int64_t)p.B * Tq; r += (int64_t)gridDim.x * 256) {
+            const int b = (int)(r / Tq);
+            const int64_t L = clamp_len(p.seq_lens[b], Tq, p.lmax, r % Tq == 0 ? p.status : nullptr);
+            for (int64_t n = (L + kBlock - 1) / kBlock; n < p.nbmax; ++n) block_scores[r * p.nbmax + n] = -INFINITY;
         }
         const int quad = warp & 3, hb = warp >> 2;
         uint32_t qi = 0;
@@ -279,23 +276,27 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     }
                     tcgen05_fence_after();
                     const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * kPfKeys + hb * kBlock);
-                    // ReLU-sum over the visible columns: 4 independent packed accumulators
+                    // ReLU-sum over the visible columns: the block's 128 columns in one round trip
+                    // to tensor memory (four loads, one wait), 4 independent packed accumulators
                     float2 acc2[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+                    float v[kBlock / 32][32];
+#pragma unroll
+                    for (int c4 = 0; c4 < kBlock / 32; ++c4) tmem_ld32(taddr + c4 * 32, v[c4]);
+                    tmem_wait_ld();
 #pragma unroll
                     for (int c4 = 0; c4 < kBlock / 32; ++c4) {
-                        float v[32];
-                        tmem_ld32(taddr + c4 * 32, v);
-                        tmem_wait_ld();
                         if (cnt >= (c4 + 1) * 32) {
 #pragma unroll
                             for (int i = 0; i < 16; ++i)
-                                acc2[i & 3] = add_f32x2(acc2[i & 3], make_float2(fmaxf(v[2 * i], 0.0f), fmaxf(v[2 * i + 1], 0.0f)));
+                                acc2[i & 3] = add_f32x2(acc2[i & 3], make_float2(fmaxf(v[c4][2 * i], 0.0f),
+                                                                                fmaxf(v[c4][2 * i + 1], 0.0f)));
                         } else {
 #pragma unroll
                             for (int i = 0; i < 16; ++i) {
                                 const int col = c4 * 32 + 2 * i;
-                                acc2[i & 3] = add_f32x2(acc2[i & 3], make_float2(col < cnt ? fmaxf(v[2 * i], 0.0f) : 0.0f,
-                                                                                col + 1 < cnt ? fmaxf(v[2 * i + 1], 0.0f) : 0.0f));
+                                acc2[i & 3] = add_f32x2(acc2[i & 3],
+                                                        make_float2(col < cnt ? fmaxf(v[c4][2 * i], 0.0f) : 0.0f,
+                                                                    col + 1 < cnt ? fmaxf(v[c4][2 * i + 1], 0.0f) : 0.0f));
                             }
                         }
                     }

@@ -32,6 +32,11 @@
  *   tensor_scale                    fp32 > 0, one per cache tensor.
  *   value = fp32(e2m1 * e4m3) * tensor_scale.   9/16 byte per element.
  *
+ * Interface notes: the device status word is a field of msa_params_t (every
+ * kernel reports through it), msa_decode also returns the log-sum-exp, and
+ * msa_attend needs no scratch (its split over the selected blocks is merged on
+ * chip).
+ *
  * Conventions for every entry point:
  *   - pointers are DEVICE pointers owned by the caller (except where stated);
  *     nothing is allocated, nothing is freed, the host never synchronises;
@@ -167,7 +172,11 @@ int msa_nvfp4_amax(const float* x, int64_t n, float* amax_out, cudaStream_t stre
  * MSA steps ("A model built for efficient inference", ainewsbites.com)
  * ------------------------------------------------------------------------- */
 
-/* Bytes of scratch msa_decode needs for this problem (0 on invalid params). */
+/* Bytes of scratch msa_decode needs for this problem (0 on invalid params): the pooled
+ * block scores and the selection; for chunked prefill (Tq * HI > 32) with Hq = 8 * Hkv
+ * also the per-block token lists and the per-(token, selected block) attention partials
+ * of the tensor-core prefill attention, B * Tq * 16 * Hq * (2 D + 4) bytes and more
+ * (about 1.07 GB for 2 sequences x 4,096 tokens x 32 heads). */
 size_t msa_workspace_size(const msa_params_t* p);
 
 /* Indexer + block pooling: streams every visible NVFP4 index key once.
@@ -194,7 +203,13 @@ int msa_attend(const msa_params_t* p, const int32_t* sel, void* out, float* lse,
 
 /* The whole MSA decode step: msa_index -> msa_select -> msa_attend (two
  * launches when the rows have <= 1,024 blocks: the selection then runs inside
- * the attention kernel).
+ * the attention kernel).  For chunked prefill (Tq * HI > 32) with Hq = 8 * Hkv
+ * the attention goes block by block on the tensor cores instead (the selection
+ * inverted into per-block token lists, each block dequantised once per KV head,
+ * tcgen05 tiles, the per-slot partials merged in slot order); results agree
+ * with msa_attend's within the attention tolerance and are bitwise
+ * reproducible.  Besides cudaMemsetAsync of a counter array in the workspace,
+ * that path enqueues seven kernels.
  *   ws, ws_bytes  device scratch of at least msa_workspace_size(p) bytes,
  *                 256-byte aligned; contents on entry are ignored
  *   out, lse      as for msa_attend
