@@ -15,18 +15,20 @@
 //      ap_tiles writes one record per tile (item, list offset, tokens, sequence length);
 //   2. ap_attend_kernel: one persistent CTA per SM walks items (sequence, KV head, block)
 //      cut into tiles of 16 listed tokens x 8 query heads = 128 rows, the tiles spread
-//      evenly over the CTAs.  Per item the 4 compute warps dequantise the block once: K as
+//      evenly over the CTAs.  Per item the 8 compute warps dequantise the block once: K as
 //      bf16 [128 keys x 128 dims] and V transposed as f16 [128 dims x 128 keys], both in the
 //      K-major 128-byte-swizzle layout the tensor cores read (e2m1 x e4m3 is exact in both
-//      types); one warp streams the raw block (bulk copies) and each tile's query rows
-//      (TMA from 16 lanes, 128-byte swizzle, one 8-row atom per token, L2 evict-last, no
-//      multicast), prefetching the records and token ids of the next tiles and publishing
+//      types); one warp streams the raw block (bulk copies, L2 evict-first) and each tile's
+//      query rows (16-byte cp.async from all 32 lanes into the 128-byte-swizzled layout, L2
+//      evict-last: a token's 8 heads are one 2 KB run of q; 1 KB TMA boxes were measured
+//      far slower), prefetching the records and token ids of the next tiles and publishing
 //      each tile's record in a 4-slot shared-memory ring for the other warps; one thread issues
 //        S = Q K^T   tcgen05.mma kind::f16, bf16, 128 x 128 x 128, fp32 in TMEM,
 //        O = P V     tcgen05.mma kind::f16, f16,  128 x 128 x 128, fp32 in TMEM,
 //      with S and O double-buffered (4 x 128 TMEM columns) so that the softmax of one tile
-//      overlaps the MMAs of the next; the compute warps (one TMEM lane = one row each) read
-//      S with tcgen05.ld, mask keys past the token's position, take the row max, write
+//      overlaps the MMAs of the next; the compute warps (two per TMEM lane quarter, each with
+//      64 of a row's 128 columns, exchanging the row's max and sum halves through shared
+//      memory) read S with tcgen05.ld, mask keys past the token's position, take the row max, write
 //      P = 2^(S c - m c) as f16 into shared memory for the second MMA, and finally write
 //      the row's output normalised by its own sum (f16, unscaled by the V tensor scale)
 //      and its log-sum-exp to the token's slot;
@@ -35,9 +37,6 @@
 // Every output row's arithmetic is independent of the tile row it occupies and the merge
 // order is fixed, so results are bitwise reproducible although the lists are filled with
 // atomics.  Every wait is bounded (MSA_STATUS_TIMEOUT | MSA_STATUS_AT_ATTEND).
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
 #include "internal.h"
 #include "tcgen05.cuh"
 
@@ -46,10 +45,10 @@ namespace {
 
 constexpr int kApG = 8;                // query heads per KV head on this path
 constexpr int kApTok = 128 / kApG;     // listed tokens per 128-row tile
-constexpr int kApComputeWarps = 4;
-constexpr int kApMmaWarp = 4;
-constexpr int kApTmaWarp = 5;
-constexpr int kApThreads = 32 * 6;
+constexpr int kApComputeWarps = 8;  // two per TMEM lane quarter, one per half of a row's 128 columns
+constexpr int kApMmaWarp = 8;
+constexpr int kApTmaWarp = 9;
+constexpr int kApThreads = 32 * 10;
 constexpr int kApTile = 32768;         // 128 rows x 128 16-bit elements: two 16 KB K-blocks
 constexpr int kApKB = 16384;           // one K-block (64 elements of 128 rows)
 constexpr int kOffK = 0;               // K, bf16 [key][dim]
@@ -58,9 +57,10 @@ constexpr int kOffQ = 2 * kApTile;     // 2 query stages
 constexpr int kOffP = 4 * kApTile;     // 2 P buffers, f16 [row][key]
 constexpr int kOffRaw = 6 * kApTile;   // the raw NVFP4 block: K nibbles, K scales, V nibbles, V scales
 constexpr int kRawK = 0, kRawKs = 8192, kRawV = 9216, kRawVs = 17408, kRawBytes = 18432;
-constexpr int kOffBar = kOffRaw + kRawBytes;  // 29 mbarriers + the TMEM address
-constexpr int kOffInfo = kOffBar + 256;       // 4 tile records
-constexpr size_t kApSmem = 1024 + kOffInfo + 4 * 96;
+constexpr int kOffBar = kOffRaw + kRawBytes;  // 37 mbarriers + the TMEM address
+constexpr int kOffInfo = kOffBar + 384;       // 4 tile records
+constexpr int kOffXch = kOffInfo + 4 * 96;    // row max / row sum halves exchanged by the two warps of a row
+constexpr size_t kApSmem = 1024 + kOffXch + 4 * 2 * 128 * 4;
 constexpr uint32_t kApTmemCols = 512;  // S at columns 0 / 128, O at 256 / 384
 constexpr float kApLog2e = 1.4426950408889634f;
 constexpr float kApLn2 = 0.6931471805599453f;
@@ -192,20 +192,38 @@ struct ApTileInfo {
 constexpr int kApInfoSlots = 4;
 static_assert(sizeof(ApTileInfo) == 96, "tile record layout");
 
-// TMA load of a 4-D box with an L2 eviction-priority hint (no multicast).
-__device__ __forceinline__ void tma_load_4d_hint(void* dst, const void* tmap, int c0, int c1, int c2, int c3,
-                                                 uint64_t* bar, uint64_t policy) {
-    asm volatile(
-        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], "
-        "[%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(smem_u32(dst)),
-        "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar)), "l"(policy)
-        : "memory");
-}
-
+// L2 eviction-priority policies: the queries are re-read by many tiles (keep them), the raw
+// cache blocks are read once per (block, KV head) (let them go first).
 __device__ __forceinline__ uint64_t l2_policy_evict_last() {
     uint64_t pol;
     asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
     return pol;
+}
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+
+// 16-byte asynchronous copy global -> shared (cache-global, L2 hint); completion is tracked by
+// ap_cp_async_arrive.
+__device__ __forceinline__ void ap_cp_async16(void* dst, const void* src, uint64_t pol) {
+    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
+                 "l"(pol)
+                 : "memory");
+}
+// Arrive on `bar` once this thread's earlier cp.async copies have landed (counted in the
+// barrier's initial arrival count).
+__device__ __forceinline__ void ap_cp_async_arrive(uint64_t* bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// Untiled bulk copy with an L2 hint (no multicast), completing `bytes` on `bar`.
+__device__ __forceinline__ void ap_bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar, uint64_t pol) {
+    asm volatile(
+        "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+        : "memory");
 }
 
 __device__ __forceinline__ uint32_t f16x2_to_bf16x2(uint32_t h) {
@@ -216,9 +234,12 @@ __device__ __forceinline__ uint32_t f16x2_to_bf16x2(uint32_t h) {
 
 // The raw NVFP4 block (keys kbase .. kbase + 127 of one KV head) -> K (bf16 [key][dim]) and
 // V^T (f16 [dim][key]), 128-byte swizzle, K-major; keys at or past L become zeros.
-__device__ __forceinline__ void ap_dequant(uint8_t* smem, int64_t kbase, int64_t L, int tid) {
+// Called by the 256 threads of the compute warps: threads 128..255 write K, threads 0..127 V^T.
+__device__ __forceinline__ void ap_dequant(uint8_t* smem, int64_t kbase, int64_t L, int tid256) {
     const uint8_t* raw = smem + kOffRaw;
     const int nvalid = (int)min64(kBlock, max64(0, L - kbase));
+    if (tid256 >= 128) {
+    const int tid = tid256 - 128;
     uint8_t* kt = smem + kOffK;
 #pragma unroll 4
     for (int k = 0; k < 16; ++k) {
@@ -237,6 +258,9 @@ __device__ __forceinline__ void ap_dequant(uint8_t* smem, int64_t kbase, int64_t
         o.w = f16x2_to_bf16x2(hmul2(h[3], s2));
         *reinterpret_cast<uint4*>(kt + (cr >> 3) * kApKB + j * 128 + (((cr & 7) ^ (j & 7)) << 4)) = o;
     }
+    return;
+    }
+    const int tid = tid256;
     // V^T: thread = (dims 16 w16 .. 16 w16 + 15, keys 8 kg .. 8 kg + 7) -> 16 rows x one 16-byte chunk
     uint8_t* vt = smem + kOffV;
     const int w16 = tid & 7, kg = tid >> 3;
@@ -281,7 +305,7 @@ __device__ __forceinline__ void ap_dequant(uint8_t* smem, int64_t kbase, int64_t
 
 template <bool PAGED>
 __global__ void __launch_bounds__(kApThreads, 1)
-    ap_attend_kernel(const Problem p, const ApWork w, const __grid_constant__ CUtensorMap tmap) {
+    ap_attend_kernel(const Problem p, const ApWork w) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kOffBar);
@@ -300,8 +324,11 @@ __global__ void __launch_bounds__(kApThreads, 1)
     uint64_t* info_full = bar + 20;   // [4]
     uint64_t* info_empty = bar + 24;  // [4]
     uint64_t* done = bar + 28;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 29);
+    uint64_t* pair = bar + 29;        // [4 lane quarters][2]: the two warps of a row met
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 37);
     ApTileInfo* info = reinterpret_cast<ApTileInfo*>(smem + kOffInfo);
+    float* xmax = reinterpret_cast<float*>(smem + kOffXch);  // [2 tile parities][2 halves][128 rows]
+    float* xsum = xmax + 2 * 2 * 128;                         // [2 tile parities][2 halves][128 rows]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     pdl_wait();
@@ -311,7 +338,7 @@ __global__ void __launch_bounds__(kApThreads, 1)
         mbar_init(kv_full, kApComputeWarps);
         mbar_init(kv_empty, 1);
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&q_full[s], 1);
+            mbar_init(&q_full[s], 32);  // one cp.async arrival per producer lane
             mbar_init(&q_empty[s], 1);
             mbar_init(&s_full[s], 1);
             mbar_init(&s_empty[s], kApComputeWarps);
@@ -325,6 +352,7 @@ __global__ void __launch_bounds__(kApThreads, 1)
             mbar_init(&info_empty[s], kApComputeWarps + 1);  // the compute warps and the MMA thread
         }
         mbar_init(done, 1);
+        for (int s = 0; s < 8; ++s) mbar_init(&pair[s], 2);
         fence_mbar_init();
     }
     if (warp == kApMmaWarp) {
@@ -349,7 +377,7 @@ __global__ void __launch_bounds__(kApThreads, 1)
         // query rows.  The tile record of tile tau + 2 and the token ids of tile tau + 1 are loaded while
         // tile tau is issued, so no global-load latency sits between two tiles.
         if (t0 < t1) {
-            const uint64_t pol = l2_policy_evict_last();  // the queries are re-read by many tiles
+            const uint64_t pol_q = l2_policy_evict_last(), pol_kv = l2_policy_evict_first();
             int4 m0 = w.tiles[t0];
             int4 m1 = t0 + 1 < t1 ? w.tiles[t0 + 1] : make_int4(0, 0, 0, 0);
             int e0 = lane < m0.z ? w.list[m0.y + lane] : 0;
@@ -372,10 +400,10 @@ __global__ void __launch_bounds__(kApThreads, 1)
                             const int64_t vec = block_vec<PAGED>(p, b, n, kvh, p.Hkv);
                             uint8_t* raw = smem + kOffRaw;
                             mbar_arrive_expect_tx(raw_full, 2 * (8192 + 1024));
-                            bulk_g2s(raw + kRawK, p.k.data + vec * 64, 8192, raw_full);
-                            bulk_g2s(raw + kRawKs, p.k.scale + vec * 8, 1024, raw_full);
-                            bulk_g2s(raw + kRawV, p.v.data + vec * 64, 8192, raw_full);
-                            bulk_g2s(raw + kRawVs, p.v.scale + vec * 8, 1024, raw_full);
+                            ap_bulk_g2s(raw + kRawK, p.k.data + vec * 64, 8192, raw_full, pol_kv);
+                            ap_bulk_g2s(raw + kRawKs, p.k.scale + vec * 8, 1024, raw_full, pol_kv);
+                            ap_bulk_g2s(raw + kRawV, p.v.data + vec * 64, 8192, raw_full, pol_kv);
+                            ap_bulk_g2s(raw + kRawVs, p.v.scale + vec * 8, 1024, raw_full, pol_kv);
                         }
                     }
                     ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -398,17 +426,19 @@ __global__ void __launch_bounds__(kApThreads, 1)
                     info[s4].L = m0.w;
                 }
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(&info_full[s4]);
-                    mbar_arrive_expect_tx(&q_full[sb], (uint32_t)(ntok * 2 * 1024));
+                if (lane == 0) mbar_arrive(&info_full[s4]);
+                // the tile's query rows: each token's 8 heads are 2 KB contiguous in q, copied by 4
+                // rounds of the warp's 32 lanes x 16 bytes into the 128-byte-swizzled K-major tile
+                uint8_t* qs = smem + kOffQ + sb * kApTile;
+                for (int k = 0; k < 4 * ntok; ++k) {
+                    const int t = __shfl_sync(0xffffffffu, e0, k >> 2) / kTopK;  // token slot k / 4
+                    const int hc = (k & 3) * 32 + lane, h = hc >> 4, c16 = hc & 15;
+                    const int rw = (k >> 2) * kApG + h;  // tile row
+                    const __nv_bfloat16* src =
+                        p.q + (((int64_t)b * Tq + t) * p.Hq + kvh * kApG + h) * 128 + c16 * 8;
+                    ap_cp_async16(qs + (c16 >> 3) * kApKB + rw * 128 + (((c16 & 7) ^ (rw & 7)) << 4), src, pol_q);
                 }
-                __syncwarp();
-                if (lane < ntok) {  // each lane gathers one token's 8 query heads
-                    const int t = e0 / kTopK;
-                    uint8_t* qs = smem + kOffQ + sb * kApTile + lane * 1024;
-                    tma_load_4d_hint(qs, &tmap, 0, kvh * kApG, t, b, &q_full[sb], pol);
-                    tma_load_4d_hint(qs + kApKB, &tmap, 64, kvh * kApG, t, b, &q_full[sb], pol);
-                }
+                ap_cp_async_arrive(&q_full[sb]);
                 issued = i + 1;
                 m0 = m1;
                 m1 = m2;
@@ -474,6 +504,7 @@ __global__ void __launch_bounds__(kApThreads, 1)
                     ok = false;
                     break;
                 }
+                fence_proxy_async_smem();  // the query rows were written by cp.async (generic proxy)
                 tcgen05_fence_after();
                 const uint32_t qa = smem_u32(smem + kOffQ + sb * kApTile);
 #pragma unroll
@@ -495,41 +526,56 @@ __global__ void __launch_bounds__(kApThreads, 1)
             if (!mbar_wait(done, 0)) fail();
         }
     } else {
-        // ------------------------------------------------------------ compute warps: dequant, softmax, output
-        const int row = threadIdx.x;  // TMEM lane and tile row: token slot row / 8, head row % 8
+        // ------------------------------------------------------------ compute warps: dequant, softmax, output.
+        // Warp w handles TMEM lanes (= tile rows) 32 (w % 4) .. + 31 and columns 64 (w / 4) .. + 63 of S,
+        // P and O; the two warps of a row exchange their halves' max and sum through shared memory,
+        // meeting on the pair mbarrier of their lane quarter (bounded waits, no unbounded named barrier).
+        const int qw = warp & 3, half = warp >> 2;
+        const int row = qw * 32 + lane;
         const int tslot = row >> 3, hq = row & 7;
-        const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+        const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16) + (uint32_t)(half * 64);
         const float c = p.softmax_scale * p.k.s_t * kApLog2e;
-        // the previous tile's row state, for its output step
         float prev_mc = 0.0f, prev_l = 0.0f;
         int64_t prev_row = -1;
         auto wait_all = [&](uint64_t* b_, uint32_t parity) -> bool {
             return __all_sync(0xffffffffu, mbar_wait(b_, parity)) != 0;
         };
-        auto output = [&](int i, float mc, float l, int64_t orow) -> bool {
+        // the two warps of this lane quarter meet (k-th meeting: parity k & 1 of pair[qw][k & 1] ... )
+        int meets = 0;
+        auto meet = [&]() -> bool {
+            uint64_t* pb = &pair[qw * 2 + (meets & 1)];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(pb);
+            const bool r = wait_all(pb, (uint32_t)((meets >> 1) & 1));
+            ++meets;
+            return r;
+        };
+        auto output = [&](int i, float mc, float lh, int64_t orow) -> bool {
             const int sb = i & 1;
             if (!wait_all(&o_full[sb], (i >> 1) & 1)) return false;
             tcgen05_fence_after();
+            const float l = lh + xsum[(sb * 2 + (half ^ 1)) * 128 + row];
             const float inv = l > 0.0f ? 1.0f / l : 0.0f;
+            float o[2][32];  // this half's 64 output columns in one round trip to tensor memory
 #pragma unroll
-            for (int c4 = 0; c4 < 4; ++c4) {
-                float o[32];
-                tmem_ld32(lane_base + 256 + sb * 128 + c4 * 32, o);
-                tmem_wait_ld();
-                if (orow >= 0) {
-                    uint4* dst = reinterpret_cast<uint4*>(w.part_o + orow * 128 + c4 * 32);
+            for (int c4 = 0; c4 < 2; ++c4) tmem_ld32(lane_base + 256 + sb * 128 + c4 * 32, o[c4]);
+            tmem_wait_ld();
+            if (orow >= 0) {
+                uint4* dst = reinterpret_cast<uint4*>(w.part_o + orow * 128 + half * 64);
+#pragma unroll
+                for (int c4 = 0; c4 < 2; ++c4)
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
-                        __stcs(dst + q, make_uint4(pack_f16x2(o[8 * q] * inv, o[8 * q + 1] * inv),
-                                                   pack_f16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
-                                                   pack_f16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv),
-                                                   pack_f16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv)));
-                }
+                        __stcs(dst + 4 * c4 + q,
+                               make_uint4(pack_f16x2(o[c4][8 * q] * inv, o[c4][8 * q + 1] * inv),
+                                          pack_f16x2(o[c4][8 * q + 2] * inv, o[c4][8 * q + 3] * inv),
+                                          pack_f16x2(o[c4][8 * q + 4] * inv, o[c4][8 * q + 5] * inv),
+                                          pack_f16x2(o[c4][8 * q + 6] * inv, o[c4][8 * q + 7] * inv)));
             }
             tcgen05_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&o_empty[sb]);
-            if (orow >= 0) __stcs(w.part_lse + orow, (mc + log2f(l)) * kApLn2);
+            if (orow >= 0 && half == 0) __stcs(w.part_lse + orow, (mc + log2f(l)) * kApLn2);
             return true;
         };
         bool ok = true;
@@ -554,7 +600,7 @@ __global__ void __launch_bounds__(kApThreads, 1)
                         ok = false;
                         break;
                     }
-                    ap_dequant(smem, (int64_t)n * kBlock, L, row);
+                    ap_dequant(smem, (int64_t)n * kBlock, L, threadIdx.x);
                     fence_proxy_async_smem();
                     __syncwarp();
                     if (lane == 0) {
@@ -562,50 +608,71 @@ __global__ void __launch_bounds__(kApThreads, 1)
                         mbar_arrive(kv_full);
                     }
                 }
-                // ---- softmax of tile i
-                int kvis = 0;
+                // ---- softmax of tile i (this warp's 64 columns of its 32 rows)
+                int kv_row = 0;  // visible keys of the row's block (0: no token in this tile row)
                 int64_t orow = -1;
                 if (tslot < ntok) {
                     const int t = e / kTopK, slot = e % kTopK;
-                    kvis = (int)min64(kBlock, L - Tq + t - (int64_t)n * kBlock + 1);
+                    kv_row = (int)min64(kBlock, L - Tq + t - (int64_t)n * kBlock + 1);
                     orow = (((int64_t)b * Tq + t) * kTopK + slot) * p.Hq + kvh * kApG + hq;
                 }
+                const int kvis = kv_row - half * 64;  // visible keys of this half (may be <= 0)
                 if (!wait_all(&s_full[sb], (i >> 1) & 1)) {
                     ok = false;
                     break;
                 }
                 tcgen05_fence_after();
-                float v[4][32];  // S row: key k in v[k / 32][k % 32]
+                float v[2][32];  // S: key 64 half + k in v[k / 32][k % 32]
 #pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) tmem_ld32(lane_base + sb * 128 + c4 * 32, v[c4]);
+                for (int c4 = 0; c4 < 2; ++c4) tmem_ld32(lane_base + sb * 128 + c4 * 32, v[c4]);
                 tmem_wait_ld();
                 tcgen05_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&s_empty[sb]);
-                float m = -INFINITY;
+                float mx[8];
+                if (__all_sync(0xffffffffu, kvis >= 64)) {
 #pragma unroll
-                for (int k = 0; k < 128; ++k)
-                    if (k < kvis) m = fmaxf(m, v[k >> 5][k & 31]);
-                const float mc = kvis > 0 ? m * c : 0.0f;
+                    for (int j = 0; j < 8; ++j) mx[j] = v[0][j];
+#pragma unroll
+                    for (int k = 8; k < 64; ++k) mx[k & 7] = fmaxf(mx[k & 7], v[k >> 5][k & 31]);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) mx[j] = -INFINITY;
+#pragma unroll
+                    for (int k = 0; k < 64; ++k)
+                        if (k < kvis) mx[k & 7] = fmaxf(mx[k & 7], v[k >> 5][k & 31]);
+                }
+                const float mh = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+                xmax[(sb * 2 + half) * 128 + row] = mh;
+                if (!meet()) {  // also publishes the partner's row sums of tile i - 1
+                    ok = false;
+                    break;
+                }
+                const float m = fmaxf(mh, xmax[(sb * 2 + (half ^ 1)) * 128 + row]);
+                const float mc = kv_row > 0 ? m * c : 0.0f;
                 if (i >= 2 && !wait_all(&p_empty[sb], ((i >> 1) - 1) & 1)) {
                     ok = false;
                     break;
                 }
-                uint8_t* prow = smem + kOffP + sb * kApTile + row * 128;
-                float l = 0.0f;
+                // P: this half's 64 keys are K-block `half` of the P tile
+                uint8_t* prow = smem + kOffP + sb * kApTile + half * kApKB + row * 128;
+                float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int cc = 0; cc < 16; ++cc) {
+                for (int cc = 0; cc < 8; ++cc) {
                     float e8[8];
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
                         const int k = cc * 8 + u;
                         e8[u] = k < kvis ? ex2_approx(fmaf(v[k >> 5][k & 31], c, -mc)) : 0.0f;
-                        l += e8[u];
+                        ls[u] += e8[u];
                     }
-                    *reinterpret_cast<uint4*>(prow + (cc >> 3) * kApKB + (((cc & 7) ^ (row & 7)) << 4)) =
+                    *reinterpret_cast<uint4*>(prow + ((cc ^ (row & 7)) << 4)) =
                         make_uint4(pack_f16x2(e8[0], e8[1]), pack_f16x2(e8[2], e8[3]), pack_f16x2(e8[4], e8[5]),
                                    pack_f16x2(e8[6], e8[7]));
                 }
+                const float lh = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+                xsum[(sb * 2 + half) * 128 + row] = lh;  // read by the partner in output(i), after the next meeting
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&p_full[sb]);
@@ -615,9 +682,11 @@ __global__ void __launch_bounds__(kApThreads, 1)
                     break;
                 }
                 prev_mc = mc;
-                prev_l = l;
+                prev_l = lh;
                 prev_row = orow;
             }
+            // the partner's row sums of the last tile: one more meeting
+            if (ok && !meet()) ok = false;
             if (ok && !output(t1 - t0 - 1, prev_mc, prev_l, prev_row)) ok = false;
             if (!ok && lane == 0) fail();
         }
@@ -742,18 +811,6 @@ cudaLaunchConfig_t ap_config(dim3 grid, dim3 block, size_t smem, bool pdl, cudaS
 
 template <bool PAGED>
 int launch_ap_attend(const Problem& p, const ApWork& w, bool pdl, cudaStream_t st) {
-    auto enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encode_entry());
-    if (enc == nullptr) return MSA_ECUDA;
-    // queries [B][Tq][Hq][128] bf16: boxes of 64 dims x 8 heads of one token, 128-byte swizzle
-    CUtensorMap tmap;
-    const cuuint64_t dims[4] = {128, (cuuint64_t)p.Hq, (cuuint64_t)p.Tq, (cuuint64_t)p.B};
-    const cuuint64_t strides[3] = {(cuuint64_t)128 * 2, (cuuint64_t)p.Hq * 128 * 2, (cuuint64_t)p.Tq * p.Hq * 128 * 2};
-    const cuuint32_t box[4] = {64, (cuuint32_t)kApG, 1, 1};
-    const cuuint32_t estr[4] = {1, 1, 1, 1};
-    if (enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<__nv_bfloat16*>(p.q), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return MSA_ECUDA;
     auto kern = ap_attend_kernel<PAGED>;
     static int configured_dev = -1;
     const DeviceInfo& di = device_info();
@@ -764,7 +821,7 @@ int launch_ap_attend(const Problem& p, const ApWork& w, bool pdl, cudaStream_t s
     }
     cudaLaunchAttribute attr[1];
     cudaLaunchConfig_t cfg = ap_config(dim3((unsigned)di.num_sms), dim3(kApThreads), kApSmem, pdl, st, attr);
-    if (cudaLaunchKernelEx(&cfg, kern, p, w, tmap) != cudaSuccess) return MSA_ECUDA;
+    if (cudaLaunchKernelEx(&cfg, kern, p, w) != cudaSuccess) return MSA_ECUDA;
     return MSA_OK;
 }
 

@@ -66,6 +66,29 @@ def test_simulated_ranks_match_oracle_and_decode(case, G):
     check_attention(out.cpu().numpy(), d["out"])
 
 
+@pytest.mark.parametrize("pool_mode,weights", [(1, False), (0, True), (1, True)])
+def test_simulated_ranks_max_pooling_and_head_weights(pool_mode, weights):
+    inp = _custom(2, 4, 16, 2, 4, 64, [20000, 3001], 20096, needles=5, seed=91)
+    if weights:
+        w = synth.Workload("dcpw", B=2, Tq=4, Hq=16, Hkv=2, D=128, HI=4, DI=64, seq_len=20000, lmax=20096,
+                           needles=5, seed=91, weights=True)
+        inp.w_idx = synth.queries(w, [0, 1])[2]
+    k, v, ik = oracle_caches(inp)
+    p = problem_from_inputs(inp)
+    p.pool_mode = pool_mode
+    d = run_decode(p)
+    out, lse, _ = msa.outputs(p)
+    sel = dcp.simulate_ranks(p, 3, out, lse)
+    torch.cuda.synchronize()
+    assert status_of(p) == 0
+    assert np.array_equal(sel.cpu().numpy(), d["sel"])
+    wts = None if inp.w_idx is None else inp.w_idx.numpy()
+    bs, _ = oracle.index(bf16_values(inp.q_idx), ik, inp.seq_lens, wts, pool_mode=pool_mode)
+    check_selection(sel.cpu().numpy(), oracle.select(bs, inp.seq_lens), bs, inp.seq_lens, inp.w.Tq)
+    o, _ = oracle.attend(bf16_values(inp.q), k, v, sel.cpu().numpy(), inp.seq_lens)
+    check_attention(out.cpu().numpy(), o)
+
+
 def test_bf16_combine(case):
     name, inp, ref = case
     p = problem_from_inputs(inp)
