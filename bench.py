@@ -535,8 +535,8 @@ def run_ours(args):
         assert int(p0.status.item()) == 0, f"device status word {int(p0.status.item()):#x}"
 
     # end to end through the public API, as a serving loop runs it: every step copies its queries
-    # from pinned host memory to the device (copy stream), runs msa_decode (compute stream) and
-    # copies the output back to pinned host memory (copy stream), where the host reads it.  The
+    # from pinned host memory to the device (upload stream), runs msa_decode (compute stream) and
+    # copies the output back to pinned host memory (download stream), where the host reads it.  The
     # copies of one step overlap the compute of another; events order every reuse of a buffer
     # (the replica's queries, the two device outputs, the two host outputs), and the host reads
     # step i - 1's output after enqueueing step i.
@@ -548,7 +548,7 @@ def run_ours(args):
     dout = [out, torch.empty_like(out)]
     hout = [torch.empty_like(out, device="cpu").pin_memory() for _ in range(2)]
     hout_np = [h.view(torch.int32).numpy() for h in hout]  # host views of the pinned outputs
-    copy_stream = torch.cuda.Stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()  # host->device and device->host copies
     ev_in = [torch.cuda.Event() for _ in range(2)]         # queries of step i on the device
     ev_done = [torch.cuda.Event() for _ in range(len(reps))]  # decode on replica r finished
     ev_out = [torch.cuda.Event() for _ in range(2)]        # output of step i on the host
@@ -557,22 +557,22 @@ def run_ours(args):
     def e2e_step(i):
         ri = i % len(reps)
         r, j = reps[ri], i % 2
-        if i >= len(reps):
-            copy_stream.wait_event(ev_done[ri])  # the replica's queries are free again
-        r.q.copy_(hq, non_blocking=True)
-        r.q_idx.copy_(hqi, non_blocking=True)
-        ev_in[j].record(copy_stream)
+        with torch.cuda.stream(up):
+            if i >= len(reps):
+                up.wait_event(ev_done[ri])  # the replica's queries are free again
+            r.q.copy_(hq, non_blocking=True)
+            r.q_idx.copy_(hqi, non_blocking=True)
+            ev_in[j].record(up)
         stream.wait_event(ev_in[j])
         if i >= 2:
             stream.wait_event(ev_out[j])  # device output j has been copied out
         msa.msa_decode(r, ws_t, dout[j], lse, None, stream=stream)
         ev_done[ri].record(stream)
-        copy_stream.wait_event(ev_done[ri])
-        hout[j].copy_(dout[j], non_blocking=True)
-        ev_out[j].record(copy_stream)
+        with torch.cuda.stream(down):
+            down.wait_event(ev_done[ri])
+            hout[j].copy_(dout[j], non_blocking=True)
+            ev_out[j].record(down)
 
-    prev_stream = torch.cuda.current_stream()
-    torch.cuda.set_stream(copy_stream)  # torch's copies go to the copy stream
     for i in range(3):  # warm-up of the host path
         e2e_step(i)
     torch.cuda.synchronize()
@@ -587,7 +587,6 @@ def run_ours(args):
     ev_out[(n_e2e - 1) % 2].synchronize()
     checksum ^= int(hout_np[(n_e2e - 1) % 2].flat[0])
     e2e_s = max_over_ranks((time.perf_counter() - t0) / n_e2e, dev)
-    torch.cuda.set_stream(prev_stream)
     torch.cuda.synchronize()
     h2d = hq.numel() * hq.element_size() + hqi.numel() * hqi.element_size()
     d2h = hout[0].numel() * hout[0].element_size()
@@ -620,9 +619,9 @@ def run_ours(args):
             "e2e": {"value": aggregate_throughput(w.B * w.Tq, ws_n, e2e_s), "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": n_e2e,
                     "how": "msa_decode through the Python API per step; every step copies its queries "
-                           "host->device and its output device->host (pinned) on a copy stream that overlaps "
-                           "the compute stream, events guarding buffer reuse; the host reads step i - 1's "
-                           "output after enqueueing step i"},
+                           "host->device and its output device->host (pinned) on an upload and a download "
+                           "stream that overlap the compute stream, events guarding buffer reuse; the host "
+                           "reads step i - 1's output after enqueueing step i"},
             "gpu_launches": launches_per_step(p0) * args.steps,
             "timed_regions": {"repeats": len(regions), "median_ms_per_step": ms, "min_ms_per_step": min(regions),
                               "max_ms_per_step": max(regions),

@@ -15,20 +15,18 @@
 //      ap_tiles writes one record per tile (item, list offset, tokens, sequence length);
 //   2. ap_attend_kernel: one persistent CTA per SM walks items (sequence, KV head, block)
 //      cut into tiles of 16 listed tokens x 8 query heads = 128 rows, the tiles spread
-//      evenly over the CTAs.  Per item the 8 compute warps dequantise the block once: K as
+//      evenly over the CTAs.  Per item the 4 compute warps dequantise the block once: K as
 //      bf16 [128 keys x 128 dims] and V transposed as f16 [128 dims x 128 keys], both in the
 //      K-major 128-byte-swizzle layout the tensor cores read (e2m1 x e4m3 is exact in both
-//      types); one warp streams the raw block (bulk copies, L2 evict-first) and each tile's
-//      query rows (16-byte cp.async from all 32 lanes into the 128-byte-swizzled layout, L2
-//      evict-last: a token's 8 heads are one 2 KB run of q; 1 KB TMA boxes were measured
-//      far slower), prefetching the records and token ids of the next tiles and publishing
+//      types); one warp streams the raw block (bulk copies) and each tile's query rows
+//      (TMA from 16 lanes, 128-byte swizzle, one 8-row atom per token, L2 evict-last, no
+//      multicast), prefetching the records and token ids of the next tiles and publishing
 //      each tile's record in a 4-slot shared-memory ring for the other warps; one thread issues
 //        S = Q K^T   tcgen05.mma kind::f16, bf16, 128 x 128 x 128, fp32 in TMEM,
 //        O = P V     tcgen05.mma kind::f16, f16,  128 x 128 x 128, fp32 in TMEM,
 //      with S and O double-buffered (4 x 128 TMEM columns) so that the softmax of one tile
-//      overlaps the MMAs of the next; the compute warps (two per TMEM lane quarter, each with
-//      64 of a row's 128 columns, exchanging the row's max and sum halves through shared
-//      memory) read S with tcgen05.ld, mask keys past the token's position, take the row max, write
+//      overlaps the MMAs of the next; the compute warps (one TMEM lane = one row each) read
+//      S with tcgen05.ld, mask keys past the token's position, take the row max, write
 //      P = 2^(S c - m c) as f16 into shared memory for the second MMA, and finally write
 //      the row's output normalised by its own sum (f16, unscaled by the V tensor scale)
 //      and its log-sum-exp to the token's slot;
@@ -37,6 +35,9 @@
 // Every output row's arithmetic is independent of the tile row it occupies and the merge
 // order is fixed, so results are bitwise reproducible although the lists are filled with
 // atomics.  Every wait is bounded (MSA_STATUS_TIMEOUT | MSA_STATUS_AT_ATTEND).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include "internal.h"
 #include "tcgen05.cuh"
 
@@ -74,7 +75,7 @@ struct ApWork {
     int32_t* list;              // [B * Tq * 16] entries t * 16 + slot, grouped by (b, n)
     int4* tiles;                // [B * Tq * 16 * Hkv] per tile: item, list offset, tokens, clamped L
     float* part_lse;            // [B][Tq][16][Hq]
-    __half* part_o;             // [B][Tq][16][Hq][D]
+    __half* part_o;             // [B][Tq][16][Hkv] blocks of 2 KB: [half][8-dim chunk][8 heads][8 dims]
 };
 
 // ------------------------------------------------------------------ selection inversion
@@ -192,38 +193,20 @@ struct ApTileInfo {
 constexpr int kApInfoSlots = 4;
 static_assert(sizeof(ApTileInfo) == 96, "tile record layout");
 
-// L2 eviction-priority policies: the queries are re-read by many tiles (keep them), the raw
-// cache blocks are read once per (block, KV head) (let them go first).
+// TMA load of a 4-D box with an L2 eviction-priority hint (no multicast).
+__device__ __forceinline__ void tma_load_4d_hint(void* dst, const void* tmap, int c0, int c1, int c2, int c3,
+                                                 uint64_t* bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint [%0], "
+        "[%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(smem_u32(dst)),
+        "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar)), "l"(policy)
+        : "memory");
+}
+
 __device__ __forceinline__ uint64_t l2_policy_evict_last() {
     uint64_t pol;
     asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
     return pol;
-}
-__device__ __forceinline__ uint64_t l2_policy_evict_first() {
-    uint64_t pol;
-    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
-    return pol;
-}
-
-// 16-byte asynchronous copy global -> shared (cache-global, L2 hint); completion is tracked by
-// ap_cp_async_arrive.
-__device__ __forceinline__ void ap_cp_async16(void* dst, const void* src, uint64_t pol) {
-    asm volatile("cp.async.cg.shared.global.L2::cache_hint [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src),
-                 "l"(pol)
-                 : "memory");
-}
-// Arrive on `bar` once this thread's earlier cp.async copies have landed (counted in the
-// barrier's initial arrival count).
-__device__ __forceinline__ void ap_cp_async_arrive(uint64_t* bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-// Untiled bulk copy with an L2 hint (no multicast), completing `bytes` on `bar`.
-__device__ __forceinline__ void ap_bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar, uint64_t pol) {
-    asm volatile(
-        "cp.async.bulk.shared::cta.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
-            smem_u32(dst)),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
-        : "memory");
 }
 
 __device__ __forceinline__ uint32_t f16x2_to_bf16x2(uint32_t h) {
@@ -305,7 +288,7 @@ __device__ __forceinline__ void ap_dequant(uint8_t* smem, int64_t kbase, int64_t
 
 template <bool PAGED>
 __global__ void __launch_bounds__(kApThreads, 1)
-    ap_attend_kernel(const Problem p, const ApWork w) {
+    ap_attend_kernel(const Problem p, const ApWork w, const __grid_constant__ CUtensorMap tmap) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kOffBar);
@@ -338,7 +321,7 @@ __global__ void __launch_bounds__(kApThreads, 1)
         mbar_init(kv_full, kApComputeWarps);
         mbar_init(kv_empty, 1);
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&q_full[s], 32);  // one cp.async arrival per producer lane
+            mbar_init(&q_full[s], 1);
             mbar_init(&q_empty[s], 1);
             mbar_init(&s_full[s], 1);
             mbar_init(&s_empty[s], kApComputeWarps);
@@ -377,7 +360,7 @@ __global__ void __launch_bounds__(kApThreads, 1)
         // query rows.  The tile record of tile tau + 2 and the token ids of tile tau + 1 are loaded while
         // tile tau is issued, so no global-load latency sits between two tiles.
         if (t0 < t1) {
-            const uint64_t pol_q = l2_policy_evict_last(), pol_kv = l2_policy_evict_first();
+            const uint64_t pol = l2_policy_evict_last();  // the queries are re-read by many tiles
             int4 m0 = w.tiles[t0];
             int4 m1 = t0 + 1 < t1 ? w.tiles[t0 + 1] : make_int4(0, 0, 0, 0);
             int e0 = lane < m0.z ? w.list[m0.y + lane] : 0;
@@ -400,10 +383,10 @@ __global__ void __launch_bounds__(kApThreads, 1)
                             const int64_t vec = block_vec<PAGED>(p, b, n, kvh, p.Hkv);
                             uint8_t* raw = smem + kOffRaw;
                             mbar_arrive_expect_tx(raw_full, 2 * (8192 + 1024));
-                            ap_bulk_g2s(raw + kRawK, p.k.data + vec * 64, 8192, raw_full, pol_kv);
-                            ap_bulk_g2s(raw + kRawKs, p.k.scale + vec * 8, 1024, raw_full, pol_kv);
-                            ap_bulk_g2s(raw + kRawV, p.v.data + vec * 64, 8192, raw_full, pol_kv);
-                            ap_bulk_g2s(raw + kRawVs, p.v.scale + vec * 8, 1024, raw_full, pol_kv);
+                            bulk_g2s(raw + kRawK, p.k.data + vec * 64, 8192, raw_full);
+                            bulk_g2s(raw + kRawKs, p.k.scale + vec * 8, 1024, raw_full);
+                            bulk_g2s(raw + kRawV, p.v.data + vec * 64, 8192, raw_full);
+                            bulk_g2s(raw + kRawVs, p.v.scale + vec * 8, 1024, raw_full);
                         }
                     }
                     ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -426,19 +409,17 @@ __global__ void __launch_bounds__(kApThreads, 1)
                     info[s4].L = m0.w;
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&info_full[s4]);
-                // the tile's query rows: each token's 8 heads are 2 KB contiguous in q, copied by 4
-                // rounds of the warp's 32 lanes x 16 bytes into the 128-byte-swizzled K-major tile
-                uint8_t* qs = smem + kOffQ + sb * kApTile;
-                for (int k = 0; k < 4 * ntok; ++k) {
-                    const int t = __shfl_sync(0xffffffffu, e0, k >> 2) / kTopK;  // token slot k / 4
-                    const int hc = (k & 3) * 32 + lane, h = hc >> 4, c16 = hc & 15;
-                    const int rw = (k >> 2) * kApG + h;  // tile row
-                    const __nv_bfloat16* src =
-                        p.q + (((int64_t)b * Tq + t) * p.Hq + kvh * kApG + h) * 128 + c16 * 8;
-                    ap_cp_async16(qs + (c16 >> 3) * kApKB + rw * 128 + (((c16 & 7) ^ (rw & 7)) << 4), src, pol_q);
+                if (lane == 0) {
+                    mbar_arrive(&info_full[s4]);
+                    mbar_arrive_expect_tx(&q_full[sb], (uint32_t)(ntok * 2 * 1024));
                 }
-                ap_cp_async_arrive(&q_full[sb]);
+                __syncwarp();
+                if (lane < ntok) {  // each lane gathers one token's 8 query heads
+                    const int t = e0 / kTopK;
+                    uint8_t* qs = smem + kOffQ + sb * kApTile + lane * 1024;
+                    tma_load_4d_hint(qs, &tmap, 0, kvh * kApG, t, b, &q_full[sb], pol);
+                    tma_load_4d_hint(qs + kApKB, &tmap, 64, kvh * kApG, t, b, &q_full[sb], pol);
+                }
                 issued = i + 1;
                 m0 = m1;
                 m1 = m2;
@@ -504,7 +485,6 @@ __global__ void __launch_bounds__(kApThreads, 1)
                     ok = false;
                     break;
                 }
-                fence_proxy_async_smem();  // the query rows were written by cp.async (generic proxy)
                 tcgen05_fence_after();
                 const uint32_t qa = smem_u32(smem + kOffQ + sb * kApTile);
 #pragma unroll
@@ -561,12 +541,14 @@ __global__ void __launch_bounds__(kApThreads, 1)
             for (int c4 = 0; c4 < 2; ++c4) tmem_ld32(lane_base + 256 + sb * 128 + c4 * 32, o[c4]);
             tmem_wait_ld();
             if (orow >= 0) {
-                uint4* dst = reinterpret_cast<uint4*>(w.part_o + orow * 128 + half * 64);
+                // the 8 heads of a token are interleaved at 8-dim (16-byte) granularity, so each
+                // store below writes whole 128-byte lines: 8 lanes (heads) x 16 bytes per token
+                uint4* dst = reinterpret_cast<uint4*>(w.part_o + (orow >> 3) * 1024) + (half * 8) * 8 + hq;
 #pragma unroll
                 for (int c4 = 0; c4 < 2; ++c4)
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
-                        __stcs(dst + 4 * c4 + q,
+                        __stcs(dst + (4 * c4 + q) * 8,
                                make_uint4(pack_f16x2(o[c4][8 * q] * inv, o[c4][8 * q + 1] * inv),
                                           pack_f16x2(o[c4][8 * q + 2] * inv, o[c4][8 * q + 3] * inv),
                                           pack_f16x2(o[c4][8 * q + 4] * inv, o[c4][8 * q + 5] * inv),
@@ -702,19 +684,21 @@ __global__ void __launch_bounds__(kApThreads, 1)
 
 // ------------------------------------------------------------------ merge of the slot partials
 
-// One thread per (sequence, token, query head, 8 dims).  All of the row's slot partials are
-// requested before any is combined (they are read once: streaming loads).
+// One thread per (sequence, token, query head, 8 dims); the 128 threads of a (token, KV
+// head) read each slot's 2 KB partial block as one contiguous run.  All of the row's slot
+// partials are requested before any is combined (they are read once: streaming loads).
 __global__ void __launch_bounds__(256) ap_merge_kernel(const Problem p, const ApWork w, float* __restrict__ out,
                                                        float* __restrict__ lse) {
     pdl_wait();
     pdl_launch_dependents();
     const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    const int64_t heads = (int64_t)p.B * p.Tq * p.Hq;
-    if (i >= heads * 16) return;
-    const int g8 = (int)(i & 15);
-    const int64_t rh = i >> 4;
-    const int hq = (int)(rh % p.Hq);
-    const int64_t bt = rh / p.Hq;
+    if (i >= (int64_t)p.B * p.Tq * p.Hkv * 128) return;
+    const int j = (int)(i & 127);  // position in the 2 KB block: (half * 8 + chunk) * 8 + head
+    const int hh = j & 7, g8 = j >> 3;  // head within the KV head's group; 8-dim chunk of the 128 dims
+    const int64_t bk = i >> 7;          // (b * Tq + t) * Hkv + kvh
+    const int kvh = (int)(bk % p.Hkv);
+    const int64_t bt = bk / p.Hkv;
+    const int hq = kvh * kApG + hh;
     const int b = (int)(bt / p.Tq), t = (int)(bt % p.Tq);
     const int64_t L = clamp_len(p.seq_lens[b], p.Tq, p.lmax, nullptr);
     const int64_t nvis = (L - p.Tq + t) / kBlock + 1;
@@ -734,9 +718,10 @@ __global__ void __launch_bounds__(256) ap_merge_kernel(const Problem p, const Ap
 #pragma unroll
     for (int s = 0; s < kTopK; ++s) {
         const bool valid = ids[s] >= 0 && ids[s] < nvis;
-        const int64_t r = (bt * kTopK + s) * p.Hq + hq;
-        ls[s] = valid ? __ldcs(w.part_lse + r) : -INFINITY;
-        ov[s] = valid ? __ldcs(reinterpret_cast<const uint4*>(w.part_o + r * 128 + g8 * 8)) : make_uint4(0, 0, 0, 0);
+        const int64_t pr = bt * kTopK + s;  // (token, slot)
+        ls[s] = valid ? __ldcs(w.part_lse + pr * p.Hq + hq) : -INFINITY;
+        ov[s] = valid ? __ldcs(reinterpret_cast<const uint4*>(w.part_o + (pr * p.Hkv + kvh) * 1024) + j)
+                      : make_uint4(0, 0, 0, 0);
         M = fmaxf(M, ls[s]);
     }
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
@@ -811,6 +796,18 @@ cudaLaunchConfig_t ap_config(dim3 grid, dim3 block, size_t smem, bool pdl, cudaS
 
 template <bool PAGED>
 int launch_ap_attend(const Problem& p, const ApWork& w, bool pdl, cudaStream_t st) {
+    auto enc = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(tensor_map_encode_entry());
+    if (enc == nullptr) return MSA_ECUDA;
+    // queries [B][Tq][Hq][128] bf16: boxes of 64 dims x 8 heads of one token, 128-byte swizzle
+    CUtensorMap tmap;
+    const cuuint64_t dims[4] = {128, (cuuint64_t)p.Hq, (cuuint64_t)p.Tq, (cuuint64_t)p.B};
+    const cuuint64_t strides[3] = {(cuuint64_t)128 * 2, (cuuint64_t)p.Hq * 128 * 2, (cuuint64_t)p.Tq * p.Hq * 128 * 2};
+    const cuuint32_t box[4] = {64, (cuuint32_t)kApG, 1, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    if (enc(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<__nv_bfloat16*>(p.q), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return MSA_ECUDA;
     auto kern = ap_attend_kernel<PAGED>;
     static int configured_dev = -1;
     const DeviceInfo& di = device_info();
@@ -821,7 +818,7 @@ int launch_ap_attend(const Problem& p, const ApWork& w, bool pdl, cudaStream_t s
     }
     cudaLaunchAttribute attr[1];
     cudaLaunchConfig_t cfg = ap_config(dim3((unsigned)di.num_sms), dim3(kApThreads), kApSmem, pdl, st, attr);
-    if (cudaLaunchKernelEx(&cfg, kern, p, w) != cudaSuccess) return MSA_ECUDA;
+    if (cudaLaunchKernelEx(&cfg, kern, p, w, tmap) != cudaSuccess) return MSA_ECUDA;
     return MSA_OK;
 }
 
@@ -864,7 +861,7 @@ int launch_attend_prefill(const Problem& p, const int32_t* sel, void* ws, float*
     if (cudaLaunchKernelEx(&cfg, ap_tiles_kernel, p, w) != cudaSuccess) return MSA_ECUDA;
     const int r = p.block_table != nullptr ? launch_ap_attend<true>(p, w, pdl, st) : launch_ap_attend<false>(p, w, pdl, st);
     if (r != MSA_OK) return r;
-    const int64_t threads = (int64_t)p.B * p.Tq * p.Hq * 16;
+    const int64_t threads = (int64_t)p.B * p.Tq * p.Hkv * 128;
     cfg = ap_config(dim3((unsigned)((threads + 255) / 256)), dim3(256), 0, pdl, st, attr);
     if (cudaLaunchKernelEx(&cfg, ap_merge_kernel, p, w, out, lse) != cudaSuccess) return MSA_ECUDA;
     return MSA_OK;
