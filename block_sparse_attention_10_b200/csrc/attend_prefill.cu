@@ -28,10 +28,11 @@
 //      overlaps the MMAs of the next; the compute warps (one TMEM lane = one row each) read
 //      S with tcgen05.ld, mask keys past the token's position, take the row max, write
 //      P = 2^(S c - m c) as f16 into shared memory for the second MMA, and finally write
-//      the row's output normalised by its own sum (f16, unscaled by the V tensor scale)
-//      and its log-sum-exp to the token's slot;
+//      the row's unnormalised output O / 128 (f16; V^T is dequantised already divided by 128,
+//      so no per-element scaling is needed and O / 128 stays below the largest dequantised
+//      value) with the row's max and sum to the token's slot;
 //   3. ap_merge_kernel combines each token's (up to) 16 slot partials in slot order:
-//      lse = log sum_s exp(lse_s), out = s_V * sum_s exp(lse_s - lse) o_s.
+//      out = s_V * 128 * sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
 // Every output row's arithmetic is independent of the tile row it occupies and the merge
 // order is fixed, so results are bitwise reproducible although the lists are filled with
 // atomics.  Every wait is bounded (MSA_STATUS_TIMEOUT | MSA_STATUS_AT_ATTEND).
@@ -74,7 +75,7 @@ struct ApWork {
     int32_t* tile_start;        // [items + 1] first tile of item (b, kvh, n); last entry = total
     int32_t* list;              // [B * Tq * 16] entries t * 16 + slot, grouped by (b, n)
     int4* tiles;                // [B * Tq * 16 * Hkv] per tile: item, list offset, tokens, clamped L
-    float* part_lse;            // [B][Tq][16][Hq]
+    float2* part_ml;            // [B][Tq][16][Hq]: (row max m * c, row sum l) of each slot's partial
     __half* part_o;             // [B][Tq][16][Hkv] blocks of 2 KB: [half][8-dim chunk][8 heads][8 dims]
 };
 
@@ -262,7 +263,9 @@ __device__ __forceinline__ void ap_dequant(uint8_t* smem, int64_t kbase, int64_t
     uint32_t rows[16][4];  // [dim 16 w16 + r][key pair i]
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-        const uint32_t sc = e4m3x2_to_f16x2(s[2 * i] | (s[2 * i + 1] << 8));  // (key 2i, key 2i+1)
+        // (key 2i, key 2i+1) scales times 2^-7: V^T is stored divided by 128 (exact in f16: every
+        // product stays a multiple of 2^-24 below 2^11), so P V is O / 128 and fits f16 unnormalised
+        const uint32_t sc = hmul2(e4m3x2_to_f16x2(s[2 * i] | (s[2 * i + 1] << 8)), 0x20002000u);
 #pragma unroll
         for (int hw = 0; hw < 2; ++hw) {
             const uint32_t A = hw ? x[2 * i].y : x[2 * i].x, Bw = hw ? x[2 * i + 1].y : x[2 * i + 1].x;
@@ -534,9 +537,7 @@ __global__ void __launch_bounds__(kApThreads, 1)
             const int sb = i & 1;
             if (!wait_all(&o_full[sb], (i >> 1) & 1)) return false;
             tcgen05_fence_after();
-            const float l = lh + xsum[(sb * 2 + (half ^ 1)) * 128 + row];
-            const float inv = l > 0.0f ? 1.0f / l : 0.0f;
-            float o[2][32];  // this half's 64 output columns in one round trip to tensor memory
+            float o[2][32];  // this half's 64 output columns (O / 128) in one round trip to tensor memory
 #pragma unroll
             for (int c4 = 0; c4 < 2; ++c4) tmem_ld32(lane_base + 256 + sb * 128 + c4 * 32, o[c4]);
             tmem_wait_ld();
@@ -549,15 +550,18 @@ __global__ void __launch_bounds__(kApThreads, 1)
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
                         __stcs(dst + (4 * c4 + q) * 8,
-                               make_uint4(pack_f16x2(o[c4][8 * q] * inv, o[c4][8 * q + 1] * inv),
-                                          pack_f16x2(o[c4][8 * q + 2] * inv, o[c4][8 * q + 3] * inv),
-                                          pack_f16x2(o[c4][8 * q + 4] * inv, o[c4][8 * q + 5] * inv),
-                                          pack_f16x2(o[c4][8 * q + 6] * inv, o[c4][8 * q + 7] * inv)));
+                               make_uint4(pack_f16x2(o[c4][8 * q], o[c4][8 * q + 1]),
+                                          pack_f16x2(o[c4][8 * q + 2], o[c4][8 * q + 3]),
+                                          pack_f16x2(o[c4][8 * q + 4], o[c4][8 * q + 5]),
+                                          pack_f16x2(o[c4][8 * q + 6], o[c4][8 * q + 7])));
             }
             tcgen05_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&o_empty[sb]);
-            if (orow >= 0 && half == 0) __stcs(w.part_lse + orow, (mc + log2f(l)) * kApLn2);
+            if (orow >= 0 && half == 0) {
+                const float l = lh + xsum[(sb * 2 + 1) * 128 + row];
+                __stcs(w.part_ml + orow, make_float2(mc, l));
+            }
             return true;
         };
         bool ok = true;
@@ -612,7 +616,7 @@ __global__ void __launch_bounds__(kApThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&s_empty[sb]);
                 float mx[8];
-                if (__all_sync(0xffffffffu, kvis >= 64)) {
+                if (__all_sync(0xffffffffu, kvis >= 64)) {  // the whole half visible: no predicates
 #pragma unroll
                     for (int j = 0; j < 8; ++j) mx[j] = v[0][j];
 #pragma unroll
@@ -640,13 +644,15 @@ __global__ void __launch_bounds__(kApThreads, 1)
                 // P: this half's 64 keys are K-block `half` of the P tile
                 uint8_t* prow = smem + kOffP + sb * kApTile + half * kApKB + row * 128;
                 float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                const bool full_half = __all_sync(0xffffffffu, kvis >= 64);
 #pragma unroll
                 for (int cc = 0; cc < 8; ++cc) {
                     float e8[8];
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
                         const int k = cc * 8 + u;
-                        e8[u] = k < kvis ? ex2_approx(fmaf(v[k >> 5][k & 31], c, -mc)) : 0.0f;
+                        if (full_half) e8[u] = ex2_approx(fmaf(v[k >> 5][k & 31], c, -mc));
+                        else e8[u] = k < kvis ? ex2_approx(fmaf(v[k >> 5][k & 31], c, -mc)) : 0.0f;
                         ls[u] += e8[u];
                     }
                     *reinterpret_cast<uint4*>(prow + ((cc ^ (row & 7)) << 4)) =
@@ -684,67 +690,90 @@ __global__ void __launch_bounds__(kApThreads, 1)
 
 // ------------------------------------------------------------------ merge of the slot partials
 
-// One thread per (sequence, token, query head, 8 dims); the 128 threads of a (token, KV
-// head) read each slot's 2 KB partial block as one contiguous run.  All of the row's slot
-// partials are requested before any is combined (they are read once: streaming loads).
-__global__ void __launch_bounds__(256) ap_merge_kernel(const Problem p, const ApWork w, float* __restrict__ out,
-                                                       float* __restrict__ lse) {
+// One thread per (sequence, token, query head, 8 dims); the 128 threads of a (token, KV head)
+// read each slot's 2 KB partial block as one run and write the group's 8 heads x 128 dims of
+// output (one contiguous run) through shared memory.  All of a row's slot partials are
+// requested before any is combined (they are read once: streaming loads).  Partial s holds
+// O_s / 128 (unnormalised) with its row max m_s (scaled, log2 domain) and row sum l_s:
+//   out = s_V * sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s,  lse = ln 2 * (M + log2 sum ...).
+constexpr int kMergeThreads = 256;  // two (token, KV head) groups per block
+__global__ void __launch_bounds__(kMergeThreads) ap_merge_kernel(const Problem p, const ApWork w,
+                                                                 float* __restrict__ out, float* __restrict__ lse) {
+    __shared__ float stage[kMergeThreads / 128][kApG * 128 + 4];
     pdl_wait();
     pdl_launch_dependents();
-    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (i >= (int64_t)p.B * p.Tq * p.Hkv * 128) return;
-    const int j = (int)(i & 127);  // position in the 2 KB block: (half * 8 + chunk) * 8 + head
-    const int hh = j & 7, g8 = j >> 3;  // head within the KV head's group; 8-dim chunk of the 128 dims
+    const int64_t groups = (int64_t)p.B * p.Tq * p.Hkv;
+    const int64_t i = (int64_t)blockIdx.x * kMergeThreads + threadIdx.x;
+    const int gl = threadIdx.x >> 7;    // group within the block
+    const int j = threadIdx.x & 127;    // position in the 2 KB block: (half * 8 + chunk) * 8 + head
+    const int hh = j & 7, g8 = j >> 3;  // head within the group; 8-dim chunk of the 128 dims
     const int64_t bk = i >> 7;          // (b * Tq + t) * Hkv + kvh
-    const int kvh = (int)(bk % p.Hkv);
-    const int64_t bt = bk / p.Hkv;
-    const int hq = kvh * kApG + hh;
-    const int b = (int)(bt / p.Tq), t = (int)(bt % p.Tq);
-    const int64_t L = clamp_len(p.seq_lens[b], p.Tq, p.lmax, nullptr);
-    const int64_t nvis = (L - p.Tq + t) / kBlock + 1;
-    const int4* selv = reinterpret_cast<const int4*>(w.sel + bt * kTopK);
-    int ids[kTopK];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const int4 x = __ldg(selv + q);
-        ids[4 * q] = x.x;
-        ids[4 * q + 1] = x.y;
-        ids[4 * q + 2] = x.z;
-        ids[4 * q + 3] = x.w;
-    }
-    float ls[kTopK];
-    uint4 ov[kTopK];
-    float M = -INFINITY;
-#pragma unroll
-    for (int s = 0; s < kTopK; ++s) {
-        const bool valid = ids[s] >= 0 && ids[s] < nvis;
-        const int64_t pr = bt * kTopK + s;  // (token, slot)
-        ls[s] = valid ? __ldcs(w.part_lse + pr * p.Hq + hq) : -INFINITY;
-        ov[s] = valid ? __ldcs(reinterpret_cast<const uint4*>(w.part_o + (pr * p.Hkv + kvh) * 1024) + j)
-                      : make_uint4(0, 0, 0, 0);
-        M = fmaxf(M, ls[s]);
-    }
+    const bool live = bk < groups;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    float W = 0.0f;
-    if (M != -INFINITY) {
+    int64_t bt = 0;
+    int hq = 0;
+    if (live) {
+        const int kvh = (int)(bk % p.Hkv);
+        bt = bk / p.Hkv;
+        hq = kvh * kApG + hh;
+        const int b = (int)(bt / p.Tq), t = (int)(bt % p.Tq);
+        const int64_t L = clamp_len(p.seq_lens[b], p.Tq, p.lmax, nullptr);
+        const int64_t nvis = (L - p.Tq + t) / kBlock + 1;
+        const int4* selv = reinterpret_cast<const int4*>(w.sel + bt * kTopK);
+        int ids[kTopK];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int4 x = __ldg(selv + q);
+            ids[4 * q] = x.x;
+            ids[4 * q + 1] = x.y;
+            ids[4 * q + 2] = x.z;
+            ids[4 * q + 3] = x.w;
+        }
+        float2 ml[kTopK];
+        uint4 ov[kTopK];
+        float M = -INFINITY;
 #pragma unroll
         for (int s = 0; s < kTopK; ++s) {
-            const float wt = ls[s] == -INFINITY ? 0.0f : expf(ls[s] - M);
-            W += wt;
-            const uint32_t vv[4] = {ov[s].x, ov[s].y, ov[s].z, ov[s].w};
+            const bool valid = ids[s] >= 0 && ids[s] < nvis;
+            const int64_t pr = bt * kTopK + s;  // (token, slot)
+            ml[s] = valid ? __ldcs(w.part_ml + pr * p.Hq + hq) : make_float2(-INFINITY, 0.0f);
+            ov[s] = valid ? __ldcs(reinterpret_cast<const uint4*>(w.part_o + (pr * p.Hkv + kvh) * 1024) + j)
+                          : make_uint4(0, 0, 0, 0);
+            M = fmaxf(M, ml[s].x);
+        }
+        float W = 0.0f;
+        if (M != -INFINITY) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&vv[q]));
-                acc[2 * q] += wt * f.x;
-                acc[2 * q + 1] += wt * f.y;
+            for (int s = 0; s < kTopK; ++s) {
+                const float wt = ml[s].x == -INFINITY ? 0.0f : exp2f(ml[s].x - M);
+                W += wt * ml[s].y;
+                const uint32_t vv[4] = {ov[s].x, ov[s].y, ov[s].z, ov[s].w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&vv[q]));
+                    acc[2 * q] += wt * f.x;
+                    acc[2 * q + 1] += wt * f.y;
+                }
             }
         }
-    }
-    const float inv = W > 0.0f ? p.v.s_t / W : 0.0f;
-    const int64_t o = (bt * p.Hq + hq) * 128 + g8 * 8;
+        const float inv = W > 0.0f ? 128.0f * p.v.s_t / W : 0.0f;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) store_out2(p, out, o + 2 * q, acc[2 * q] * inv, acc[2 * q + 1] * inv);
-    if (g8 == 0 && lse != nullptr) lse[bt * p.Hq + hq] = W > 0.0f ? M + logf(W) : -INFINITY;
+        for (int q = 0; q < 8; ++q) acc[q] *= inv;
+        if (g8 == 0 && lse != nullptr) lse[bt * p.Hq + hq] = W > 0.0f ? (M + log2f(W)) * kApLn2 : -INFINITY;
+    }
+    // the group's output is [8 heads][128 dims], contiguous in out: stage it, then write it in order
+    float* st = stage[gl];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) st[hh * 128 + g8 * 8 + q] = acc[q];
+    __syncthreads();
+    if (live) {
+        const int64_t o0 = (bt * p.Hq + (hq - hh)) * 128;  // first element of the group's 8 heads
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int e = 2 * (j + 128 * q);  // this thread's pairs are e, e + 256, e + 512, e + 768
+            store_out2(p, out, o0 + e, st[e], st[e + 1]);
+        }
+    }
 }
 
 // ------------------------------------------------------------------ host side
@@ -773,7 +802,7 @@ ApLayout ap_layout(const Problem& p) {
     a.tiles = at;
     at += ap_round(entries * p.Hkv * sizeof(int4));
     a.lse = at;
-    at += ap_round(entries * p.Hq * 4);
+    at += ap_round(entries * p.Hq * sizeof(float2));
     a.po = at;
     at += ap_round(entries * p.Hq * 128 * 2);
     a.total = at;
@@ -844,7 +873,7 @@ int launch_attend_prefill(const Problem& p, const int32_t* sel, void* ws, float*
     w.tile_start = reinterpret_cast<int32_t*>(base + a.tstart);
     w.list = reinterpret_cast<int32_t*>(base + a.list);
     w.tiles = reinterpret_cast<int4*>(base + a.tiles);
-    w.part_lse = reinterpret_cast<float*>(base + a.lse);
+    w.part_ml = reinterpret_cast<float2*>(base + a.lse);
     w.part_o = reinterpret_cast<__half*>(base + a.po);
     const int64_t entries = (int64_t)p.B * p.Tq * kTopK;
     if (cudaMemsetAsync(w.cnt, 0, (size_t)p.B * p.nbmax * 4, st) != cudaSuccess) return MSA_ECUDA;
@@ -862,7 +891,8 @@ int launch_attend_prefill(const Problem& p, const int32_t* sel, void* ws, float*
     const int r = p.block_table != nullptr ? launch_ap_attend<true>(p, w, pdl, st) : launch_ap_attend<false>(p, w, pdl, st);
     if (r != MSA_OK) return r;
     const int64_t threads = (int64_t)p.B * p.Tq * p.Hkv * 128;
-    cfg = ap_config(dim3((unsigned)((threads + 255) / 256)), dim3(256), 0, pdl, st, attr);
+    cfg = ap_config(dim3((unsigned)((threads + kMergeThreads - 1) / kMergeThreads)), dim3(kMergeThreads), 0, pdl, st,
+                    attr);
     if (cudaLaunchKernelEx(&cfg, ap_merge_kernel, p, w, out, lse) != cudaSuccess) return MSA_ECUDA;
     return MSA_OK;
 }
