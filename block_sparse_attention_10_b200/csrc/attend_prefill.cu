@@ -643,23 +643,22 @@ __global__ void __launch_bounds__(kApThreads, 1)
                 }
                 // P: this half's 64 keys are K-block `half` of the P tile
                 uint8_t* prow = smem + kOffP + sb * kApTile + half * kApKB + row * 128;
-                float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-                const bool full_half = __all_sync(0xffffffffu, kvis >= 64);
+                float ls[4] = {0.f, 0.f, 0.f, 0.f};  // 4 independent partial sums
+                // P = 2^(S c - m c) for this half's 64 keys (selects, not branches, for the mask)
 #pragma unroll
                 for (int cc = 0; cc < 8; ++cc) {
                     float e8[8];
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
                         const int k = cc * 8 + u;
-                        if (full_half) e8[u] = ex2_approx(fmaf(v[k >> 5][k & 31], c, -mc));
-                        else e8[u] = k < kvis ? ex2_approx(fmaf(v[k >> 5][k & 31], c, -mc)) : 0.0f;
-                        ls[u] += e8[u];
+                        e8[u] = k < kvis ? ex2_approx(fmaf(v[k >> 5][k & 31], c, -mc)) : 0.0f;
+                        ls[u & 3] += e8[u];
                     }
                     *reinterpret_cast<uint4*>(prow + ((cc ^ (row & 7)) << 4)) =
                         make_uint4(pack_f16x2(e8[0], e8[1]), pack_f16x2(e8[2], e8[3]), pack_f16x2(e8[4], e8[5]),
                                    pack_f16x2(e8[6], e8[7]));
                 }
-                const float lh = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
+                const float lh = (ls[0] + ls[1]) + (ls[2] + ls[3]);
                 xsum[(sb * 2 + half) * 128 + row] = lh;  // read by the partner in output(i), after the next meeting
                 fence_proxy_async_smem();
                 __syncwarp();
