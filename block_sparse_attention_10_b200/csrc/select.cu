@@ -9,7 +9,8 @@
 //
 // Rows of <= 1,024 blocks: one warp per (sequence, query token), the threshold
 // selection of select_row.cuh.  Rows of <= 4,096 blocks: one CTA of 8 warps per
-// row; each warp selects the best 15 of its 512-block chunk (the row's best 15
+// row; each warp selects the best 15 of its 256-block (rows of <= 2,048 blocks) or
+// 512-block chunk (the row's best 15
 // are among those 120), then one warp selects from the 120 candidates, which
 // sit in ascending block order so the index tie-break carries over.  Longer
 // rows: 64-bit keys (score key, inverted index) and 15 rounds of "largest key
@@ -24,10 +25,12 @@ constexpr int kSelThreads = 256;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kPer = 16;  // candidates per thread held in registers (rows of <= 4,096 blocks)
 
-// Rows of <= 4,096 blocks: one CTA of 8 warps per (sequence, query token), two levels.
+// Rows of <= 4,096 blocks: one CTA of 8 warps per (sequence, query token), two levels; each
+// lane holds PER candidates (16: rows of <= 4,096 blocks, 8: rows of <= 2,048 blocks).
 constexpr int kCtaPer = 16;  // 8 warps x 32 lanes x 16 candidates
 constexpr int kCtaMaxBlocks = kSelWarps * 32 * kCtaPer;
 
+template <int PER>
 __global__ void __launch_bounds__(kSelThreads)
     select_cta_kernel(const Problem p, const float* __restrict__ block_scores, int32_t* __restrict__ sel,
                       int32_t* __restrict__ sel_copy) {
@@ -41,7 +44,7 @@ __global__ void __launch_bounds__(kSelThreads)
     const int b = (int)(row / p.Tq), t = (int)(row % p.Tq);
     const int64_t L = clamp_len(p.seq_lens[b], p.Tq, p.lmax, nullptr);
     const int64_t r = (L - p.Tq + t) / kBlock;  // forced block
-    select_row_cta<kSelWarps, kCtaPer>(block_scores + row * p.nbmax, r + 1, r, warp, lane, ckey, cid, res);
+    select_row_cta<kSelWarps, PER>(block_scores + row * p.nbmax, r + 1, r, warp, lane, ckey, cid, res);
     if (warp != 0) return;
     __syncwarp();
     if (lane < kTopK) {
@@ -164,8 +167,10 @@ int launch_select(const Problem& p, const float* block_scores, int32_t* sel, int
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cudaError_t e;
-    if (!short_rows && p.nbmax <= kCtaMaxBlocks)
-        e = cudaLaunchKernelEx(&cfg, select_cta_kernel, p, block_scores, sel, sel_copy);
+    if (!short_rows && p.nbmax <= kCtaMaxBlocks / 2)
+        e = cudaLaunchKernelEx(&cfg, select_cta_kernel<kCtaPer / 2>, p, block_scores, sel, sel_copy);
+    else if (!short_rows && p.nbmax <= kCtaMaxBlocks)
+        e = cudaLaunchKernelEx(&cfg, select_cta_kernel<kCtaPer>, p, block_scores, sel, sel_copy);
     else if (!short_rows) e = cudaLaunchKernelEx(&cfg, select_kernel, p, block_scores, sel, sel_copy);
     else if (p.nbmax <= 32 * 4) e = cudaLaunchKernelEx(&cfg, select_warp_kernel<4>, p, block_scores, sel, sel_copy);
     else if (p.nbmax <= 32 * 16) e = cudaLaunchKernelEx(&cfg, select_warp_kernel<16>, p, block_scores, sel, sel_copy);
