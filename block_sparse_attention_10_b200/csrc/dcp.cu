@@ -11,7 +11,8 @@
 // query's own block plus the best 15 others, exact softmax attention over them):
 //   1. rank g scores the blocks [n0, n1) it holds (the decode indexer restricted to the
 //      range) and keeps its best min(15, count) blocks other than the query's own block,
-//      by (score desc, index asc): dcp_candidates_kernel;
+//      by (score desc, index asc): dcp_candidates_cta_kernel (threshold selection, ranges of
+//      up to 4,096 blocks) or dcp_candidates_kernel (rounds of a warp maximum, any range);
 //   2. the G lists are exchanged; every rank merges the G x 16 (score, id) pairs the same
 //      way: the query's own block plus the best min(15, r) of the pairs.  The best 15
 //      blocks of the whole context are among the ranks' best 15, so this is the
@@ -64,8 +65,8 @@ __device__ __forceinline__ uint64_t warp_best_keys(const float* __restrict__ s, 
 
 __device__ __forceinline__ int32_t key_index(uint64_t key) { return (int32_t)(0xFFFFFFFFu - (uint32_t)key); }
 
-// Step 1: block_scores (written by the range indexer) -> this rank's candidates per row:
-// slots 0..want-1 in (score desc, index asc) order, the rest (-inf, -1).
+// Step 1 for any range: block_scores (written by the range indexer) -> this rank's candidates
+// per row: slots 0..want-1 in (score desc, index asc) order, the rest (-inf, -1).
 __global__ void __launch_bounds__(32 * kDcpWarps)
     dcp_candidates_kernel(const Problem p, const float* __restrict__ block_scores, float* __restrict__ cand_score,
                           int32_t* __restrict__ cand_id) {
@@ -87,6 +88,76 @@ __global__ void __launch_bounds__(32 * kDcpWarps)
         const int32_t id = have ? key_index(key) : -1;
         cand_id[row * kTopK + lane] = id;
         cand_score[row * kTopK + lane] = have ? __ldg(s + id) : -INFINITY;
+    }
+}
+
+// Step 1 for ranges of up to 8 * 32 * PER blocks: one CTA of 8 warps per row.  Warp w finds
+// the best min(15, c_w) blocks of its 32 * PER blocks of the range by threshold (the k-th best
+// 32-bit score key, then an ordered pass that keeps the lowest-indexed ties), writing them in
+// ascending block order; warp 0 then does the same over the warps' candidates, which are in
+// ascending block order, so the index tie-break carries over.  Output ascending by block.
+constexpr int kDcpCtaWarps = 8;
+template <int PER>
+__global__ void __launch_bounds__(32 * kDcpCtaWarps)
+    dcp_candidates_cta_kernel(const Problem p, const float* __restrict__ block_scores, float* __restrict__ cand_score,
+                              int32_t* __restrict__ cand_id) {
+    constexpr int kCand = kTopK - 1;
+    __shared__ uint32_t ckey[kDcpCtaWarps * kCand];
+    __shared__ int32_t cid[kDcpCtaWarps * kCand];
+    __shared__ int32_t res[kTopK];
+    pdl_wait();
+    pdl_launch_dependents();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t row = blockIdx.x;
+    const int b = (int)(row / p.Tq), t = (int)(row % p.Tq);
+    const int64_t L = clamp_len(p.seq_lens[b], p.Tq, p.lmax, nullptr);
+    const int64_t r = (L - p.Tq + t) / kBlock;  // the query's own block
+    const int64_t lo = p.blk_lo, hi = min64(p.blk_hi, r + 1);
+    const float* s = block_scores + row * p.nbmax;
+    const int64_t base = lo + (int64_t)warp * 32 * PER;
+    uint32_t k[PER];
+    int cnt = 0;
+#pragma unroll
+    for (int j = 0; j < PER; ++j) {
+        const int64_t n = base + (int64_t)j * 32 + lane;
+        k[j] = (n < hi && n != r) ? score_key(__ldg(s + n)) : 0u;
+        cnt += k[j] != 0u ? 1 : 0;
+    }
+    cnt = (int)__reduce_add_sync(0xffffffffu, (unsigned)cnt);
+    const int want_w = min(kCand, cnt);
+    if (want_w > 0) {
+        int n_gt;
+        const uint32_t T = warp_kth_key(k, want_w, n_gt);
+        warp_compact(k, T, want_w - n_gt, lane, [&](int slot, int j) {
+            ckey[warp * kCand + slot] = k[j];
+            cid[warp * kCand + slot] = (int32_t)(base + j * 32 + lane);
+        });
+    }
+    if (lane >= want_w && lane < kCand) ckey[warp * kCand + lane] = 0u;
+    __syncthreads();
+    if (warp != 0) return;
+    constexpr int kC = kDcpCtaWarps * kCand;
+    constexpr int kPer2 = (kC + 31) / 32;
+    uint32_t kk[kPer2];
+    int c2 = 0;
+#pragma unroll
+    for (int j = 0; j < kPer2; ++j) {
+        const int cc = j * 32 + lane;
+        kk[j] = cc < kC ? ckey[cc] : 0u;
+        c2 += kk[j] != 0u ? 1 : 0;
+    }
+    c2 = (int)__reduce_add_sync(0xffffffffu, (unsigned)c2);
+    const int want = min(kCand, c2);
+    if (want > 0) {
+        int n_gt;
+        const uint32_t T = warp_kth_key(kk, want, n_gt);
+        warp_compact(kk, T, want - n_gt, lane, [&](int slot, int j) { res[slot] = cid[j * 32 + lane]; });
+    }
+    __syncwarp();
+    if (lane < kTopK) {
+        const int32_t id = lane < want ? res[lane] : -1;
+        cand_id[row * kTopK + lane] = id;
+        cand_score[row * kTopK + lane] = id >= 0 ? __ldg(s + id) : -INFINITY;
     }
 }
 
@@ -210,6 +281,18 @@ int launch_merge_per(const Problem& p, int G, const float* cs, const int32_t* ci
 int launch_dcp_candidates(const Problem& p, const float* block_scores, float* cand_score, int32_t* cand_id, bool pdl,
                           cudaStream_t st) {
     const int64_t rows = (int64_t)p.B * p.Tq;
+    const int64_t span = p.blk_hi - p.blk_lo;
+    if (span <= 8 * 32 * 16 && rows <= 0x7FFFFFFFll) {  // one CTA per row, threshold selection
+        cudaLaunchAttribute attr[1];
+        cudaLaunchConfig_t cfg = pdl_config(dim3((unsigned)rows), dim3(32 * kDcpCtaWarps), pdl, st, attr);
+        cudaError_t e = span <= 8 * 32 * 4 ? cudaLaunchKernelEx(&cfg, dcp_candidates_cta_kernel<4>, p, block_scores,
+                                                                cand_score, cand_id)
+                        : span <= 8 * 32 * 8 ? cudaLaunchKernelEx(&cfg, dcp_candidates_cta_kernel<8>, p, block_scores,
+                                                                  cand_score, cand_id)
+                                             : cudaLaunchKernelEx(&cfg, dcp_candidates_cta_kernel<16>, p, block_scores,
+                                                                  cand_score, cand_id);
+        return e == cudaSuccess ? MSA_OK : MSA_ECUDA;
+    }
     if ((rows + kDcpWarps - 1) / kDcpWarps > 0x7FFFFFFFll) return MSA_EUNSUPPORTED;
     cudaLaunchAttribute attr[1];
     cudaLaunchConfig_t cfg =

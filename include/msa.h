@@ -251,8 +251,10 @@ size_t msa_dcp_workspace_size(const msa_params_t* p);
  * blocks other than the query's own block r (c = the visible blocks of the range
  * other than r), by (score desc, block index asc):
  *   ws, ws_bytes  at least msa_dcp_workspace_size(p) bytes, 256-byte aligned
- *   cand_score    fp32 [B][Tq][16], cand_id int32 [B][Tq][16]: the candidates in
- *                 that order, then (-inf, -1) padding (slot 15 is always padding)
+ *   cand_score    fp32 [B][Tq][16], cand_id int32 [B][Tq][16]: the candidates
+ *                 (ascending block order for ranges of up to 4,096 blocks, else by
+ *                 descending score; the merge does not depend on the order), then
+ *                 (-inf, -1) padding (slot 15 is always padding)
  * Returns MSA_EINVAL for an empty or out-of-bounds range, MSA_EUNSUPPORTED for
  * Tq * HI > 32. */
 int msa_dcp_candidates(const msa_params_t* p, int64_t n0, int64_t n1, void* ws, size_t ws_bytes,

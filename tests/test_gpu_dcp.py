@@ -135,8 +135,13 @@ def test_ranks_read_only_their_own_blocks(case, G):
         assert status_of(r) == 0  # no page outside a rank's range was read
     assert np.array_equal(sel.cpu().numpy(), d["sel"])
     check_attention(out.cpu().numpy(), d["out"])
-    # candidates: per rank, at most 15, descending (score, then ascending id), inside the range
+    # candidates: per rank, exactly the best min(15, c) blocks of its range other than the
+    # query's own block by (score desc, id asc) -- checked against the pooled scores of the
+    # whole-context indexer -- ascending by id, inside the range, scores equal to the pooled ones
     cs_h, ci_h = cs.cpu().numpy(), ci.cpu().numpy()
+    bs = torch.empty(B, Tq, p.nbmax, dtype=torch.float32, device="cuda")
+    msa.msa_index(p, bs)
+    bs_h = bs.cpu().numpy()
     for g, (n0, n1) in enumerate(ranges):
         for b in range(B):
             for t in range(Tq):
@@ -144,9 +149,12 @@ def test_ranks_read_only_their_own_blocks(case, G):
                 k = int((ids >= 0).sum())
                 assert (ids[:k] >= 0).all() and (ids[k:] == -1).all() and ids[15] == -1
                 assert ((ids[:k] >= n0) & (ids[:k] < n1)).all()
-                sc = cs_h[g, b, t, :k]
-                order = sorted(range(k), key=lambda i: (-sc[i], ids[i]))
-                assert order == list(range(k))
+                assert list(ids[:k]) == sorted(ids[:k])
+                assert np.array_equal(cs_h[g, b, t, :k], bs_h[b, t, ids[:k]])
+                r = (inp.seq_lens[b] - Tq + t) // 128
+                pool = [n for n in range(n0, min(n1, r + 1)) if n != r]
+                best = sorted(pool, key=lambda n: (-bs_h[b, t, n], n))[:15]
+                assert sorted(best) == list(ids[:k])
 
 
 def test_full_size_speculative_verify_ranks():
