@@ -47,23 +47,22 @@ namespace {
 
 constexpr int kApG = 8;                // query heads per KV head on this path
 constexpr int kApTok = 128 / kApG;     // listed tokens per 128-row tile
-constexpr int kApComputeWarps = 8;  // two per TMEM lane quarter, one per half of a row's 128 columns
-constexpr int kApMmaWarp = 8;
-constexpr int kApTmaWarp = 9;
-constexpr int kApThreads = 32 * 10;
+constexpr int kApDqWarp = 8;           // warps 8..11: the dequantising warpgroup
+constexpr int kApMmaWarp = 12;
+constexpr int kApTmaWarp = 13;
+constexpr int kApRawWarp = 14;
+constexpr int kApThreads = 32 * 16;    // warps 0..7: two softmax warpgroups (one per tile parity); warp 15 idle
 constexpr int kApTile = 32768;         // 128 rows x 128 16-bit elements: two 16 KB K-blocks
 constexpr int kApKB = 16384;           // one K-block (64 elements of 128 rows)
-constexpr int kOffK = 0;               // K, bf16 [key][dim]
-constexpr int kOffV = kApTile;         // V^T, f16 [dim][key]
-constexpr int kOffQ = 2 * kApTile;     // 2 query stages
-constexpr int kOffP = 4 * kApTile;     // 2 P buffers, f16 [row][key]
+constexpr int kOffQ = 0;               // 2 query stages
+constexpr int kOffKV = 2 * kApTile;    // 2 item buffers: K bf16 [key][dim], then V^T f16 [dim][key]
 constexpr int kOffRaw = 6 * kApTile;   // the raw NVFP4 block: K nibbles, K scales, V nibbles, V scales
 constexpr int kRawK = 0, kRawKs = 8192, kRawV = 9216, kRawVs = 17408, kRawBytes = 18432;
-constexpr int kOffBar = kOffRaw + kRawBytes;  // 37 mbarriers + the TMEM address
-constexpr int kOffInfo = kOffBar + 384;       // 4 tile records
-constexpr int kOffXch = kOffInfo + 4 * 96;    // row max / row sum halves exchanged by the two warps of a row
-constexpr size_t kApSmem = 1024 + kOffXch + 4 * 2 * 128 * 4;
-constexpr uint32_t kApTmemCols = 512;  // S at columns 0 / 128, O at 256 / 384
+constexpr int kOffBar = kOffRaw + kRawBytes;  // 29 mbarriers + the TMEM address
+constexpr int kOffInfo = kOffBar + 256;       // 4 tile records
+constexpr int kApInfoSlots = 4;
+constexpr size_t kApSmem = 1024 + kOffInfo + kApInfoSlots * 96;
+constexpr uint32_t kApTmemCols = 512;  // S (then P) at columns 0 / 128, O at 256 / 384
 constexpr float kApLog2e = 1.4426950408889634f;
 constexpr float kApLn2 = 0.6931471805599453f;
 
@@ -185,13 +184,13 @@ __global__ void ap_tiles_kernel(const Problem p, const ApWork w) {
 
 // ------------------------------------------------------------------ block-major attention
 
-// One tile as the producer warp publishes it to the MMA thread and the compute warps.
+// One tile as the producer warp publishes it to the MMA thread and the softmax warps.
 struct ApTileInfo {
     int32_t item, b, kvh, n, ntok, L;
-    int32_t pad[2];
+    int32_t seq;  // the item's number among this CTA's items (selects its K/V buffer)
+    int32_t pad;
     int32_t entry[kApTok];  // t * 16 + slot of the tile's tokens
 };
-constexpr int kApInfoSlots = 4;
 static_assert(sizeof(ApTileInfo) == 96, "tile record layout");
 
 // TMA load of a 4-D box with an L2 eviction-priority hint (no multicast).
@@ -216,25 +215,40 @@ __device__ __forceinline__ uint32_t f16x2_to_bf16x2(uint32_t h) {
     return *reinterpret_cast<const uint32_t*>(&b);
 }
 
-// The raw NVFP4 block (keys kbase .. kbase + 127 of one KV head) -> K (bf16 [key][dim]) and
-// V^T (f16 [dim][key]), 128-byte swizzle, K-major; keys at or past L become zeros.
-// Called by the 256 threads of the compute warps: threads 128..255 write K, threads 0..127 V^T.
-__device__ __forceinline__ void ap_dequant(uint8_t* smem, int64_t kbase, int64_t L, int tid256) {
-    const uint8_t* raw = smem + kOffRaw;
-    const int nvalid = (int)min64(kBlock, max64(0, L - kbase));
-    if (tid256 >= 128) {
-    const int tid = tid256 - 128;
-    uint8_t* kt = smem + kOffK;
+// One thread's V share (of 128) of a raw NVFP4 block, read into registers so that the raw
+// buffer can be refilled while V^T is converted: keys 8 (tid / 8) + a, dims 16 (tid % 8) .. + 15.
+struct ApRawV {
+    uint2 vx[8];
+    uint32_t vs[8];
+};
+
+__device__ __forceinline__ void ap_raw_read_v(ApRawV& r, const uint8_t* raw, int nvalid, int tid) {
+    const int w16 = tid & 7, kg = tid >> 3;
+#pragma unroll
+    for (int a = 0; a < 8; ++a) {
+        const int key = kg * 8 + a;
+        r.vx[a] = *reinterpret_cast<const uint2*>(raw + kRawV + key * 64 + w16 * 8);
+        r.vs[a] = raw[kRawVs + key * 8 + w16];
+        if (key >= nvalid) {
+            r.vx[a] = make_uint2(0u, 0u);
+            r.vs[a] = 0u;
+        }
+    }
+}
+
+// K, bf16 [key][dim], 128-byte swizzle, K-major (e2m1 x e4m3 is exact in bf16), straight from
+// the raw block; keys at or past nvalid become zeros.
+__device__ __forceinline__ void ap_dequant_k(uint8_t* kt, const uint8_t* raw, int nvalid, int tid) {
 #pragma unroll 4
-    for (int k = 0; k < 16; ++k) {
-        const int q = tid + 128 * k;
+    for (int i = 0; i < 16; ++i) {
+        const int q = tid + 128 * i;
         const int j = q >> 4, cr = q & 15;  // key j, dims 8 cr .. 8 cr + 7
-        uint32_t w = *reinterpret_cast<const uint32_t*>(raw + kRawK + j * 64 + cr * 4);
-        uint32_t sc = raw[kRawKs + j * 8 + (cr >> 1)];
-        if (j >= nvalid) w = sc = 0u;
+        uint32_t kw = *reinterpret_cast<const uint32_t*>(raw + kRawK + j * 64 + cr * 4);
+        uint32_t ks = raw[kRawKs + j * 8 + (cr >> 1)];
+        if (j >= nvalid) kw = ks = 0u;
         uint32_t h[4];
-        e2m1x8_to_f16x8(w, h[0], h[1], h[2], h[3]);
-        const uint32_t s2 = e4m3_bcast_f16x2(sc);
+        e2m1x8_to_f16x8(kw, h[0], h[1], h[2], h[3]);
+        const uint32_t s2 = e4m3_bcast_f16x2(ks);
         uint4 o;
         o.x = f16x2_to_bf16x2(hmul2(h[0], s2));
         o.y = f16x2_to_bf16x2(hmul2(h[1], s2));
@@ -242,33 +256,21 @@ __device__ __forceinline__ void ap_dequant(uint8_t* smem, int64_t kbase, int64_t
         o.w = f16x2_to_bf16x2(hmul2(h[3], s2));
         *reinterpret_cast<uint4*>(kt + (cr >> 3) * kApKB + j * 128 + (((cr & 7) ^ (j & 7)) << 4)) = o;
     }
-    return;
-    }
-    const int tid = tid256;
-    // V^T: thread = (dims 16 w16 .. 16 w16 + 15, keys 8 kg .. 8 kg + 7) -> 16 rows x one 16-byte chunk
-    uint8_t* vt = smem + kOffV;
+}
+
+// V^T, f16 [dim][key] divided by 128, 128-byte swizzle, K-major: thread = (dims 16 w16 ..
+// 16 w16 + 15, keys 8 kg .. 8 kg + 7), written as 16 rows x one 16-byte chunk.
+__device__ __forceinline__ void ap_dequant_vt(uint8_t* vt, const ApRawV& r, int tid) {
     const int w16 = tid & 7, kg = tid >> 3;
-    uint2 x[8];
-    uint32_t s[8];
-#pragma unroll
-    for (int a = 0; a < 8; ++a) {
-        const int key = kg * 8 + a;
-        x[a] = *reinterpret_cast<const uint2*>(raw + kRawV + key * 64 + w16 * 8);
-        s[a] = raw[kRawVs + key * 8 + w16];
-        if (key >= nvalid) {
-            x[a] = make_uint2(0u, 0u);
-            s[a] = 0u;
-        }
-    }
     uint32_t rows[16][4];  // [dim 16 w16 + r][key pair i]
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         // (key 2i, key 2i+1) scales times 2^-7: V^T is stored divided by 128 (exact in f16: every
         // product stays a multiple of 2^-24 below 2^11), so P V is O / 128 and fits f16 unnormalised
-        const uint32_t sc = hmul2(e4m3x2_to_f16x2(s[2 * i] | (s[2 * i + 1] << 8)), 0x20002000u);
+        const uint32_t sc = hmul2(e4m3x2_to_f16x2(r.vs[2 * i] | (r.vs[2 * i + 1] << 8)), 0x20002000u);
 #pragma unroll
         for (int hw = 0; hw < 2; ++hw) {
-            const uint32_t A = hw ? x[2 * i].y : x[2 * i].x, Bw = hw ? x[2 * i + 1].y : x[2 * i + 1].x;
+            const uint32_t A = hw ? r.vx[2 * i].y : r.vx[2 * i].x, Bw = hw ? r.vx[2 * i + 1].y : r.vx[2 * i + 1].x;
             const uint32_t ev = (A & 0x0F0F0F0Fu) | ((Bw << 4) & 0xF0F0F0F0u);  // byte k: dim 8 hw + 2k
             const uint32_t od = ((A >> 4) & 0x0F0F0F0Fu) | (Bw & 0xF0F0F0F0u);  // byte k: dim 8 hw + 2k + 1
             uint32_t e[4], o[4];
@@ -282,11 +284,59 @@ __device__ __forceinline__ void ap_dequant(uint8_t* smem, int64_t kbase, int64_t
         }
     }
 #pragma unroll
-    for (int r = 0; r < 16; ++r) {
-        const int d = 16 * w16 + r;
+    for (int rr = 0; rr < 16; ++rr) {
+        const int d = 16 * w16 + rr;
         *reinterpret_cast<uint4*>(vt + (kg >> 3) * kApKB + d * 128 + (((kg & 7) ^ (d & 7)) << 4)) =
-            make_uint4(rows[r][0], rows[r][1], rows[r][2], rows[r][3]);
+            make_uint4(rows[rr][0], rows[rr][1], rows[rr][2], rows[rr][3]);
     }
+}
+
+// One row's softmax numerators: m = max of the row's first kvis scores of the S tile at
+// taddr (128 fp32 TMEM columns of this thread's lane), P_k = 2^(S_k c - m c) (0 for k >= kvis),
+// written as f16 pairs over the first 64 of those columns; returns the row sum of the fp32 P
+// and sets mc = m c (0 for an empty row).  S is read twice (max, then exponentials) in chunks
+// of 32 columns, in loops that are not unrolled: the code stays small enough for the
+// instruction cache while the other warp roles run beside it.  MASKED = false: every key
+// visible (kvis >= 128), no selects.
+template <bool MASKED>
+__device__ __forceinline__ float ap_softmax_row(uint32_t taddr, float c, int kvis, float& mc) {
+    float mx[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) mx[j] = -INFINITY;
+#pragma unroll 1
+    for (int k0 = 0; k0 < 128; k0 += 32) {
+        float v[32];
+        tmem_ld32(taddr + k0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < 32; ++k)
+            if (!MASKED || k0 + k < kvis) mx[k & 7] = fmaxf(mx[k & 7], v[k]);
+    }
+    const float m = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])), fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+    mc = kvis > 0 ? m * c : 0.0f;
+    float ls[4] = {0.f, 0.f, 0.f, 0.f};  // 4 independent partial sums
+    // keys k0 .. k0 + 31 -> P columns k0 / 2 .. k0 / 2 + 15, which lie in S columns already read
+#pragma unroll 1
+    for (int k0 = 0; k0 < 128; k0 += 32) {
+        float v[32];
+        tmem_ld32(taddr + k0, v);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            float x0 = ex2_approx(fmaf(v[2 * u], c, -mc));
+            float x1 = ex2_approx(fmaf(v[2 * u + 1], c, -mc));
+            if (MASKED) {
+                x0 = k0 + 2 * u < kvis ? x0 : 0.0f;
+                x1 = k0 + 2 * u + 1 < kvis ? x1 : 0.0f;
+            }
+            ls[(2 * u) & 3] += x0;
+            ls[(2 * u + 1) & 3] += x1;
+            pk[u] = pack_f16x2(x0, x1);
+        }
+        tmem_st16(taddr + (k0 >> 1), pk);
+    }
+    return (ls[0] + ls[1]) + (ls[2] + ls[3]);
 }
 
 template <bool PAGED>
@@ -297,48 +347,43 @@ __global__ void __launch_bounds__(kApThreads, 1)
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kOffBar);
     uint64_t* raw_full = bar + 0;
     uint64_t* raw_empty = bar + 1;
-    uint64_t* kv_full = bar + 2;
-    uint64_t* kv_empty = bar + 3;
-    uint64_t* q_full = bar + 4;       // [2]
-    uint64_t* q_empty = bar + 6;      // [2]
-    uint64_t* s_full = bar + 8;       // [2]
-    uint64_t* s_empty = bar + 10;     // [2]
-    uint64_t* p_full = bar + 12;      // [2]
-    uint64_t* p_empty = bar + 14;     // [2]
+    uint64_t* k_full = bar + 2;       // [2 item buffers]
+    uint64_t* v_full = bar + 4;       // [2]
+    uint64_t* kv_empty = bar + 6;     // [2]
+    uint64_t* q_full = bar + 8;       // [2 query stages = tile parities]
+    uint64_t* q_empty = bar + 10;     // [2]
+    uint64_t* s_full = bar + 12;      // [2 warpgroups = tile parities]
+    uint64_t* p_full = bar + 14;      // [2]
     uint64_t* o_full = bar + 16;      // [2]
     uint64_t* o_empty = bar + 18;     // [2]
     uint64_t* info_full = bar + 20;   // [4]
     uint64_t* info_empty = bar + 24;  // [4]
     uint64_t* done = bar + 28;
-    uint64_t* pair = bar + 29;        // [4 lane quarters][2]: the two warps of a row met
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 37);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 29);
     ApTileInfo* info = reinterpret_cast<ApTileInfo*>(smem + kOffInfo);
-    float* xmax = reinterpret_cast<float*>(smem + kOffXch);  // [2 tile parities][2 halves][128 rows]
-    float* xsum = xmax + 2 * 2 * 128;                         // [2 tile parities][2 halves][128 rows]
+    uint8_t* raw = smem + kOffRaw;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     pdl_wait();
     if (threadIdx.x == 0) {
         mbar_init(raw_full, 1);
-        mbar_init(raw_empty, kApComputeWarps);
-        mbar_init(kv_full, kApComputeWarps);
-        mbar_init(kv_empty, 1);
+        mbar_init(raw_empty, 4);  // the 4 dequantising warps have read the block
         for (int s = 0; s < 2; ++s) {
+            mbar_init(&k_full[s], 4);
+            mbar_init(&v_full[s], 4);
+            mbar_init(&kv_empty[s], 1);
             mbar_init(&q_full[s], 1);
             mbar_init(&q_empty[s], 1);
             mbar_init(&s_full[s], 1);
-            mbar_init(&s_empty[s], kApComputeWarps);
-            mbar_init(&p_full[s], kApComputeWarps);
-            mbar_init(&p_empty[s], 1);
+            mbar_init(&p_full[s], 4);
             mbar_init(&o_full[s], 1);
-            mbar_init(&o_empty[s], kApComputeWarps);
+            mbar_init(&o_empty[s], 4);
         }
         for (int s = 0; s < kApInfoSlots; ++s) {
             mbar_init(&info_full[s], 1);
-            mbar_init(&info_empty[s], kApComputeWarps + 1);  // the compute warps and the MMA thread
+            mbar_init(&info_empty[s], 4 + 1);  // the tile's warpgroup and the MMA thread
         }
         mbar_init(done, 1);
-        for (int s = 0; s < 8; ++s) mbar_init(&pair[s], 2);
         fence_mbar_init();
     }
     if (warp == kApMmaWarp) {
@@ -355,23 +400,23 @@ __global__ void __launch_bounds__(kApThreads, 1)
     const int total = w.tile_start[items];
     const int t0 = (int)((int64_t)total * blockIdx.x / gridDim.x);
     const int t1 = (int)((int64_t)total * (blockIdx.x + 1) / gridDim.x);
+    const int ntiles = t1 - t0;
     const int Tq = p.Tq;
     auto fail = [&]() { set_status(p.status, MSA_STATUS_TIMEOUT | MSA_STATUS_AT_ATTEND); };
 
     if (warp == kApTmaWarp) {
-        // ------------------------------------------------------------ producer warp: tile records, raw blocks,
-        // query rows.  The tile record of tile tau + 2 and the token ids of tile tau + 1 are loaded while
-        // tile tau is issued, so no global-load latency sits between two tiles.
-        if (t0 < t1) {
+        // ------------------------------------------------------------ producer warp: tile records and query
+        // rows.  The tile record of tile tau + 2 and the token ids of tile tau + 1 are loaded while tile tau
+        // is issued, so no global-load latency sits between two tiles.
+        if (ntiles > 0) {
             const uint64_t pol = l2_policy_evict_last();  // the queries are re-read by many tiles
             int4 m0 = w.tiles[t0];
             int4 m1 = t0 + 1 < t1 ? w.tiles[t0 + 1] : make_int4(0, 0, 0, 0);
             int e0 = lane < m0.z ? w.list[m0.y + lane] : 0;
-            int cur = -1, it = -1, issued = 0;
+            int cur = -1, seq = -1, issued = 0;
             bool ok = true;
             for (int tau = t0; tau < t1 && ok; ++tau) {
                 const int i = tau - t0, sb = i & 1, s4 = i & (kApInfoSlots - 1);
-                // prefetch: token ids of the next tile, record of the one after
                 const int e1 = (tau + 1 < t1 && lane < m1.z) ? w.list[m1.y + lane] : 0;
                 const int4 m2 = tau + 2 < t1 ? w.tiles[tau + 2] : make_int4(0, 0, 0, 0);
                 const int item = m0.x, ntok = m0.z;
@@ -379,21 +424,7 @@ __global__ void __launch_bounds__(kApThreads, 1)
                 const int kvh = bk % p.Hkv, b = bk / p.Hkv;
                 if (item != cur) {
                     cur = item;
-                    ++it;
-                    if (lane == 0) {
-                        if (it >= 1 && !mbar_wait(raw_empty, (it - 1) & 1)) ok = false;
-                        if (ok) {
-                            const int64_t vec = block_vec<PAGED>(p, b, n, kvh, p.Hkv);
-                            uint8_t* raw = smem + kOffRaw;
-                            mbar_arrive_expect_tx(raw_full, 2 * (8192 + 1024));
-                            bulk_g2s(raw + kRawK, p.k.data + vec * 64, 8192, raw_full);
-                            bulk_g2s(raw + kRawKs, p.k.scale + vec * 8, 1024, raw_full);
-                            bulk_g2s(raw + kRawV, p.v.data + vec * 64, 8192, raw_full);
-                            bulk_g2s(raw + kRawVs, p.v.scale + vec * 8, 1024, raw_full);
-                        }
-                    }
-                    ok = __shfl_sync(0xffffffffu, ok, 0);
-                    if (!ok) break;
+                    ++seq;
                 }
                 if (lane == 0) {
                     if (i >= kApInfoSlots && !mbar_wait(&info_empty[s4], ((i >> 2) - 1) & 1)) ok = false;
@@ -401,7 +432,6 @@ __global__ void __launch_bounds__(kApThreads, 1)
                 }
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
-                // publish the tile record
                 if (lane < kApTok) info[s4].entry[lane] = e0;
                 if (lane == 0) {
                     info[s4].item = item;
@@ -410,6 +440,7 @@ __global__ void __launch_bounds__(kApThreads, 1)
                     info[s4].n = n;
                     info[s4].ntok = ntok;
                     info[s4].L = m0.w;
+                    info[s4].seq = seq;
                 }
                 __syncwarp();
                 if (lane == 0) {
@@ -430,253 +461,228 @@ __global__ void __launch_bounds__(kApThreads, 1)
             }
             if (!ok && lane == 0) fail();
             // never leave with copies in flight into this CTA's shared memory
-            if (lane == 0) {
+            if (lane == 0)
                 for (int i = max(0, issued - 2); i < issued; ++i)
                     if (!mbar_wait(&q_full[i & 1], (i >> 1) & 1)) {
                         fail();
                         break;
                     }
-                if (it >= 0 && !mbar_wait(raw_full, it & 1)) fail();
+        }
+    } else if (warp >= kApDqWarp && warp < kApDqWarp + 4) {
+        // ------------------------------------------------------------ dequantising warpgroup: every item of
+        // this CTA in order, into item buffer seq & 1 (free once the PV MMAs of item seq - 2 are done): the
+        // thread's V share of the raw block goes to registers, K is converted from the raw block (the S MMAs
+        // wait for K only), the raw buffer is released (the next block streams in meanwhile), then V^T.
+        if (ntiles > 0) {
+            const int tid = threadIdx.x - 32 * kApDqWarp;
+            auto wait_all = [&](uint64_t* b_, uint32_t parity) -> bool {
+                return __all_sync(0xffffffffu, mbar_wait(b_, parity)) != 0;
+            };
+            int cur = -1, seq = -1;
+            bool ok = true;
+            int4 nxt = w.tiles[t0];
+            for (int tau = t0; tau < t1; ++tau) {
+                const int4 m = nxt;
+                if (tau + 1 < t1) nxt = w.tiles[tau + 1];
+                if (m.x == cur) continue;
+                cur = m.x;
+                ++seq;
+                const int kb = seq & 1;
+                if (!wait_all(raw_full, seq & 1) || (seq >= 2 && !wait_all(&kv_empty[kb], ((seq >> 1) - 1) & 1))) {
+                    ok = false;
+                    break;
+                }
+                const int n = m.x % (int)p.nbmax;
+                const int nvalid = (int)min64(kBlock, max64(0, (int64_t)m.w - (int64_t)n * kBlock));
+                ApRawV r;
+                ap_raw_read_v(r, raw, nvalid, tid);
+                uint8_t* kvb = smem + kOffKV + kb * 2 * kApTile;
+                ap_dequant_k(kvb, raw, nvalid, tid);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(raw_empty);  // every read of the raw block is done
+                    mbar_arrive(&k_full[kb]);
+                }
+                ap_dequant_vt(kvb + kApTile, r, tid);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&v_full[kb]);
             }
+            if (!ok && lane == 0) fail();
+        }
+    } else if (warp == kApRawWarp) {
+        // ------------------------------------------------------------ raw-block loader (one thread): each
+        // item's NVFP4 K and V block (bulk copies), as soon as the previous item has been dequantised, so
+        // that the copy runs while the tiles of that item are computed.
+        if (lane == 0 && ntiles > 0) {
+            int cur = -1, seq = -1;
+            bool ok = true;
+            int nxt = w.tiles[t0].x;
+            for (int tau = t0; tau < t1; ++tau) {
+                const int item = nxt;
+                if (tau + 1 < t1) nxt = w.tiles[tau + 1].x;
+                if (item == cur) continue;
+                cur = item;
+                ++seq;
+                if (seq >= 1 && !mbar_wait(raw_empty, (seq - 1) & 1)) {
+                    ok = false;
+                    break;
+                }
+                const int n = item % (int)p.nbmax, bk = item / (int)p.nbmax;
+                const int kvh = bk % p.Hkv, b = bk / p.Hkv;
+                const int64_t vec = block_vec<PAGED>(p, b, n, kvh, p.Hkv);
+                mbar_arrive_expect_tx(raw_full, 2 * (8192 + 1024));
+                bulk_g2s(raw + kRawK, p.k.data + vec * 64, 8192, raw_full);
+                bulk_g2s(raw + kRawKs, p.k.scale + vec * 8, 1024, raw_full);
+                bulk_g2s(raw + kRawV, p.v.data + vec * 64, 8192, raw_full);
+                bulk_g2s(raw + kRawVs, p.v.scale + vec * 8, 1024, raw_full);
+            }
+            if (!ok) fail();
+            if (seq >= 0 && !mbar_wait(raw_full, seq & 1)) fail();  // the last copy has landed
         }
     } else if (warp == kApMmaWarp) {
-        // ------------------------------------------------------------ MMA issuer (one thread)
-        if (lane == 0 && t0 < t1) {
+        // ------------------------------------------------------------ MMA issuer (one thread).  Order:
+        // S(0), S(1), PV(0), S(2), PV(1), ...: S(i) reuses the TMEM columns that held P(i - 2), which
+        // PV(i - 2), issued earlier by this thread, reads first (tcgen05.mma runs in issue order).
+        if (lane == 0 && ntiles > 0) {
             constexpr uint32_t idesc_s = umma_idesc_bf16_f32(128, 128);
             constexpr uint32_t idesc_o = umma_idesc_f16_f32(128, 128);
-            const uint32_t kt = smem_u32(smem + kOffK), vt = smem_u32(smem + kOffV);
-            auto pv = [&](int i) -> bool {
-                const int sb = i & 1;
-                if (!mbar_wait(&p_full[sb], (i >> 1) & 1)) return false;
-                if (i >= 2 && !mbar_wait(&o_empty[sb], ((i >> 1) - 1) & 1)) return false;
+            int kseq = -1, vseq = -1, seq_prev = -1;
+            auto pv = [&](int j, int seq_j, bool last_of_item) -> bool {
+                const int g = j & 1;
+                if (!mbar_wait(&p_full[g], (j >> 1) & 1)) return false;
+                if (seq_j != vseq) {
+                    if (!mbar_wait(&v_full[seq_j & 1], (seq_j >> 1) & 1)) return false;
+                    vseq = seq_j;
+                }
+                if (j >= 2 && !mbar_wait(&o_empty[g], ((j >> 1) - 1) & 1)) return false;
                 tcgen05_fence_after();
-                const uint32_t pa = smem_u32(smem + kOffP + sb * kApTile);
+                const uint32_t vt = smem_u32(smem + kOffKV + (seq_j & 1) * 2 * kApTile + kApTile);
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    umma_bf16_ss(tmem + 256 + sb * 128, umma_desc_k_sw128(pa + (k >> 2) * kApKB + (k & 3) * 32),
-                                 umma_desc_k_sw128(vt + (k >> 2) * kApKB + (k & 3) * 32), idesc_o, k > 0 ? 1u : 0u);
-                umma_commit(&p_empty[sb]);
-                umma_commit(&o_full[sb]);
+                    umma_f16_ts(tmem + 256 + g * 128, tmem + g * 128 + k * 8,
+                                umma_desc_k_sw128(vt + (k >> 2) * kApKB + (k & 3) * 32), idesc_o, k > 0 ? 1u : 0u);
+                umma_commit(&o_full[g]);
+                if (last_of_item) umma_commit(&kv_empty[seq_j & 1]);  // every MMA reading the item's K and V
                 return true;
             };
-            int cur = -1, it = -1;
-            bool ok = true, pending = false;
-            for (int tau = t0; tau < t1 && ok; ++tau) {
-                const int i = tau - t0, sb = i & 1, s4 = i & (kApInfoSlots - 1);
+            bool ok = true;
+            for (int i = 0; i < ntiles; ++i) {
+                const int g = i & 1, s4 = i & (kApInfoSlots - 1);
                 if (!mbar_wait(&info_full[s4], (i >> 2) & 1)) {
                     ok = false;
                     break;
                 }
-                const int item = info[s4].item;
+                const int seq = info[s4].seq;
                 mbar_arrive(&info_empty[s4]);
-                if (item != cur) {
-                    if (pending && !pv(i - 1)) {
+                if (seq != kseq) {
+                    if (!mbar_wait(&k_full[seq & 1], (seq >> 1) & 1)) {
                         ok = false;
                         break;
                     }
-                    pending = false;
-                    if (it >= 0) umma_commit(kv_empty);  // every MMA reading this item's K and V
-                    cur = item;
-                    ++it;
-                    if (!mbar_wait(kv_full, it & 1)) {
-                        ok = false;
-                        break;
-                    }
-                    tcgen05_fence_after();
+                    kseq = seq;
                 }
-                if (!mbar_wait(&q_full[sb], (i >> 1) & 1) || (i >= 2 && !mbar_wait(&s_empty[sb], ((i >> 1) - 1) & 1))) {
+                if (!mbar_wait(&q_full[g], (i >> 1) & 1)) {
                     ok = false;
                     break;
                 }
                 tcgen05_fence_after();
-                const uint32_t qa = smem_u32(smem + kOffQ + sb * kApTile);
+                const uint32_t qa = smem_u32(smem + kOffQ + g * kApTile);
+                const uint32_t kt = smem_u32(smem + kOffKV + (seq & 1) * 2 * kApTile);
 #pragma unroll
                 for (int k = 0; k < 8; ++k)
-                    umma_bf16_ss(tmem + sb * 128, umma_desc_k_sw128(qa + (k >> 2) * kApKB + (k & 3) * 32),
+                    umma_bf16_ss(tmem + g * 128, umma_desc_k_sw128(qa + (k >> 2) * kApKB + (k & 3) * 32),
                                  umma_desc_k_sw128(kt + (k >> 2) * kApKB + (k & 3) * 32), idesc_s, k > 0 ? 1u : 0u);
-                umma_commit(&q_empty[sb]);
-                umma_commit(&s_full[sb]);
-                if (pending && !pv(i - 1)) {
+                umma_commit(&q_empty[g]);
+                umma_commit(&s_full[g]);
+                if (i >= 1 && !pv(i - 1, seq_prev, seq != seq_prev)) {
                     ok = false;
                     break;
                 }
-                pending = true;
+                seq_prev = seq;
             }
-            if (ok && pending && !pv(t1 - t0 - 1)) ok = false;
+            if (ok && !pv(ntiles - 1, seq_prev, false)) ok = false;
             if (!ok) fail();
             // every MMA issued has completed before the CTA releases its tensor memory
             umma_commit(done);
             if (!mbar_wait(done, 0)) fail();
         }
-    } else {
-        // ------------------------------------------------------------ compute warps: dequant, softmax, output.
-        // Warp w handles TMEM lanes (= tile rows) 32 (w % 4) .. + 31 and columns 64 (w / 4) .. + 63 of S,
-        // P and O; the two warps of a row exchange their halves' max and sum through shared memory,
-        // meeting on the pair mbarrier of their lane quarter (bounded waits, no unbounded named barrier).
-        const int qw = warp & 3, half = warp >> 2;
-        const int row = qw * 32 + lane;
-        const int tslot = row >> 3, hq = row & 7;
-        const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16) + (uint32_t)(half * 64);
+    } else if (warp < 8) {
+        // ------------------------------------------------------------ softmax warpgroups: warpgroup g takes
+        // the tiles of parity g, so that one warpgroup's exponentials overlap the other's tensor-memory
+        // traffic and output.  Thread = one row (TMEM lane) = (token slot row / 8, query head row % 8).
+        const int g = warp >> 2, qw = warp & 3;
+        const int row = qw * 32 + lane, tslot = row >> 3, hq = row & 7;
+        const uint32_t lane_base = tmem + ((uint32_t)(qw * 32) << 16);
         const float c = p.softmax_scale * p.k.s_t * kApLog2e;
-        float prev_mc = 0.0f, prev_l = 0.0f;
-        int64_t prev_row = -1;
         auto wait_all = [&](uint64_t* b_, uint32_t parity) -> bool {
             return __all_sync(0xffffffffu, mbar_wait(b_, parity)) != 0;
         };
-        // the two warps of this lane quarter meet (k-th meeting: parity k & 1 of pair[qw][k & 1] ... )
-        int meets = 0;
-        auto meet = [&]() -> bool {
-            uint64_t* pb = &pair[qw * 2 + (meets & 1)];
+        bool ok = true;
+        for (int i = g; i < ntiles; i += 2) {
+            const int s4 = i & (kApInfoSlots - 1);
+            if (!wait_all(&info_full[s4], (i >> 2) & 1)) {
+                ok = false;
+                break;
+            }
+            const ApTileInfo& ti = info[s4];
+            const int n = ti.n, b = ti.b, kvh = ti.kvh, ntok = ti.ntok;
+            const int64_t L = ti.L;
+            const int e = tslot < ntok ? ti.entry[tslot] : 0;
             __syncwarp();
-            if (lane == 0) mbar_arrive(pb);
-            const bool r = wait_all(pb, (uint32_t)((meets >> 1) & 1));
-            ++meets;
-            return r;
-        };
-        auto output = [&](int i, float mc, float lh, int64_t orow) -> bool {
-            const int sb = i & 1;
-            if (!wait_all(&o_full[sb], (i >> 1) & 1)) return false;
+            if (lane == 0) mbar_arrive(&info_empty[s4]);
+            int kvis = 0;  // visible keys of the row's block (0: no token in this tile row)
+            int64_t orow = -1;
+            if (tslot < ntok) {
+                const int t = e / kTopK, slot = e % kTopK;
+                kvis = (int)min64(kBlock, L - Tq + t - (int64_t)n * kBlock + 1);
+                orow = (((int64_t)b * Tq + t) * kTopK + slot) * p.Hq + kvh * kApG + hq;
+            }
+            if (!wait_all(&s_full[g], (i >> 1) & 1)) {
+                ok = false;
+                break;
+            }
             tcgen05_fence_after();
-            float o[2][32];  // this half's 64 output columns (O / 128) in one round trip to tensor memory
-#pragma unroll
-            for (int c4 = 0; c4 < 2; ++c4) tmem_ld32(lane_base + 256 + sb * 128 + c4 * 32, o[c4]);
-            tmem_wait_ld();
-            if (orow >= 0) {
-                // the 8 heads of a token are interleaved at 8-dim (16-byte) granularity, so each
-                // store below writes whole 128-byte lines: 8 lanes (heads) x 16 bytes per token
-                uint4* dst = reinterpret_cast<uint4*>(w.part_o + (orow >> 3) * 1024) + (half * 8) * 8 + hq;
-#pragma unroll
-                for (int c4 = 0; c4 < 2; ++c4)
+            // no key masked in this warp: the unpredicated form
+            float mc;
+            const float l = __all_sync(0xffffffffu, kvis >= kBlock) ? ap_softmax_row<false>(lane_base + g * 128, c, kvis, mc)
+                                                                    : ap_softmax_row<true>(lane_base + g * 128, c, kvis, mc);
+            tmem_wait_st();
+            tcgen05_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full[g]);
+            // ---- output: the row's O / 128 (f16) and (m c, l)
+            if (!wait_all(&o_full[g], (i >> 1) & 1)) {
+                ok = false;
+                break;
+            }
+            tcgen05_fence_after();
+            // the 8 heads of a token are interleaved at 8-dim (16-byte) granularity, so each store
+            // below writes whole 128-byte lines: 8 lanes (heads) x 16 bytes per token
+            uint4* dst = reinterpret_cast<uint4*>(w.part_o + (orow >> 3) * 1024) + hq;
+#pragma unroll 1
+            for (int c4 = 0; c4 < 4; ++c4) {
+                float o[32];
+                tmem_ld32(lane_base + 256 + g * 128 + c4 * 32, o);
+                tmem_wait_ld();
+                if (c4 == 3) {
+                    tcgen05_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&o_empty[g]);
+                }
+                if (orow >= 0) {
 #pragma unroll
                     for (int q = 0; q < 4; ++q)
                         __stcs(dst + (4 * c4 + q) * 8,
-                               make_uint4(pack_f16x2(o[c4][8 * q], o[c4][8 * q + 1]),
-                                          pack_f16x2(o[c4][8 * q + 2], o[c4][8 * q + 3]),
-                                          pack_f16x2(o[c4][8 * q + 4], o[c4][8 * q + 5]),
-                                          pack_f16x2(o[c4][8 * q + 6], o[c4][8 * q + 7])));
+                               make_uint4(pack_f16x2(o[8 * q], o[8 * q + 1]), pack_f16x2(o[8 * q + 2], o[8 * q + 3]),
+                                          pack_f16x2(o[8 * q + 4], o[8 * q + 5]),
+                                          pack_f16x2(o[8 * q + 6], o[8 * q + 7])));
+                }
             }
-            tcgen05_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&o_empty[sb]);
-            if (orow >= 0 && half == 0) {
-                const float l = lh + xsum[(sb * 2 + 1) * 128 + row];
-                __stcs(w.part_ml + orow, make_float2(mc, l));
-            }
-            return true;
-        };
-        bool ok = true;
-        if (t0 < t1) {
-            int cur = -1, it = -1;
-            for (int tau = t0; tau < t1; ++tau) {
-                const int i = tau - t0, sb = i & 1, s4 = i & (kApInfoSlots - 1);
-                if (!wait_all(&info_full[s4], (i >> 2) & 1)) {
-                    ok = false;
-                    break;
-                }
-                const ApTileInfo& ti = info[s4];
-                const int item = ti.item, n = ti.n, b = ti.b, kvh = ti.kvh, ntok = ti.ntok;
-                const int64_t L = ti.L;
-                const int e = tslot < ntok ? ti.entry[tslot] : 0;
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&info_empty[s4]);
-                if (item != cur) {
-                    cur = item;
-                    ++it;
-                    if (!wait_all(raw_full, it & 1) || (it >= 1 && !wait_all(kv_empty, (it - 1) & 1))) {
-                        ok = false;
-                        break;
-                    }
-                    ap_dequant(smem, (int64_t)n * kBlock, L, threadIdx.x);
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                    if (lane == 0) {
-                        mbar_arrive(raw_empty);
-                        mbar_arrive(kv_full);
-                    }
-                }
-                // ---- softmax of tile i (this warp's 64 columns of its 32 rows)
-                int kv_row = 0;  // visible keys of the row's block (0: no token in this tile row)
-                int64_t orow = -1;
-                if (tslot < ntok) {
-                    const int t = e / kTopK, slot = e % kTopK;
-                    kv_row = (int)min64(kBlock, L - Tq + t - (int64_t)n * kBlock + 1);
-                    orow = (((int64_t)b * Tq + t) * kTopK + slot) * p.Hq + kvh * kApG + hq;
-                }
-                const int kvis = kv_row - half * 64;  // visible keys of this half (may be <= 0)
-                if (!wait_all(&s_full[sb], (i >> 1) & 1)) {
-                    ok = false;
-                    break;
-                }
-                tcgen05_fence_after();
-                float v[2][32];  // S: key 64 half + k in v[k / 32][k % 32]
-#pragma unroll
-                for (int c4 = 0; c4 < 2; ++c4) tmem_ld32(lane_base + sb * 128 + c4 * 32, v[c4]);
-                tmem_wait_ld();
-                tcgen05_fence_before();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&s_empty[sb]);
-                float mx[8];
-                if (__all_sync(0xffffffffu, kvis >= 64)) {  // the whole half visible: no predicates
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) mx[j] = v[0][j];
-#pragma unroll
-                    for (int k = 8; k < 64; ++k) mx[k & 7] = fmaxf(mx[k & 7], v[k >> 5][k & 31]);
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) mx[j] = -INFINITY;
-#pragma unroll
-                    for (int k = 0; k < 64; ++k)
-                        if (k < kvis) mx[k & 7] = fmaxf(mx[k & 7], v[k >> 5][k & 31]);
-                }
-                const float mh = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-                xmax[(sb * 2 + half) * 128 + row] = mh;
-                if (!meet()) {  // also publishes the partner's row sums of tile i - 1
-                    ok = false;
-                    break;
-                }
-                const float m = fmaxf(mh, xmax[(sb * 2 + (half ^ 1)) * 128 + row]);
-                const float mc = kv_row > 0 ? m * c : 0.0f;
-                if (i >= 2 && !wait_all(&p_empty[sb], ((i >> 1) - 1) & 1)) {
-                    ok = false;
-                    break;
-                }
-                // P: this half's 64 keys are K-block `half` of the P tile
-                uint8_t* prow = smem + kOffP + sb * kApTile + half * kApKB + row * 128;
-                float ls[4] = {0.f, 0.f, 0.f, 0.f};  // 4 independent partial sums
-                // P = 2^(S c - m c) for this half's 64 keys (selects, not branches, for the mask)
-#pragma unroll
-                for (int cc = 0; cc < 8; ++cc) {
-                    float e8[8];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const int k = cc * 8 + u;
-                        e8[u] = k < kvis ? ex2_approx(fmaf(v[k >> 5][k & 31], c, -mc)) : 0.0f;
-                        ls[u & 3] += e8[u];
-                    }
-                    *reinterpret_cast<uint4*>(prow + ((cc ^ (row & 7)) << 4)) =
-                        make_uint4(pack_f16x2(e8[0], e8[1]), pack_f16x2(e8[2], e8[3]), pack_f16x2(e8[4], e8[5]),
-                                   pack_f16x2(e8[6], e8[7]));
-                }
-                const float lh = (ls[0] + ls[1]) + (ls[2] + ls[3]);
-                xsum[(sb * 2 + half) * 128 + row] = lh;  // read by the partner in output(i), after the next meeting
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&p_full[sb]);
-                // ---- output of tile i - 1 (its PV MMA ran while this tile's softmax did)
-                if (i >= 1 && !output(i - 1, prev_mc, prev_l, prev_row)) {
-                    ok = false;
-                    break;
-                }
-                prev_mc = mc;
-                prev_l = lh;
-                prev_row = orow;
-            }
-            // the partner's row sums of the last tile: one more meeting
-            if (ok && !meet()) ok = false;
-            if (ok && !output(t1 - t0 - 1, prev_mc, prev_l, prev_row)) ok = false;
-            if (!ok && lane == 0) fail();
+            if (orow >= 0) __stcs(w.part_ml + orow, make_float2(mc, l));
         }
+        if (!ok && lane == 0) fail();
     }
 
     tcgen05_fence_before();
