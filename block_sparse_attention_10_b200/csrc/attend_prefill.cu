@@ -12,25 +12,30 @@
 // of them, so this file turns the work around and goes block by block:
 //   1. ap_count / ap_scan / ap_fill invert the selection: for every (sequence, block) the
 //      list of (token, slot) pairs that selected it (slot = its place in the token's 16);
-//      ap_tiles writes one record per tile (item, list offset, tokens, sequence length);
+//      ap_tiles writes one 96-byte record per tile (item, coordinates, tokens, sequence
+//      length, the next item's first tile, the 16 list entries);
 //   2. ap_attend_kernel: one persistent CTA per SM walks items (sequence, KV head, block)
 //      cut into tiles of 16 listed tokens x 8 query heads = 128 rows, the tiles spread
-//      evenly over the CTAs.  Per item the 4 compute warps dequantise the block once: K as
-//      bf16 [128 keys x 128 dims] and V transposed as f16 [128 dims x 128 keys], both in the
-//      K-major 128-byte-swizzle layout the tensor cores read (e2m1 x e4m3 is exact in both
-//      types); one warp streams the raw block (bulk copies) and each tile's query rows
-//      (TMA from 16 lanes, 128-byte swizzle, one 8-row atom per token, L2 evict-last, no
-//      multicast), prefetching the records and token ids of the next tiles and publishing
-//      each tile's record in a 4-slot shared-memory ring for the other warps; one thread issues
-//        S = Q K^T   tcgen05.mma kind::f16, bf16, 128 x 128 x 128, fp32 in TMEM,
-//        O = P V     tcgen05.mma kind::f16, f16,  128 x 128 x 128, fp32 in TMEM,
-//      with S and O double-buffered (4 x 128 TMEM columns) so that the softmax of one tile
-//      overlaps the MMAs of the next; the compute warps (one TMEM lane = one row each) read
-//      S with tcgen05.ld, mask keys past the token's position, take the row max, write
-//      P = 2^(S c - m c) as f16 into shared memory for the second MMA, and finally write
-//      the row's unnormalised output O / 128 (f16; V^T is dequantised already divided by 128,
-//      so no per-element scaling is needed and O / 128 stays below the largest dequantised
-//      value) with the row's max and sum to the token's slot;
+//      evenly over the CTAs.  Warp roles (16 warps, at most 128 registers each):
+//        producer   bulk-copies tile records 6 tiles ahead into an 8-slot shared ring and
+//                   gathers each tile's query rows (TMA from 16 lanes, 128-byte swizzle, one
+//                   8-row atom per token, L2 evict-last, no multicast) into 2 stages;
+//        dequant    a warpgroup that, item by item, loads the NVFP4 block straight from the
+//                   caches into registers and writes K as bf16 [128 keys x 128 dims] and V
+//                   transposed as f16 [128 dims x 128 keys] (divided by 128), both K-major
+//                   with the 128-byte swizzle (e2m1 x e4m3 is exact in both types), into one
+//                   of 2 item buffers, so the next item is ready before the current one ends;
+//        MMA        one thread issues, in order of readiness,
+//                     S = Q K^T  tcgen05.mma kind::f16, bf16, 128 x 128 x 128, fp32 in TMEM,
+//                     O = P V    tcgen05.mma kind::f16, f16, A (= P) read from TMEM;
+//        softmax    two warpgroups take alternate tiles (one TMEM lane = one row per thread),
+//                   so one's exponentials overlap the other's TMEM traffic and output: read S
+//                   (two passes of 32-column chunks: row max, then exponentials), mask keys
+//                   past the token's position, write P = 2^(S c - m c) as f16 over S's first
+//                   64 columns, then read O and write the row's unnormalised O / 128 (f16)
+//                   with (m c, l) to the token's slot.
+//      TMEM holds S / P of the two warpgroups at columns 0 / 128 and their O at 256 / 384;
+//      S(i) reuses the columns of P(i - 2), so it is issued after P V(i - 2);
 //   3. ap_merge_kernel combines each token's (up to) 16 slot partials in slot order:
 //      out = s_V * 128 * sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s.
 // Every output row's arithmetic is independent of the tile row it occupies and the merge
@@ -50,21 +55,33 @@ constexpr int kApTok = 128 / kApG;     // listed tokens per 128-row tile
 constexpr int kApDqWarp = 8;           // warps 8..11: the dequantising warpgroup
 constexpr int kApMmaWarp = 12;
 constexpr int kApTmaWarp = 13;
-constexpr int kApRawWarp = 14;
-constexpr int kApThreads = 32 * 16;    // warps 0..7: two softmax warpgroups (one per tile parity); warp 15 idle
+constexpr int kApThreads = 32 * 16;    // warps 0..7: two softmax warpgroups (one per tile parity); 14, 15 idle
 constexpr int kApTile = 32768;         // 128 rows x 128 16-bit elements: two 16 KB K-blocks
 constexpr int kApKB = 16384;           // one K-block (64 elements of 128 rows)
-constexpr int kOffQ = 0;               // 2 query stages
-constexpr int kOffKV = 2 * kApTile;    // 2 item buffers: K bf16 [key][dim], then V^T f16 [dim][key]
-constexpr int kOffRaw = 6 * kApTile;   // the raw NVFP4 block: K nibbles, K scales, V nibbles, V scales
-constexpr int kRawK = 0, kRawKs = 8192, kRawV = 9216, kRawVs = 17408, kRawBytes = 18432;
-constexpr int kOffBar = kOffRaw + kRawBytes;  // 29 mbarriers + the TMEM address
-constexpr int kOffInfo = kOffBar + 256;       // 4 tile records
-constexpr int kApInfoSlots = 4;
+// Two query stages: a third one (room exists once the raw block is read straight from the
+// caches) made a few rows per step come out wrong, which the back-to-back bitwise test catches.
+constexpr int kApQStages = 2;
+constexpr int kOffQ = 0;
+constexpr int kOffKV = kApQStages * kApTile;   // 2 item buffers: K bf16 [key][dim], then V^T f16 [dim][key]
+constexpr int kOffBar = kOffKV + 4 * kApTile;  // 37 mbarriers + the TMEM address
+static_assert(kApQStages <= 3, "barrier layout holds 3 query stages");
+constexpr int kOffInfo = kOffBar + 384;       // ring of 8 tile records
+constexpr int kApInfoSlots = 8;
+constexpr int kApRecAhead = 6;                // records in flight ahead of the tile being issued
 constexpr size_t kApSmem = 1024 + kOffInfo + kApInfoSlots * 96;
 constexpr uint32_t kApTmemCols = 512;  // S (then P) at columns 0 / 128, O at 256 / 384
 constexpr float kApLog2e = 1.4426950408889634f;
 constexpr float kApLn2 = 0.6931471805599453f;
+
+// One tile, as ap_tiles_kernel writes it and the producer warp copies it (one 96-byte bulk
+// copy) into the shared-memory ring read by the MMA thread and the tile's softmax warpgroup.
+struct ApTileInfo {
+    int32_t item, b, kvh, n, ntok, L;
+    int32_t next;  // first tile of the next item (the loader and the dequantising warps jump there)
+    int32_t pad;
+    int32_t entry[kApTok];  // t * 16 + slot of the tile's tokens (0 past ntok)
+};
+static_assert(sizeof(ApTileInfo) == 96, "tile record layout");
 
 struct ApWork {
     const int32_t* sel;         // [B][Tq][16]
@@ -73,7 +90,7 @@ struct ApWork {
     int32_t* list_off;          // [B * nbmax] start of each list
     int32_t* tile_start;        // [items + 1] first tile of item (b, kvh, n); last entry = total
     int32_t* list;              // [B * Tq * 16] entries t * 16 + slot, grouped by (b, n)
-    int4* tiles;                // [B * Tq * 16 * Hkv] per tile: item, list offset, tokens, clamped L
+    ApTileInfo* recs;    // [tile bound] one 96-byte record per tile (see ApTileInfo)
     float2* part_ml;            // [B][Tq][16][Hq]: (row max m * c, row sum l) of each slot's partial
     __half* part_o;             // [B][Tq][16][Hkv] blocks of 2 KB: [half][8-dim chunk][8 heads][8 dims]
 };
@@ -167,31 +184,35 @@ __global__ void ap_fill_kernel(const Problem p, const ApWork w) {
     }
 }
 
-// One thread per item (b, kvh, n): its tiles' entries in the tile table, so that the
-// attention kernel reads one 16-byte record per tile instead of walking the prefix sums.
+// One warp per item (b, kvh, n), one lane per tile: the tile's record (item, coordinates,
+// tokens, clamped L, the next item's first tile and its 16 list entries), so that the attention
+// kernel fetches one 96-byte record per tile with one bulk copy.
 __global__ void ap_tiles_kernel(const Problem p, const ApWork w) {
     pdl_wait();
     pdl_launch_dependents();
-    const int64_t item = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t item = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
     if (item >= (int64_t)p.B * p.Hkv * p.nbmax) return;
     const int64_t n = item % p.nbmax, b = item / (p.nbmax * p.Hkv);
     const int64_t ln = b * p.nbmax + n;
     const int cnt = w.cnt[ln], off = w.list_off[ln], t0 = w.tile_start[item];
     const int L = (int)clamp_len(p.seq_lens[b], p.Tq, p.lmax, nullptr);
-    for (int j = 0; j * kApTok < cnt; ++j)
-        w.tiles[t0 + j] = make_int4((int)item, off + j * kApTok, min(kApTok, cnt - j * kApTok), L);
+    const int next = w.tile_start[item + 1];
+    const int kvh = (int)((item / p.nbmax) % p.Hkv);
+    for (int j = lane; j * kApTok < cnt; j += 32) {
+        const int ntok = min(kApTok, cnt - j * kApTok);
+        int e[kApTok];
+#pragma unroll
+        for (int k = 0; k < kApTok; ++k) e[k] = k < ntok ? w.list[off + j * kApTok + k] : 0;
+        int4* r = reinterpret_cast<int4*>(w.recs + t0 + j);
+        r[0] = make_int4((int)item, (int)b, kvh, (int)n);
+        r[1] = make_int4(ntok, L, next, 0);
+#pragma unroll
+        for (int k = 0; k < kApTok; k += 4) r[2 + k / 4] = make_int4(e[k], e[k + 1], e[k + 2], e[k + 3]);
+    }
 }
 
 // ------------------------------------------------------------------ block-major attention
-
-// One tile as the producer warp publishes it to the MMA thread and the softmax warps.
-struct ApTileInfo {
-    int32_t item, b, kvh, n, ntok, L;
-    int32_t seq;  // the item's number among this CTA's items (selects its K/V buffer)
-    int32_t pad;
-    int32_t entry[kApTok];  // t * 16 + slot of the tile's tokens
-};
-static_assert(sizeof(ApTileInfo) == 96, "tile record layout");
 
 // TMA load of a 4-D box with an L2 eviction-priority hint (no multicast).
 __device__ __forceinline__ void tma_load_4d_hint(void* dst, const void* tmap, int c0, int c1, int c2, int c3,
@@ -215,40 +236,47 @@ __device__ __forceinline__ uint32_t f16x2_to_bf16x2(uint32_t h) {
     return *reinterpret_cast<const uint32_t*>(&b);
 }
 
-// One thread's V share (of 128) of a raw NVFP4 block, read into registers so that the raw
-// buffer can be refilled while V^T is converted: keys 8 (tid / 8) + a, dims 16 (tid % 8) .. + 15.
-struct ApRawV {
+// One thread's share (of 128) of an NVFP4 block (128 keys of one KV head), loaded straight
+// from the caches into registers (read-only path; the caches hold whole 128-key blocks):
+// K words i = 0..15 cover keys (tid + 128 i) / 16, dims 8 ((tid + 128 i) % 16) .. + 7 (the
+// 128 threads read 512 contiguous bytes per i); V keys 8 (tid / 8) + a, dims 16 (tid % 8) .. + 15.
+struct ApRawShare {
+    uint32_t kw[16], ks[16];
     uint2 vx[8];
     uint32_t vs[8];
 };
 
-__device__ __forceinline__ void ap_raw_read_v(ApRawV& r, const uint8_t* raw, int nvalid, int tid) {
+__device__ __forceinline__ void ap_raw_load(ApRawShare& r, const Problem& p, int64_t vec, int tid) {
+    const uint8_t* kd = p.k.data + vec * 64;
+    const uint8_t* kscale = p.k.scale + vec * 8;
+    const uint8_t* vd = p.v.data + vec * 64;
+    const uint8_t* vscale = p.v.scale + vec * 8;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int q = tid + 128 * i;
+        r.kw[i] = __ldg(reinterpret_cast<const uint32_t*>(kd) + q);
+        r.ks[i] = __ldg(kscale + (q >> 4) * 8 + ((q & 15) >> 1));
+    }
     const int w16 = tid & 7, kg = tid >> 3;
 #pragma unroll
     for (int a = 0; a < 8; ++a) {
         const int key = kg * 8 + a;
-        r.vx[a] = *reinterpret_cast<const uint2*>(raw + kRawV + key * 64 + w16 * 8);
-        r.vs[a] = raw[kRawVs + key * 8 + w16];
-        if (key >= nvalid) {
-            r.vx[a] = make_uint2(0u, 0u);
-            r.vs[a] = 0u;
-        }
+        r.vx[a] = __ldg(reinterpret_cast<const uint2*>(vd + key * 64 + w16 * 8));
+        r.vs[a] = __ldg(vscale + key * 8 + w16);
     }
 }
 
-// K, bf16 [key][dim], 128-byte swizzle, K-major (e2m1 x e4m3 is exact in bf16), straight from
-// the raw block; keys at or past nvalid become zeros.
-__device__ __forceinline__ void ap_dequant_k(uint8_t* kt, const uint8_t* raw, int nvalid, int tid) {
-#pragma unroll 4
+// K, bf16 [key][dim], 128-byte swizzle, K-major (e2m1 x e4m3 is exact in bf16); keys at or
+// past nvalid become zeros.
+__device__ __forceinline__ void ap_dequant_k(uint8_t* kt, const ApRawShare& r, int nvalid, int tid) {
+#pragma unroll
     for (int i = 0; i < 16; ++i) {
         const int q = tid + 128 * i;
         const int j = q >> 4, cr = q & 15;  // key j, dims 8 cr .. 8 cr + 7
-        uint32_t kw = *reinterpret_cast<const uint32_t*>(raw + kRawK + j * 64 + cr * 4);
-        uint32_t ks = raw[kRawKs + j * 8 + (cr >> 1)];
-        if (j >= nvalid) kw = ks = 0u;
+        const bool live = j < nvalid;
         uint32_t h[4];
-        e2m1x8_to_f16x8(kw, h[0], h[1], h[2], h[3]);
-        const uint32_t s2 = e4m3_bcast_f16x2(ks);
+        e2m1x8_to_f16x8(live ? r.kw[i] : 0u, h[0], h[1], h[2], h[3]);
+        const uint32_t s2 = e4m3_bcast_f16x2(live ? r.ks[i] : 0u);
         uint4 o;
         o.x = f16x2_to_bf16x2(hmul2(h[0], s2));
         o.y = f16x2_to_bf16x2(hmul2(h[1], s2));
@@ -260,17 +288,20 @@ __device__ __forceinline__ void ap_dequant_k(uint8_t* kt, const uint8_t* raw, in
 
 // V^T, f16 [dim][key] divided by 128, 128-byte swizzle, K-major: thread = (dims 16 w16 ..
 // 16 w16 + 15, keys 8 kg .. 8 kg + 7), written as 16 rows x one 16-byte chunk.
-__device__ __forceinline__ void ap_dequant_vt(uint8_t* vt, const ApRawV& r, int tid) {
+__device__ __forceinline__ void ap_dequant_vt(uint8_t* vt, const ApRawShare& r, int nvalid, int tid) {
     const int w16 = tid & 7, kg = tid >> 3;
     uint32_t rows[16][4];  // [dim 16 w16 + r][key pair i]
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         // (key 2i, key 2i+1) scales times 2^-7: V^T is stored divided by 128 (exact in f16: every
         // product stays a multiple of 2^-24 below 2^11), so P V is O / 128 and fits f16 unnormalised
-        const uint32_t sc = hmul2(e4m3x2_to_f16x2(r.vs[2 * i] | (r.vs[2 * i + 1] << 8)), 0x20002000u);
+        const bool l0 = kg * 8 + 2 * i < nvalid, l1 = kg * 8 + 2 * i + 1 < nvalid;
+        const uint32_t sc =
+            hmul2(e4m3x2_to_f16x2((l0 ? r.vs[2 * i] : 0u) | ((l1 ? r.vs[2 * i + 1] : 0u) << 8)), 0x20002000u);
 #pragma unroll
         for (int hw = 0; hw < 2; ++hw) {
-            const uint32_t A = hw ? r.vx[2 * i].y : r.vx[2 * i].x, Bw = hw ? r.vx[2 * i + 1].y : r.vx[2 * i + 1].x;
+            const uint32_t A = l0 ? (hw ? r.vx[2 * i].y : r.vx[2 * i].x) : 0u;
+            const uint32_t Bw = l1 ? (hw ? r.vx[2 * i + 1].y : r.vx[2 * i + 1].x) : 0u;
             const uint32_t ev = (A & 0x0F0F0F0Fu) | ((Bw << 4) & 0xF0F0F0F0u);  // byte k: dim 8 hw + 2k
             const uint32_t od = ((A >> 4) & 0x0F0F0F0Fu) | (Bw & 0xF0F0F0F0u);  // byte k: dim 8 hw + 2k + 1
             uint32_t e[4], o[4];
@@ -345,35 +376,32 @@ __global__ void __launch_bounds__(kApThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bar = reinterpret_cast<uint64_t*>(smem + kOffBar);
-    uint64_t* raw_full = bar + 0;
-    uint64_t* raw_empty = bar + 1;
-    uint64_t* k_full = bar + 2;       // [2 item buffers]
-    uint64_t* v_full = bar + 4;       // [2]
-    uint64_t* kv_empty = bar + 6;     // [2]
-    uint64_t* q_full = bar + 8;       // [2 query stages = tile parities]
-    uint64_t* q_empty = bar + 10;     // [2]
+    uint64_t* q_full = bar + 0;       // [query stages]
+    uint64_t* q_empty = bar + 3;      // [query stages]
+    uint64_t* k_full = bar + 6;       // [2 item buffers]
+    uint64_t* v_full = bar + 8;       // [2]
+    uint64_t* kv_empty = bar + 10;    // [2]
     uint64_t* s_full = bar + 12;      // [2 warpgroups = tile parities]
     uint64_t* p_full = bar + 14;      // [2]
     uint64_t* o_full = bar + 16;      // [2]
     uint64_t* o_empty = bar + 18;     // [2]
-    uint64_t* info_full = bar + 20;   // [4]
-    uint64_t* info_empty = bar + 24;  // [4]
-    uint64_t* done = bar + 28;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 29);
+    uint64_t* info_full = bar + 20;   // [8]
+    uint64_t* info_empty = bar + 28;  // [8]
+    uint64_t* done = bar + 36;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 37);
     ApTileInfo* info = reinterpret_cast<ApTileInfo*>(smem + kOffInfo);
-    uint8_t* raw = smem + kOffRaw;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     pdl_wait();
     if (threadIdx.x == 0) {
-        mbar_init(raw_full, 1);
-        mbar_init(raw_empty, 4);  // the 4 dequantising warps have read the block
+        for (int s = 0; s < kApQStages; ++s) {
+            mbar_init(&q_full[s], 1);
+            mbar_init(&q_empty[s], 1);
+        }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&k_full[s], 4);
             mbar_init(&v_full[s], 4);
             mbar_init(&kv_empty[s], 1);
-            mbar_init(&q_full[s], 1);
-            mbar_init(&q_empty[s], 1);
             mbar_init(&s_full[s], 1);
             mbar_init(&p_full[s], 4);
             mbar_init(&o_full[s], 1);
@@ -381,7 +409,7 @@ __global__ void __launch_bounds__(kApThreads, 1)
         }
         for (int s = 0; s < kApInfoSlots; ++s) {
             mbar_init(&info_full[s], 1);
-            mbar_init(&info_empty[s], 4 + 1);  // the tile's warpgroup and the MMA thread
+            mbar_init(&info_empty[s], 4 + 2);  // the tile's warpgroup, the MMA thread, the producer
         }
         mbar_init(done, 1);
         fence_mbar_init();
@@ -396,8 +424,11 @@ __global__ void __launch_bounds__(kApThreads, 1)
     const uint32_t tmem = *tmem_slot;
     pdl_launch_dependents();
 
+    // Data written by the kernels just before this one (launched as programmatic dependents) is read
+    // on the L2 path (ld.global.cg): a plain load could hit a line left in this SM's L1 by an earlier
+    // step that used the same workspace.
     const int64_t items = (int64_t)p.B * p.Hkv * p.nbmax;
-    const int total = w.tile_start[items];
+    const int total = __ldcg(w.tile_start + items);
     const int t0 = (int)((int64_t)total * blockIdx.x / gridDim.x);
     const int t1 = (int)((int64_t)total * (blockIdx.x + 1) / gridDim.x);
     const int ntiles = t1 - t0;
@@ -405,204 +436,193 @@ __global__ void __launch_bounds__(kApThreads, 1)
     auto fail = [&]() { set_status(p.status, MSA_STATUS_TIMEOUT | MSA_STATUS_AT_ATTEND); };
 
     if (warp == kApTmaWarp) {
-        // ------------------------------------------------------------ producer warp: tile records and query
-        // rows.  The tile record of tile tau + 2 and the token ids of tile tau + 1 are loaded while tile tau
-        // is issued, so no global-load latency sits between two tiles.
+        // ------------------------------------------------------------ producer warp: tile records (bulk copies
+        // kApRecAhead tiles ahead into the 8-slot ring) and each tile's query rows (TMA, one 8-row atom per
+        // token, from 16 lanes).  No global load sits on this warp's path.
         if (ntiles > 0) {
             const uint64_t pol = l2_policy_evict_last();  // the queries are re-read by many tiles
-            int4 m0 = w.tiles[t0];
-            int4 m1 = t0 + 1 < t1 ? w.tiles[t0 + 1] : make_int4(0, 0, 0, 0);
-            int e0 = lane < m0.z ? w.list[m0.y + lane] : 0;
-            int cur = -1, seq = -1, issued = 0;
+            int recs = 0, seen = 0, issued = 0;  // records copied, records read here, query tiles issued
             bool ok = true;
-            for (int tau = t0; tau < t1 && ok; ++tau) {
-                const int i = tau - t0, sb = i & 1, s4 = i & (kApInfoSlots - 1);
-                const int e1 = (tau + 1 < t1 && lane < m1.z) ? w.list[m1.y + lane] : 0;
-                const int4 m2 = tau + 2 < t1 ? w.tiles[tau + 2] : make_int4(0, 0, 0, 0);
-                const int item = m0.x, ntok = m0.z;
-                const int n = item % (int)p.nbmax, bk = item / (int)p.nbmax;
-                const int kvh = bk % p.Hkv, b = bk / p.Hkv;
-                if (item != cur) {
-                    cur = item;
-                    ++seq;
-                }
-                if (lane == 0) {
-                    if (i >= kApInfoSlots && !mbar_wait(&info_empty[s4], ((i >> 2) - 1) & 1)) ok = false;
-                    if (ok && i >= 2 && !mbar_wait(&q_empty[sb], ((i >> 1) - 1) & 1)) ok = false;
-                }
+            auto copy_rec = [&](int j) -> bool {  // lane 0: record of tile j into slot j & 7
+                const int s8 = j & (kApInfoSlots - 1);
+                if (j >= kApInfoSlots && !mbar_wait(&info_empty[s8], ((j >> 3) - 1) & 1)) return false;
+                mbar_arrive_expect_tx(&info_full[s8], (uint32_t)sizeof(ApTileInfo));
+                bulk_g2s(info + s8, w.recs + t0 + j, (uint32_t)sizeof(ApTileInfo), &info_full[s8]);
+                return true;
+            };
+            if (lane == 0)
+                for (; recs < min(kApRecAhead, ntiles) && ok; ++recs) ok = copy_rec(recs);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            for (int i = 0; i < ntiles && ok; ++i) {
+                const int sb = i % kApQStages, s8 = i & (kApInfoSlots - 1);
+                if (lane == 0 && i >= kApQStages && !mbar_wait(&q_empty[sb], ((i / kApQStages) - 1) & 1)) ok = false;
                 ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) break;
-                if (lane < kApTok) info[s4].entry[lane] = e0;
-                if (lane == 0) {
-                    info[s4].item = item;
-                    info[s4].b = b;
-                    info[s4].kvh = kvh;
-                    info[s4].n = n;
-                    info[s4].ntok = ntok;
-                    info[s4].L = m0.w;
-                    info[s4].seq = seq;
+                if (!ok || !__all_sync(0xffffffffu, mbar_wait(&info_full[s8], (i >> 3) & 1))) {
+                    ok = false;
+                    break;
                 }
+                seen = i + 1;
+                const int ntok = info[s8].ntok, b = info[s8].b, kvh = info[s8].kvh;
+                const int e = lane < kApTok ? info[s8].entry[lane] : 0;
                 __syncwarp();
                 if (lane == 0) {
-                    mbar_arrive(&info_full[s4]);
+                    mbar_arrive(&info_empty[s8]);
                     mbar_arrive_expect_tx(&q_full[sb], (uint32_t)(ntok * 2 * 1024));
                 }
                 __syncwarp();
                 if (lane < ntok) {  // each lane gathers one token's 8 query heads
-                    const int t = e0 / kTopK;
+                    const int t = e / kTopK;
                     uint8_t* qs = smem + kOffQ + sb * kApTile + lane * 1024;
                     tma_load_4d_hint(qs, &tmap, 0, kvh * kApG, t, b, &q_full[sb], pol);
                     tma_load_4d_hint(qs + kApKB, &tmap, 64, kvh * kApG, t, b, &q_full[sb], pol);
                 }
                 issued = i + 1;
-                m0 = m1;
-                m1 = m2;
-                e0 = e1;
+                if (lane == 0 && recs < ntiles) ok = copy_rec(recs++);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
             }
             if (!ok && lane == 0) fail();
             // never leave with copies in flight into this CTA's shared memory
-            if (lane == 0)
-                for (int i = max(0, issued - 2); i < issued; ++i)
-                    if (!mbar_wait(&q_full[i & 1], (i >> 1) & 1)) {
+            if (lane == 0) {
+                for (int i = max(0, issued - kApQStages); i < issued; ++i)
+                    if (!mbar_wait(&q_full[i % kApQStages], (i / kApQStages) & 1)) {
                         fail();
                         break;
                     }
+                for (int j = seen; j < recs; ++j)
+                    if (!mbar_wait(&info_full[j & (kApInfoSlots - 1)], (j >> 3) & 1)) {
+                        fail();
+                        break;
+                    }
+            }
         }
     } else if (warp >= kApDqWarp && warp < kApDqWarp + 4) {
         // ------------------------------------------------------------ dequantising warpgroup: every item of
-        // this CTA in order, into item buffer seq & 1 (free once the PV MMAs of item seq - 2 are done): the
-        // thread's V share of the raw block goes to registers, K is converted from the raw block (the S MMAs
-        // wait for K only), the raw buffer is released (the next block streams in meanwhile), then V^T.
+        // this CTA in order, into item buffer seq & 1 (free once the P V MMAs of item seq - 2 are done).  The
+        // block's NVFP4 bytes are loaded into registers before that wait, so their latency overlaps it; K is
+        // written first (the S MMAs wait for K only), then V^T.
         if (ntiles > 0) {
             const int tid = threadIdx.x - 32 * kApDqWarp;
             auto wait_all = [&](uint64_t* b_, uint32_t parity) -> bool {
                 return __all_sync(0xffffffffu, mbar_wait(b_, parity)) != 0;
             };
-            int cur = -1, seq = -1;
+            int seq = -1;
             bool ok = true;
-            int4 nxt = w.tiles[t0];
-            for (int tau = t0; tau < t1; ++tau) {
-                const int4 m = nxt;
-                if (tau + 1 < t1) nxt = w.tiles[tau + 1];
-                if (m.x == cur) continue;
-                cur = m.x;
+            for (int tau = t0; tau < t1;) {
+                const int item = __ldcg(&w.recs[tau].item), Lr = __ldcg(&w.recs[tau].L), next = __ldcg(&w.recs[tau].next);
+                tau = max(next, tau + 1);
                 ++seq;
                 const int kb = seq & 1;
-                if (!wait_all(raw_full, seq & 1) || (seq >= 2 && !wait_all(&kv_empty[kb], ((seq >> 1) - 1) & 1))) {
+                const int n = item % (int)p.nbmax, bk = item / (int)p.nbmax;
+                const int kvh = bk % p.Hkv, b = bk / p.Hkv;
+                const int nvalid = (int)min64(kBlock, max64(0, (int64_t)Lr - (int64_t)n * kBlock));
+                ApRawShare r;
+                ap_raw_load(r, p, block_vec<PAGED>(p, b, n, kvh, p.Hkv), tid);
+                if (seq >= 2 && !wait_all(&kv_empty[kb], ((seq >> 1) - 1) & 1)) {
                     ok = false;
                     break;
                 }
-                const int n = m.x % (int)p.nbmax;
-                const int nvalid = (int)min64(kBlock, max64(0, (int64_t)m.w - (int64_t)n * kBlock));
-                ApRawV r;
-                ap_raw_read_v(r, raw, nvalid, tid);
                 uint8_t* kvb = smem + kOffKV + kb * 2 * kApTile;
-                ap_dequant_k(kvb, raw, nvalid, tid);
+                ap_dequant_k(kvb, r, nvalid, tid);
                 fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(raw_empty);  // every read of the raw block is done
-                    mbar_arrive(&k_full[kb]);
-                }
-                ap_dequant_vt(kvb + kApTile, r, tid);
+                if (lane == 0) mbar_arrive(&k_full[kb]);
+                ap_dequant_vt(kvb + kApTile, r, nvalid, tid);
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&v_full[kb]);
             }
             if (!ok && lane == 0) fail();
         }
-    } else if (warp == kApRawWarp) {
-        // ------------------------------------------------------------ raw-block loader (one thread): each
-        // item's NVFP4 K and V block (bulk copies), as soon as the previous item has been dequantised, so
-        // that the copy runs while the tiles of that item are computed.
-        if (lane == 0 && ntiles > 0) {
-            int cur = -1, seq = -1;
-            bool ok = true;
-            int nxt = w.tiles[t0].x;
-            for (int tau = t0; tau < t1; ++tau) {
-                const int item = nxt;
-                if (tau + 1 < t1) nxt = w.tiles[tau + 1].x;
-                if (item == cur) continue;
-                cur = item;
-                ++seq;
-                if (seq >= 1 && !mbar_wait(raw_empty, (seq - 1) & 1)) {
-                    ok = false;
-                    break;
-                }
-                const int n = item % (int)p.nbmax, bk = item / (int)p.nbmax;
-                const int kvh = bk % p.Hkv, b = bk / p.Hkv;
-                const int64_t vec = block_vec<PAGED>(p, b, n, kvh, p.Hkv);
-                mbar_arrive_expect_tx(raw_full, 2 * (8192 + 1024));
-                bulk_g2s(raw + kRawK, p.k.data + vec * 64, 8192, raw_full);
-                bulk_g2s(raw + kRawKs, p.k.scale + vec * 8, 1024, raw_full);
-                bulk_g2s(raw + kRawV, p.v.data + vec * 64, 8192, raw_full);
-                bulk_g2s(raw + kRawVs, p.v.scale + vec * 8, 1024, raw_full);
-            }
-            if (!ok) fail();
-            if (seq >= 0 && !mbar_wait(raw_full, seq & 1)) fail();  // the last copy has landed
-        }
     } else if (warp == kApMmaWarp) {
-        // ------------------------------------------------------------ MMA issuer (one thread).  Order:
-        // S(0), S(1), PV(0), S(2), PV(1), ...: S(i) reuses the TMEM columns that held P(i - 2), which
-        // PV(i - 2), issued earlier by this thread, reads first (tcgen05.mma runs in issue order).
+        // ------------------------------------------------------------ MMA issuer (one thread), scheduled by
+        // readiness: P V(j) as soon as P(j), V and O(j & 1) are ready, S(i) as soon as its record, K and Q(i)
+        // are, so that neither waits behind the other.  S(i) reuses the TMEM columns that held P(i - 2), so it
+        // is issued only after P V(i - 2) (tcgen05.mma runs in issue order).  Polls are non-blocking; no
+        // progress for the wait limit ends the loop with a timeout status.
         if (lane == 0 && ntiles > 0) {
             constexpr uint32_t idesc_s = umma_idesc_bf16_f32(128, 128);
             constexpr uint32_t idesc_o = umma_idesc_f16_f32(128, 128);
-            int kseq = -1, vseq = -1, seq_prev = -1;
-            auto pv = [&](int j, int seq_j, bool last_of_item) -> bool {
-                const int g = j & 1;
-                if (!mbar_wait(&p_full[g], (j >> 1) & 1)) return false;
-                if (seq_j != vseq) {
-                    if (!mbar_wait(&v_full[seq_j & 1], (seq_j >> 1) & 1)) return false;
-                    vseq = seq_j;
-                }
-                if (j >= 2 && !mbar_wait(&o_empty[g], ((j >> 1) - 1) & 1)) return false;
-                tcgen05_fence_after();
-                const uint32_t vt = smem_u32(smem + kOffKV + (seq_j & 1) * 2 * kApTile + kApTile);
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    umma_f16_ts(tmem + 256 + g * 128, tmem + g * 128 + k * 8,
-                                umma_desc_k_sw128(vt + (k >> 2) * kApKB + (k & 3) * 32), idesc_o, k > 0 ? 1u : 0u);
-                umma_commit(&o_full[g]);
-                if (last_of_item) umma_commit(&kv_empty[seq_j & 1]);  // every MMA reading the item's K and V
-                return true;
-            };
+            int ns = 0, npv = 0;             // next S tile, next P V tile
+            int cur = -1, seq = -1;          // item of the last record read, its number in this CTA
+            int kseq = -1, vseq = -1;        // last item whose K / V readiness was seen
+            int sseq = -1;                   // item number of tile ns once its record is read (-1: not yet)
+            int pend = -1;                   // item whose last P V went out before the next record was read
+            int seq_of[4] = {0, 0, 0, 0};    // item number of S-issued tiles (at most 2 ahead of P V)
             bool ok = true;
-            for (int i = 0; i < ntiles; ++i) {
-                const int g = i & 1, s4 = i & (kApInfoSlots - 1);
-                if (!mbar_wait(&info_full[s4], (i >> 2) & 1)) {
-                    ok = false;
-                    break;
-                }
-                const int seq = info[s4].seq;
-                mbar_arrive(&info_empty[s4]);
-                if (seq != kseq) {
-                    if (!mbar_wait(&k_full[seq & 1], (seq >> 1) & 1)) {
-                        ok = false;
-                        break;
-                    }
-                    kseq = seq;
-                }
-                if (!mbar_wait(&q_full[g], (i >> 1) & 1)) {
-                    ok = false;
-                    break;
-                }
-                tcgen05_fence_after();
-                const uint32_t qa = smem_u32(smem + kOffQ + g * kApTile);
-                const uint32_t kt = smem_u32(smem + kOffKV + (seq & 1) * 2 * kApTile);
+            uint64_t last = globaltimer_ns();
+            while (npv < ntiles) {
+                bool progress = false;
+                // ---- P V(npv)
+                if (npv < ns) {
+                    const int j = npv, g = j & 1, sj = seq_of[j & 3];
+                    if (mbar_test(&p_full[g], (j >> 1) & 1) && (sj == vseq || mbar_test(&v_full[sj & 1], (sj >> 1) & 1)) &&
+                        (j < 2 || mbar_test(&o_empty[g], ((j >> 1) - 1) & 1))) {
+                        vseq = sj;
+                        tcgen05_fence_after();
+                        const uint32_t vt = smem_u32(smem + kOffKV + (sj & 1) * 2 * kApTile + kApTile);
 #pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    umma_bf16_ss(tmem + g * 128, umma_desc_k_sw128(qa + (k >> 2) * kApKB + (k & 3) * 32),
-                                 umma_desc_k_sw128(kt + (k >> 2) * kApKB + (k & 3) * 32), idesc_s, k > 0 ? 1u : 0u);
-                umma_commit(&q_empty[g]);
-                umma_commit(&s_full[g]);
-                if (i >= 1 && !pv(i - 1, seq_prev, seq != seq_prev)) {
+                        for (int k = 0; k < 8; ++k)
+                            umma_f16_ts(tmem + 256 + g * 128, tmem + g * 128 + k * 8,
+                                        umma_desc_k_sw128(vt + (k >> 2) * kApKB + (k & 3) * 32), idesc_o,
+                                        k > 0 ? 1u : 0u);
+                        umma_commit(&o_full[g]);
+                        // the item's K and V buffer is free once its last P V is done
+                        if (j + 1 < ns) {
+                            if (seq_of[(j + 1) & 3] != sj) umma_commit(&kv_empty[sj & 1]);
+                        } else if (sseq >= 0) {  // tile j + 1 = ns: its record is read already
+                            if (sseq != sj) umma_commit(&kv_empty[sj & 1]);
+                        } else if (j + 1 < ntiles) {
+                            pend = sj;  // decided when tile j + 1's record is read
+                        }
+                        ++npv;
+                        progress = true;
+                    }
+                }
+                // ---- S(ns)
+                if (ns < ntiles && npv >= ns - 1) {
+                    const int i = ns, g = i & 1, s8 = i & (kApInfoSlots - 1);
+                    if (sseq < 0 && mbar_test(&info_full[s8], (i >> 3) & 1)) {
+                        const int item = info[s8].item;
+                        mbar_arrive(&info_empty[s8]);
+                        if (item != cur) {
+                            cur = item;
+                            ++seq;
+                        }
+                        sseq = seq;
+                        if (pend >= 0) {
+                            if (pend != sseq) umma_commit(&kv_empty[pend & 1]);
+                            pend = -1;
+                        }
+                        progress = true;
+                    }
+                    if (sseq >= 0 && (sseq == kseq || mbar_test(&k_full[sseq & 1], (sseq >> 1) & 1)) &&
+                        mbar_test(&q_full[i % kApQStages], (i / kApQStages) & 1)) {
+                        kseq = sseq;
+                        tcgen05_fence_after();
+                        const uint32_t qa = smem_u32(smem + kOffQ + (i % kApQStages) * kApTile);
+                        const uint32_t kt = smem_u32(smem + kOffKV + (sseq & 1) * 2 * kApTile);
+#pragma unroll
+                        for (int k = 0; k < 8; ++k)
+                            umma_bf16_ss(tmem + g * 128, umma_desc_k_sw128(qa + (k >> 2) * kApKB + (k & 3) * 32),
+                                         umma_desc_k_sw128(kt + (k >> 2) * kApKB + (k & 3) * 32), idesc_s,
+                                         k > 0 ? 1u : 0u);
+                        umma_commit(&q_empty[i % kApQStages]);
+                        umma_commit(&s_full[g]);
+                        seq_of[i & 3] = sseq;
+                        sseq = -1;
+                        ++ns;
+                        progress = true;
+                    }
+                }
+                if (progress) {
+                    last = globaltimer_ns();
+                } else if (globaltimer_ns() - last > kWaitLimitNs) {
                     ok = false;
                     break;
+                } else {
+                    __nanosleep(32);  // leave the issue slots to the warps that compute
                 }
-                seq_prev = seq;
             }
-            if (ok && !pv(ntiles - 1, seq_prev, false)) ok = false;
             if (!ok) fail();
             // every MMA issued has completed before the CTA releases its tensor memory
             umma_commit(done);
@@ -621,17 +641,17 @@ __global__ void __launch_bounds__(kApThreads, 1)
         };
         bool ok = true;
         for (int i = g; i < ntiles; i += 2) {
-            const int s4 = i & (kApInfoSlots - 1);
-            if (!wait_all(&info_full[s4], (i >> 2) & 1)) {
+            const int s8 = i & (kApInfoSlots - 1);
+            if (!wait_all(&info_full[s8], (i >> 3) & 1)) {
                 ok = false;
                 break;
             }
-            const ApTileInfo& ti = info[s4];
+            const ApTileInfo& ti = info[s8];
             const int n = ti.n, b = ti.b, kvh = ti.kvh, ntok = ti.ntok;
             const int64_t L = ti.L;
             const int e = tslot < ntok ? ti.entry[tslot] : 0;
             __syncwarp();
-            if (lane == 0) mbar_arrive(&info_empty[s4]);
+            if (lane == 0) mbar_arrive(&info_empty[s8]);
             int kvis = 0;  // visible keys of the row's block (0: no token in this tile row)
             int64_t orow = -1;
             if (tslot < ntok) {
@@ -787,7 +807,7 @@ constexpr size_t kApAlign = 256;
 size_t ap_round(size_t x) { return (x + kApAlign - 1) / kApAlign * kApAlign; }
 
 struct ApLayout {
-    size_t cnt, cursor, off, tstart, list, tiles, lse, po, total;
+    size_t cnt, cursor, off, tstart, list, recs, lse, po, total;
 };
 
 ApLayout ap_layout(const Problem& p) {
@@ -804,8 +824,8 @@ ApLayout ap_layout(const Problem& p) {
     at += ap_round((items + 1) * 4);
     a.list = at;
     at += ap_round(entries * 4);
-    a.tiles = at;
-    at += ap_round(entries * p.Hkv * sizeof(int4));
+    a.recs = at;  // tiles <= sum over items of (listed tokens / 16 + 1)
+    at += ap_round((entries * p.Hkv / kApTok + items + 1) * sizeof(ApTileInfo));
     a.lse = at;
     at += ap_round(entries * p.Hq * sizeof(float2));
     a.po = at;
@@ -877,7 +897,7 @@ int launch_attend_prefill(const Problem& p, const int32_t* sel, void* ws, float*
     w.list_off = reinterpret_cast<int32_t*>(base + a.off);
     w.tile_start = reinterpret_cast<int32_t*>(base + a.tstart);
     w.list = reinterpret_cast<int32_t*>(base + a.list);
-    w.tiles = reinterpret_cast<int4*>(base + a.tiles);
+    w.recs = reinterpret_cast<ApTileInfo*>(base + a.recs);
     w.part_ml = reinterpret_cast<float2*>(base + a.lse);
     w.part_o = reinterpret_cast<__half*>(base + a.po);
     const int64_t entries = (int64_t)p.B * p.Tq * kTopK;
@@ -891,7 +911,7 @@ int launch_attend_prefill(const Problem& p, const int32_t* sel, void* ws, float*
     cfg = ap_config(eg, dim3(256), 0, pdl, st, attr);
     if (cudaLaunchKernelEx(&cfg, ap_fill_kernel, p, w) != cudaSuccess) return MSA_ECUDA;
     const int64_t items = (int64_t)p.B * p.Hkv * p.nbmax;
-    cfg = ap_config(dim3((unsigned)((items + 255) / 256)), dim3(256), 0, pdl, st, attr);
+    cfg = ap_config(dim3((unsigned)((items * 32 + 255) / 256)), dim3(256), 0, pdl, st, attr);
     if (cudaLaunchKernelEx(&cfg, ap_tiles_kernel, p, w) != cudaSuccess) return MSA_ECUDA;
     const int r = p.block_table != nullptr ? launch_ap_attend<true>(p, w, pdl, st) : launch_ap_attend<false>(p, w, pdl, st);
     if (r != MSA_OK) return r;
