@@ -175,8 +175,8 @@ int msa_nvfp4_amax(const float* x, int64_t n, float* amax_out, cudaStream_t stre
 /* Bytes of scratch msa_decode needs for this problem (0 on invalid params): the pooled
  * block scores and the selection; for chunked prefill (Tq * HI > 32) with Hq = 8 * Hkv
  * also the per-block token lists and the per-(token, selected block) attention partials
- * of the tensor-core prefill attention, B * Tq * 16 * Hq * (2 D + 4) bytes and more
- * (about 1.07 GB for 2 sequences x 4,096 tokens x 32 heads). */
+ * of the tensor-core prefill attention, B * Tq * 16 * Hq * (2 D + 8) bytes and more
+ * (about 1.15 GB for 2 sequences x 4,096 tokens x 32 heads on a 128K context). */
 size_t msa_workspace_size(const msa_params_t* p);
 
 /* Indexer + block pooling: streams every visible NVFP4 index key once.
