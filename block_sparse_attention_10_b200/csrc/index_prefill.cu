@@ -259,14 +259,25 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(k_ready);
             }
-            for (int qt = qc * kPfQChunk; qt < qt_end; ++qt) {
-                const int row = quad * 32 + lane;
-                const int R = qt * kPfRows + row;
-                const int t = R / HI, h = R % HI;
+            // Per tile, the row's token moves on by kPfRows / HI and its head stays the same, so the
+            // token, its count of visible keys in this warp's block and its score address step by
+            // constants (32-bit where the values are bounded by a block); the tail between tiles
+            // is then the head sum and one store.
+            const int row = quad * 32 + lane;
+            const int h = row % HI;  // kPfRows is a multiple of HI
+            const int q0 = qc * kPfQChunk;
+            int t = (q0 * kPfRows + row) / HI;
+            // visible keys of block n for token t: L - Tq + t + 1 - n * 128, clamped to [0, 128]
+            const int64_t vis0 = L - Tq + 1 - n * kBlock;
+            const bool n_ok = n < nb_b;
+            const float wrow = p.w_idx != nullptr;  // weights are read per token below
+            float* dst = block_scores + ((int64_t)b * Tq + t) * p.nbmax + n;
+            const int64_t dst_step = (int64_t)(kPfRows / HI) * p.nbmax;
+            for (int qt = q0; qt < qt_end; ++qt, t += kPfRows / HI, dst += dst_step) {
                 const bool live = pf_tile_live<HI>(qt, k0, L, Tq);
+                const bool t_ok = t < Tq && n_ok;
+                const int cnt = t_ok ? (int)min64(kBlock, max64(0, vis0 + t)) : 0;
                 float sum = 0.0f;
-                int64_t cnt = 0;
-                if (t < Tq && n < nb_b) cnt = min64(kBlock, max64(0, L - Tq + t + 1 - n * kBlock));
                 if (live) {
                     const int buf = (int)(qi & 1u);
                     if (!mbar_wait(&t_full[buf], (qi >> 1) & 1u)) {
@@ -306,11 +317,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     if (lane == 0) mbar_arrive(&t_empty[buf]);
                     ++qi;
                 }
-                float x = t < Tq ? sum * (p.w_idx ? p.w_idx[((int64_t)b * Tq + t) * HI + h] : 1.0f) : 0.0f;
+                float x = t < Tq ? sum * (wrow != 0.0f ? p.w_idx[((int64_t)b * Tq + t) * HI + h] : 1.0f) : 0.0f;
 #pragma unroll
                 for (int o = 1; o < HI; o <<= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-                if (h == 0 && t < Tq && n < nb_b)
-                    block_scores[((int64_t)b * Tq + t) * p.nbmax + n] = cnt > 0 ? (x / (float)cnt) * s_t : -INFINITY;
+                // mean over the visible keys; a full block divides by 128, a power of two (exact as a product)
+                if (h == 0 && t_ok)
+                    *dst = cnt == kBlock ? (x * (1.0f / kBlock)) * s_t : cnt > 0 ? (x / (float)cnt) * s_t : -INFINITY;
             }
         }
     }
