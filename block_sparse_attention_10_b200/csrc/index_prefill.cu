@@ -273,10 +273,12 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             const float wrow = p.w_idx != nullptr;  // weights are read per token below
             float* dst = block_scores + ((int64_t)b * Tq + t) * p.nbmax + n;
             const int64_t dst_step = (int64_t)(kPfRows / HI) * p.nbmax;
+            // the tile's visibility and key count, computed one tile ahead (they fill the latency of
+            // the previous tile's head sum)
+            bool live = q0 < qt_end && pf_tile_live<HI>(q0, k0, L, Tq);
+            bool t_ok = t < Tq && n_ok;
+            int cnt = t_ok ? (int)min64(kBlock, max64(0, vis0 + t)) : 0;
             for (int qt = q0; qt < qt_end; ++qt, t += kPfRows / HI, dst += dst_step) {
-                const bool live = pf_tile_live<HI>(qt, k0, L, Tq);
-                const bool t_ok = t < Tq && n_ok;
-                const int cnt = t_ok ? (int)min64(kBlock, max64(0, vis0 + t)) : 0;
                 float sum = 0.0f;
                 if (live) {
                     const int buf = (int)(qi & 1u);
@@ -317,12 +319,28 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     if (lane == 0) mbar_arrive(&t_empty[buf]);
                     ++qi;
                 }
-                float x = t < Tq ? sum * (wrow != 0.0f ? p.w_idx[((int64_t)b * Tq + t) * HI + h] : 1.0f) : 0.0f;
+                const float x = t < Tq ? sum * (wrow != 0.0f ? p.w_idx[((int64_t)b * Tq + t) * HI + h] : 1.0f) : 0.0f;
+                const bool st_ok = h == 0 && t_ok;
+                const int st_cnt = cnt;
+                {
+                    const int tn = t + kPfRows / HI;
+                    live = qt + 1 < qt_end && pf_tile_live<HI>(qt + 1, k0, L, Tq);
+                    t_ok = tn < Tq && n_ok;
+                    cnt = t_ok ? (int)min64(kBlock, max64(0, vis0 + tn)) : 0;
+                }
+                // head sum: the token's HI rows are HI consecutive lanes; every lane reads them at
+                // once (independent shuffles) and adds pairwise
+                float xs[HI];
 #pragma unroll
-                for (int o = 1; o < HI; o <<= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+                for (int o = 0; o < HI; ++o) xs[o] = __shfl_sync(0xffffffffu, x, (lane & ~(HI - 1)) + o);
+#pragma unroll
+                for (int w2 = HI / 2; w2 >= 1; w2 >>= 1)
+#pragma unroll
+                    for (int o = 0; o < w2; ++o) xs[o] += xs[o + w2];
                 // mean over the visible keys; a full block divides by 128, a power of two (exact as a product)
-                if (h == 0 && t_ok)
-                    *dst = cnt == kBlock ? (x * (1.0f / kBlock)) * s_t : cnt > 0 ? (x / (float)cnt) * s_t : -INFINITY;
+                if (st_ok)
+                    *dst = st_cnt == kBlock ? (xs[0] * (1.0f / kBlock)) * s_t
+                                            : st_cnt > 0 ? (xs[0] / (float)st_cnt) * s_t : -INFINITY;
             }
         }
     }
