@@ -715,89 +715,99 @@ __global__ void __launch_bounds__(kApThreads, 1)
 
 // ------------------------------------------------------------------ merge of the slot partials
 
-// One thread per (sequence, token, query head, 8 dims); the 128 threads of a (token, KV head)
-// read each slot's 2 KB partial block as one run and write the group's 8 heads x 128 dims of
-// output (one contiguous run) through shared memory.  All of a row's slot partials are
-// requested before any is combined (they are read once: streaming loads).  Partial s holds
-// O_s / 128 (unnormalised) with its row max m_s (scaled, log2 domain) and row sum l_s:
-//   out = s_V * sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s,  lse = ln 2 * (M + log2 sum ...).
-constexpr int kMergeThreads = 256;  // two (token, KV head) groups per block
+// One CTA of 128 threads per (sequence, token, KV head): one thread copies the group's valid
+// slot partials (2 KB blocks of 8 heads x 128 dims, O / 128 in f16) and their (m, l) pairs into
+// shared memory with bulk copies (one mbarrier), so the whole group is in flight at once without
+// holding it in registers; then thread (head, 8 dims) combines the slots in slot order:
+//   out = s_V * 128 * sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s,  lse = ln 2 * (M + log2 sum ...),
+// stages the group's [8 heads][128 dims] output over the slot buffer and writes it in order.
+constexpr int kMergeThreads = 128;
+constexpr int kMergeSlot = kApG * 128 * 2;  // bytes of one slot partial of a group
+constexpr size_t kMergeSmem = (size_t)kTopK * kMergeSlot + (size_t)kTopK * kApG * 8 + 16;
 __global__ void __launch_bounds__(kMergeThreads) ap_merge_kernel(const Problem p, const ApWork w,
                                                                  float* __restrict__ out, float* __restrict__ lse) {
-    __shared__ float stage[kMergeThreads / 128][kApG * 128 + 4];
+    extern __shared__ __align__(128) uint8_t msm[];
+    const uint4* slots = reinterpret_cast<const uint4*>(msm);                            // [slot][128 x 16 B]
+    const float2* mls = reinterpret_cast<const float2*>(msm + kTopK * kMergeSlot);       // [slot][8 heads]
+    uint64_t* full = reinterpret_cast<uint64_t*>(msm + kTopK * kMergeSlot + kTopK * kApG * 8);
     pdl_wait();
     pdl_launch_dependents();
-    const int64_t groups = (int64_t)p.B * p.Tq * p.Hkv;
-    const int64_t i = (int64_t)blockIdx.x * kMergeThreads + threadIdx.x;
-    const int gl = threadIdx.x >> 7;    // group within the block
-    const int j = threadIdx.x & 127;    // position in the 2 KB block: (half * 8 + chunk) * 8 + head
-    const int hh = j & 7, g8 = j >> 3;  // head within the group; 8-dim chunk of the 128 dims
-    const int64_t bk = i >> 7;          // (b * Tq + t) * Hkv + kvh
-    const bool live = bk < groups;
+    const int64_t bk = blockIdx.x;  // (b * Tq + t) * Hkv + kvh
+    const int j = threadIdx.x;      // position in the 2 KB block: (half * 8 + chunk) * 8 + head
+    const int hh = j & 7, g8 = j >> 3;
+    const int kvh = (int)(bk % p.Hkv);
+    const int64_t bt = bk / p.Hkv;
+    const int hq = kvh * kApG + hh;
+    const int b = (int)(bt / p.Tq), t = (int)(bt % p.Tq);
+    const int64_t L = clamp_len(p.seq_lens[b], p.Tq, p.lmax, nullptr);
+    const int64_t nvis = (L - p.Tq + t) / kBlock + 1;
+    const int4* selv = reinterpret_cast<const int4*>(w.sel + bt * kTopK);
+    uint32_t valid = 0;  // bit s: slot s holds a visible selected block
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int4 x = __ldg(selv + q);
+        const int id[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int r = 0; r < 4; ++r) valid |= (uint32_t)(id[r] >= 0 && id[r] < nvis) << (4 * q + r);
+    }
+    if (j == 0) {
+        mbar_init(full, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (j == 0) {
+        mbar_arrive_expect_tx(full, (uint32_t)__popc(valid) * (kMergeSlot + kApG * 8));
+        for (int s2 = 0; s2 < kTopK; ++s2) {
+            if (!((valid >> s2) & 1u)) continue;
+            const int64_t pr = bt * kTopK + s2;  // (token, slot)
+            bulk_g2s(msm + s2 * kMergeSlot, w.part_o + (pr * p.Hkv + kvh) * (kApG * 128), kMergeSlot, full);
+            bulk_g2s(msm + kTopK * kMergeSlot + s2 * kApG * 8, w.part_ml + pr * p.Hq + kvh * kApG, kApG * 8, full);
+        }
+    }
+    if (!mbar_wait(full, 0)) {
+        set_status(p.status, MSA_STATUS_TIMEOUT | MSA_STATUS_AT_ATTEND);
+        if (!mbar_wait(full, 0)) return;  // never leave with copies in flight, within the limit
+        valid = 0;
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int s2 = 0; s2 < kTopK; ++s2)
+        if ((valid >> s2) & 1u) M = fmaxf(M, mls[s2 * kApG + hh].x);
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    int64_t bt = 0;
-    int hq = 0;
-    if (live) {
-        const int kvh = (int)(bk % p.Hkv);
-        bt = bk / p.Hkv;
-        hq = kvh * kApG + hh;
-        const int b = (int)(bt / p.Tq), t = (int)(bt % p.Tq);
-        const int64_t L = clamp_len(p.seq_lens[b], p.Tq, p.lmax, nullptr);
-        const int64_t nvis = (L - p.Tq + t) / kBlock + 1;
-        const int4* selv = reinterpret_cast<const int4*>(w.sel + bt * kTopK);
-        int ids[kTopK];
+    float W = 0.0f;
+    if (M != -INFINITY) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int4 x = __ldg(selv + q);
-            ids[4 * q] = x.x;
-            ids[4 * q + 1] = x.y;
-            ids[4 * q + 2] = x.z;
-            ids[4 * q + 3] = x.w;
-        }
-        float2 ml[kTopK];
-        uint4 ov[kTopK];
-        float M = -INFINITY;
+        for (int s2 = 0; s2 < kTopK; ++s2) {
+            if (!((valid >> s2) & 1u)) continue;
+            const float2 ml = mls[s2 * kApG + hh];
+            const float wt = ml.x == -INFINITY ? 0.0f : exp2f(ml.x - M);
+            W += wt * ml.y;
+            const uint4 ov = slots[s2 * (kMergeSlot / 16) + j];
+            const uint32_t vv[4] = {ov.x, ov.y, ov.z, ov.w};
 #pragma unroll
-        for (int s = 0; s < kTopK; ++s) {
-            const bool valid = ids[s] >= 0 && ids[s] < nvis;
-            const int64_t pr = bt * kTopK + s;  // (token, slot)
-            ml[s] = valid ? __ldcs(w.part_ml + pr * p.Hq + hq) : make_float2(-INFINITY, 0.0f);
-            ov[s] = valid ? __ldcs(reinterpret_cast<const uint4*>(w.part_o + (pr * p.Hkv + kvh) * 1024) + j)
-                          : make_uint4(0, 0, 0, 0);
-            M = fmaxf(M, ml[s].x);
-        }
-        float W = 0.0f;
-        if (M != -INFINITY) {
-#pragma unroll
-            for (int s = 0; s < kTopK; ++s) {
-                const float wt = ml[s].x == -INFINITY ? 0.0f : exp2f(ml[s].x - M);
-                W += wt * ml[s].y;
-                const uint32_t vv[4] = {ov[s].x, ov[s].y, ov[s].z, ov[s].w};
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&vv[q]));
-                    acc[2 * q] += wt * f.x;
-                    acc[2 * q + 1] += wt * f.y;
-                }
+            for (int q = 0; q < 4; ++q) {
+                const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&vv[q]));
+                acc[2 * q] += wt * f.x;
+                acc[2 * q + 1] += wt * f.y;
             }
         }
-        const float inv = W > 0.0f ? 128.0f * p.v.s_t / W : 0.0f;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) acc[q] *= inv;
-        if (g8 == 0 && lse != nullptr) lse[bt * p.Hq + hq] = W > 0.0f ? (M + log2f(W)) * kApLn2 : -INFINITY;
     }
-    // the group's output is [8 heads][128 dims], contiguous in out: stage it, then write it in order
-    float* st = stage[gl];
+    const float inv = W > 0.0f ? 128.0f * p.v.s_t / W : 0.0f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) acc[q] *= inv;
+    if (g8 == 0 && lse != nullptr) lse[bt * p.Hq + hq] = W > 0.0f ? (M + log2f(W)) * kApLn2 : -INFINITY;
+    // the group's output is [8 heads][128 dims], contiguous in out: stage it over the slot buffer
+    // (every read of it is done at the barrier), then write it in order
+    __syncthreads();
+    float* st = reinterpret_cast<float*>(msm);
 #pragma unroll
     for (int q = 0; q < 8; ++q) st[hh * 128 + g8 * 8 + q] = acc[q];
     __syncthreads();
-    if (live) {
-        const int64_t o0 = (bt * p.Hq + (hq - hh)) * 128;  // first element of the group's 8 heads
+    const int64_t o0 = (bt * p.Hq + kvh * kApG) * 128;  // first element of the group's 8 heads
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            const int e = 2 * (j + 128 * q);  // this thread's pairs are e, e + 256, e + 512, e + 768
-            store_out2(p, out, o0 + e, st[e], st[e + 1]);
-        }
+    for (int q = 0; q < 4; ++q) {
+        const int e = 2 * (j + 128 * q);  // this thread's pairs are e, e + 256, e + 512, e + 768
+        store_out2(p, out, o0 + e, st[e], st[e + 1]);
     }
 }
 
@@ -915,9 +925,14 @@ int launch_attend_prefill(const Problem& p, const int32_t* sel, void* ws, float*
     if (cudaLaunchKernelEx(&cfg, ap_tiles_kernel, p, w) != cudaSuccess) return MSA_ECUDA;
     const int r = p.block_table != nullptr ? launch_ap_attend<true>(p, w, pdl, st) : launch_ap_attend<false>(p, w, pdl, st);
     if (r != MSA_OK) return r;
-    const int64_t threads = (int64_t)p.B * p.Tq * p.Hkv * 128;
-    cfg = ap_config(dim3((unsigned)((threads + kMergeThreads - 1) / kMergeThreads)), dim3(kMergeThreads), 0, pdl, st,
-                    attr);
+    static int merge_dev = -1;
+    if (merge_dev != device_info().device) {
+        if (cudaFuncSetAttribute(ap_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMergeSmem) !=
+            cudaSuccess)
+            return MSA_ECUDA;
+        merge_dev = device_info().device;
+    }
+    cfg = ap_config(dim3((unsigned)((int64_t)p.B * p.Tq * p.Hkv)), dim3(kMergeThreads), kMergeSmem, pdl, st, attr);
     if (cudaLaunchKernelEx(&cfg, ap_merge_kernel, p, w, out, lse) != cudaSuccess) return MSA_ECUDA;
     return MSA_OK;
 }
