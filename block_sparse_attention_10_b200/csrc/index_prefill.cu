@@ -229,31 +229,48 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             bool any = false;
             for (int qt = qc * kPfQChunk; qt < qt_end; ++qt) any |= pf_tile_live<HI>(qt, k0, L, Tq);
             if (any) {
-                // dequantise the unit's 256 keys into the bf16 K-major SW128 tile (keys >= L read as 0)
+                // dequantise the unit's 256 keys into the bf16 K-major SW128 tile (keys >= L read as 0).
+                // Each thread owns one 8-element chunk column of every kKeyStep-th key; per MSA block
+                // all of its loads are issued before the first conversion, so the unit boundary (where
+                // the tensor pipe waits for this tile) pays two memory latencies instead of one per chunk.
                 constexpr int kChunksPerRow = DI / 8;
-                for (int ci = et; ci < kPfKeys * kChunksPerRow; ci += 256) {
-                    const int j = ci / kChunksPerRow, cr = ci % kChunksPerRow;
-                    const int64_t key = k0 + j;
-                    uint32_t w = 0u, sc = 0u;
-                    if (key < L) {
-                        const int64_t vec = block_vec<PAGED>(p, b, key / kBlock, 0, 1) + key % kBlock;
-                        w = *reinterpret_cast<const uint32_t*>(p.ik.data + vec * (DI / 2) + cr * 4);
-                        sc = p.ik.scale[vec * (DI / 16) + (cr >> 1)];
-                    }
-                    uint32_t h[4];
-                    e2m1x8_to_f16x8(w, h[0], h[1], h[2], h[3]);
-                    const uint32_t s2 = e4m3_bcast_f16x2(sc);
-                    uint4 o;
-                    uint32_t* op = &o.x;
+                constexpr int kKeyStep = 256 / kChunksPerRow;
+                constexpr int kIt = kBlock / kKeyStep;  // chunks per thread per block
+                static_assert(kBlock % kKeyStep == 0, "a thread's keys must not straddle a block inside one step");
+                const int cr = et % kChunksPerRow, j0 = et / kChunksPerRow;
+                const int kb = cr >> 3, cc = cr & 7;
+#pragma unroll 1
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int jb = h2 * kBlock + j0;
+                    const int64_t vb = k0 + h2 * kBlock < L ? block_vec<PAGED>(p, b, k0 / kBlock + h2, 0, 1) : 0;
+                    uint32_t wv[kIt], sv[kIt];
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const uint32_t m = hmul2(h[i], s2);  // e2m1 * e4m3, exact in f16 and in bf16
-                        const __half2 vm = *reinterpret_cast<const __half2*>(&m);
-                        const __nv_bfloat162 bb = __floats2bfloat162_rn(__low2float(vm), __high2float(vm));
-                        op[i] = *reinterpret_cast<const uint32_t*>(&bb);
+                    for (int it = 0; it < kIt; ++it) {
+                        const int64_t vec = vb + j0 + it * kKeyStep;
+                        wv[it] = 0u;
+                        sv[it] = 0u;
+                        if (k0 + jb + it * kKeyStep < L) {
+                            wv[it] = *reinterpret_cast<const uint32_t*>(p.ik.data + vec * (DI / 2) + cr * 4);
+                            sv[it] = p.ik.scale[vec * (DI / 16) + (cr >> 1)];
+                        }
                     }
-                    const int kb = cr >> 3, cc = cr & 7;
-                    *reinterpret_cast<uint4*>(kbuf + kb * G::kKBlock + j * 128 + ((cc ^ (j & 7)) << 4)) = o;
+#pragma unroll
+                    for (int it = 0; it < kIt; ++it) {
+                        const int j = jb + it * kKeyStep;
+                        uint32_t h[4];
+                        e2m1x8_to_f16x8(wv[it], h[0], h[1], h[2], h[3]);
+                        const uint32_t s2 = e4m3_bcast_f16x2(sv[it]);
+                        uint4 o;
+                        uint32_t* op = &o.x;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const uint32_t m = hmul2(h[i], s2);  // e2m1 * e4m3, exact in f16 and in bf16
+                            const __half2 vm = *reinterpret_cast<const __half2*>(&m);
+                            const __nv_bfloat162 bb = __floats2bfloat162_rn(__low2float(vm), __high2float(vm));
+                            op[i] = *reinterpret_cast<const uint32_t*>(&bb);
+                        }
+                        *reinterpret_cast<uint4*>(kbuf + kb * G::kKBlock + j * 128 + ((cc ^ (j & 7)) << 4)) = o;
+                    }
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
