@@ -15,12 +15,14 @@
 //
 // Design (B200, one persistent CTA per SM, 10 warps):
 //   * work unit = (sequence, 256 keys = 2 MSA blocks, up to 64 query tiles);
-//   * warps 0-7 dequantise the unit's 256 NVFP4 keys into a bf16 shared tile
-//     in the canonical K-major 128-byte-swizzle layout (e2m1*e4m3 is exact in
-//     bf16; the fp32 tensor scale is applied to the pooled score), then run
-//     the epilogue;
+//   * warps 0-7 dequantise each unit's 256 NVFP4 keys into one of two bf16
+//     shared tiles in the canonical K-major 128-byte-swizzle layout (e2m1*e4m3
+//     is exact in bf16; the fp32 tensor scale is applied to the pooled score)
+//     and run the epilogue.  The next unit's keys are written into the other
+//     tile at the start of the current unit, while the MMAs of its first two
+//     query tiles run, so the tensor pipe does not drain at unit boundaries;
 //   * warp 9 (one lane) streams 128-row query tiles [128 x DI] bf16 with TMA
-//     (128-byte swizzle, no multicast) into a 4-stage ring;
+//     (128-byte swizzle, no multicast) into a 3-stage ring;
 //   * warp 8 (one lane) issues tcgen05.mma 128 x 256 x 16 (bf16 -> fp32 in
 //     tensor memory), double-buffered over 2 x 256 TMEM columns, and commits
 //     to mbarriers;
@@ -41,7 +43,7 @@ constexpr int kPfEpiWarps = 8;
 constexpr int kPfMmaWarp = 8;
 constexpr int kPfTmaWarp = 9;
 constexpr int kPfThreads = 32 * 10;
-constexpr int kPfQStages = 4;
+constexpr int kPfQStages = 3;
 constexpr int kPfRows = 128;    // M: query rows (token, head) per tile
 constexpr int kPfKeys = 256;    // N: keys per unit (2 MSA blocks)
 constexpr int kPfQChunk = 64;   // query tiles per unit
@@ -54,7 +56,8 @@ struct PfGeom {
     static constexpr int kQBlock = kPfRows * 128;         // one K-block of a query stage
     static constexpr int kKTile = kPfKeys * DI * 2;       // bf16 key tile
     static constexpr int kKBlock = kPfKeys * 128;         // one K-block of the key tile
-    static constexpr size_t kSmem = 1024 + kKTile + kPfQStages * kQStage + 256;
+    static constexpr size_t kSmem = 1024 + 2 * kKTile + kPfQStages * kQStage + 256;
+    static_assert(kSmem <= 232448, "shared memory per CTA");
 };
 
 struct PfShape {
@@ -86,14 +89,14 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     using G = PfGeom<DI>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* kbuf = smem;
-    uint8_t* qbuf = smem + G::kKTile;
+    uint8_t* kbuf = smem;  // two key tiles
+    uint8_t* qbuf = smem + 2 * G::kKTile;
     uint64_t* q_full = reinterpret_cast<uint64_t*>(qbuf + kPfQStages * G::kQStage);
     uint64_t* q_empty = q_full + kPfQStages;
     uint64_t* t_full = q_empty + kPfQStages;
     uint64_t* t_empty = t_full + 2;
-    uint64_t* k_ready = t_empty + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(k_ready + 1);
+    uint64_t* k_full = t_empty + 2;  // [2]: key tile complete
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(k_full + 2);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     pdl_wait();
@@ -106,7 +109,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             mbar_init(&t_full[s], 1);
             mbar_init(&t_empty[s], kPfEpiWarps);
         }
-        mbar_init(k_ready, kPfEpiWarps);
+        mbar_init(&k_full[0], kPfEpiWarps);
+        mbar_init(&k_full[1], kPfEpiWarps);
         fence_mbar_init();
     }
     if (warp == kPfMmaWarp) {
@@ -173,7 +177,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                 bool any = false;
                 for (int qt = qc * kPfQChunk; qt < qt_end; ++qt) any |= pf_tile_live<HI>(qt, k0, L, Tq);
                 if (!any) continue;
-                if (!mbar_wait(k_ready, ui & 1u)) {
+                if (!mbar_wait(&k_full[ui & 1u], (ui >> 1) & 1u)) {
                     set_status(p.status, MSA_STATUS_TIMEOUT | MSA_STATUS_AT_INDEX_CONSUMER);
                     break;
                 }
@@ -189,7 +193,8 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                         break;
                     }
                     tcgen05_fence_after();
-                    const uint32_t qs = smem_u32(qbuf + s * G::kQStage), ks = smem_u32(kbuf);
+                    const uint32_t qs = smem_u32(qbuf + s * G::kQStage),
+                                   ks = smem_u32(kbuf + (ui & 1u) * G::kKTile);
 #pragma unroll
                     for (int k = 0; k < DI / 16; ++k) {
                         const int kb = k >> 2, kk = k & 3;
@@ -215,7 +220,85 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             for (int64_t n = (L + kBlock - 1) / kBlock; n < p.nbmax; ++n) block_scores[r * p.nbmax + n] = -INFINITY;
         }
         const int quad = warp & 3, hb = warp >> 2;
-        uint32_t qi = 0;
+        // Key dequantisation: each thread owns one 8-element chunk column of every kKeyStep-th
+        // key of an MSA block (keys >= L read as 0); a block's loads are all issued before its
+        // first conversion.
+        constexpr int kChunksPerRow = DI / 8;
+        constexpr int kKeyStep = 256 / kChunksPerRow;
+        constexpr int kIt = kBlock / kKeyStep;  // chunks per thread per block
+        static_assert(kBlock % kKeyStep == 0, "a thread's keys must not straddle a block inside one step");
+        const int cr = et % kChunksPerRow, j0 = et / kChunksPerRow;
+        const int ckb = cr >> 3, ccc = cr & 7;
+        auto load_block = [&](int64_t uu, int h2, uint32_t(&wv)[kIt], uint32_t(&sv)[kIt]) {
+            const int kb_b = (int)(uu / ((int64_t)sh.nkt * sh.nqc));
+            const int64_t kb_k0 = ((uu % ((int64_t)sh.nkt * sh.nqc)) / sh.nqc) * kPfKeys;
+            const int64_t kb_L = clamp_len(p.seq_lens[kb_b], Tq, p.lmax, nullptr);
+            const int64_t vb = kb_k0 + h2 * kBlock < kb_L ? block_vec<PAGED>(p, kb_b, kb_k0 / kBlock + h2, 0, 1) : 0;
+#pragma unroll
+            for (int it = 0; it < kIt; ++it) {
+                const int64_t vec = vb + j0 + it * kKeyStep;
+                wv[it] = 0u;
+                sv[it] = 0u;
+                if (kb_k0 + h2 * kBlock + j0 + it * kKeyStep < kb_L) {
+                    wv[it] = *reinterpret_cast<const uint32_t*>(p.ik.data + vec * (DI / 2) + cr * 4);
+                    sv[it] = p.ik.scale[vec * (DI / 16) + (cr >> 1)];
+                }
+            }
+        };
+        auto store_block = [&](uint8_t* kdst, int h2, const uint32_t(&wv)[kIt], const uint32_t(&sv)[kIt]) {
+#pragma unroll
+            for (int it = 0; it < kIt; ++it) {
+                const int j = h2 * kBlock + j0 + it * kKeyStep;
+                uint32_t hh[4];
+                e2m1x8_to_f16x8(wv[it], hh[0], hh[1], hh[2], hh[3]);
+                const uint32_t s2 = e4m3_bcast_f16x2(sv[it]);
+                uint4 o;
+                uint32_t* op = &o.x;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t m = hmul2(hh[i], s2);  // e2m1 * e4m3, exact in f16 and in bf16
+                    const __half2 vm = *reinterpret_cast<const __half2*>(&m);
+                    const __nv_bfloat162 bb = __floats2bfloat162_rn(__low2float(vm), __high2float(vm));
+                    op[i] = *reinterpret_cast<const uint32_t*>(&bb);
+                }
+                *reinterpret_cast<uint4*>(kdst + ckb * G::kKBlock + j * 128 + ((ccc ^ (j & 7)) << 4)) = o;
+            }
+        };
+        auto publish = [&](uint32_t kbi) {
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&k_full[kbi]);
+        };
+        auto unit_live = [&](int64_t uu) {
+            const int ub = (int)(uu / ((int64_t)sh.nkt * sh.nqc));
+            const int64_t urem = uu % ((int64_t)sh.nkt * sh.nqc);
+            const int64_t uk0 = (urem / sh.nqc) * kPfKeys;
+            const int uqc = (int)(urem % sh.nqc);
+            const int64_t uL = clamp_len(p.seq_lens[ub], Tq, p.lmax, nullptr);
+            bool a2 = false;
+            for (int qt = uqc * kPfQChunk; qt < min(sh.nqt, (uqc + 1) * kPfQChunk); ++qt)
+                a2 |= pf_tile_live<HI>(qt, uk0, uL, Tq);
+            return a2;
+        };
+        auto next_live = [&](int64_t uu) {
+            for (uu += gridDim.x; uu < sh.units; uu += gridDim.x)
+                if (unit_live(uu)) return uu;
+            return sh.units;
+        };
+        // this CTA's first live unit: its keys go to tile 0 before any query tile
+        int64_t u_live = (int64_t)blockIdx.x >= sh.units ? sh.units
+                         : unit_live(blockIdx.x)            ? (int64_t)blockIdx.x
+                                                            : next_live(blockIdx.x);
+        if (u_live < sh.units) {
+#pragma unroll 1
+            for (int h2 = 0; h2 < 2; ++h2) {
+                uint32_t wv[kIt], sv[kIt];
+                load_block(u_live, h2, wv, sv);
+                store_block(kbuf, h2, wv, sv);
+            }
+            publish(0);
+        }
+        uint32_t qi = 0, ui = 0;
         bool ok = true;
         for (int64_t u = blockIdx.x; u < sh.units && ok; u += gridDim.x) {
             const int b = (int)(u / ((int64_t)sh.nkt * sh.nqc));
@@ -226,55 +309,21 @@ __global__ void __launch_bounds__(kPfThreads, 1)
             const int64_t nb_b = (L + kBlock - 1) / kBlock;
             const int64_t n = k0 / kBlock + hb;  // this warp's block
             const int qt_end = min(sh.nqt, (qc + 1) * kPfQChunk);
-            bool any = false;
-            for (int qt = qc * kPfQChunk; qt < qt_end; ++qt) any |= pf_tile_live<HI>(qt, k0, L, Tq);
+            const bool any = u == u_live;
+            // A live unit first writes the next live unit's keys into the other tile (free: its MMAs
+            // ended before this unit's first tile); the MMAs of this unit's first two query tiles
+            // need nothing from these warps and run meanwhile.
             if (any) {
-                // dequantise the unit's 256 keys into the bf16 K-major SW128 tile (keys >= L read as 0).
-                // Each thread owns one 8-element chunk column of every kKeyStep-th key; per MSA block
-                // all of its loads are issued before the first conversion, so the unit boundary (where
-                // the tensor pipe waits for this tile) pays two memory latencies instead of one per chunk.
-                constexpr int kChunksPerRow = DI / 8;
-                constexpr int kKeyStep = 256 / kChunksPerRow;
-                constexpr int kIt = kBlock / kKeyStep;  // chunks per thread per block
-                static_assert(kBlock % kKeyStep == 0, "a thread's keys must not straddle a block inside one step");
-                const int cr = et % kChunksPerRow, j0 = et / kChunksPerRow;
-                const int kb = cr >> 3, cc = cr & 7;
+                u_live = next_live(u);
+                if (u_live < sh.units) {
 #pragma unroll 1
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    const int jb = h2 * kBlock + j0;
-                    const int64_t vb = k0 + h2 * kBlock < L ? block_vec<PAGED>(p, b, k0 / kBlock + h2, 0, 1) : 0;
-                    uint32_t wv[kIt], sv[kIt];
-#pragma unroll
-                    for (int it = 0; it < kIt; ++it) {
-                        const int64_t vec = vb + j0 + it * kKeyStep;
-                        wv[it] = 0u;
-                        sv[it] = 0u;
-                        if (k0 + jb + it * kKeyStep < L) {
-                            wv[it] = *reinterpret_cast<const uint32_t*>(p.ik.data + vec * (DI / 2) + cr * 4);
-                            sv[it] = p.ik.scale[vec * (DI / 16) + (cr >> 1)];
-                        }
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        uint32_t wv[kIt], sv[kIt];
+                        load_block(u_live, h2, wv, sv);
+                        store_block(kbuf + ((ui + 1) & 1u) * G::kKTile, h2, wv, sv);
                     }
-#pragma unroll
-                    for (int it = 0; it < kIt; ++it) {
-                        const int j = jb + it * kKeyStep;
-                        uint32_t h[4];
-                        e2m1x8_to_f16x8(wv[it], h[0], h[1], h[2], h[3]);
-                        const uint32_t s2 = e4m3_bcast_f16x2(sv[it]);
-                        uint4 o;
-                        uint32_t* op = &o.x;
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const uint32_t m = hmul2(h[i], s2);  // e2m1 * e4m3, exact in f16 and in bf16
-                            const __half2 vm = *reinterpret_cast<const __half2*>(&m);
-                            const __nv_bfloat162 bb = __floats2bfloat162_rn(__low2float(vm), __high2float(vm));
-                            op[i] = *reinterpret_cast<const uint32_t*>(&bb);
-                        }
-                        *reinterpret_cast<uint4*>(kbuf + kb * G::kKBlock + j * 128 + ((cc ^ (j & 7)) << 4)) = o;
-                    }
+                    publish((ui + 1) & 1u);
                 }
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(k_ready);
             }
             // Per tile, the row's token moves on by kPfRows / HI and its head stays the same, so the
             // token, its count of visible keys in this warp's block and its score address step by
@@ -359,6 +408,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
                     *dst = st_cnt == kBlock ? (xs[0] * (1.0f / kBlock)) * s_t
                                             : st_cnt > 0 ? (xs[0] / (float)st_cnt) * s_t : -INFINITY;
             }
+            if (any) ++ui;
         }
     }
 
