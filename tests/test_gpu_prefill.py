@@ -111,6 +111,33 @@ def _sample_tokens(Tq, L, n, seed):
     return sorted(toks)
 
 
+def test_prefill_indexer_many_units_per_cta():
+    """Every CTA of the tensor-core indexer runs several (sequence, 256-key, query-chunk) units
+    here (2 x 256 key tiles x 1 chunk over 148 CTAs), and the shorter sequence's units past its
+    length see no token, so live and dead units alternate within a CTA: the pooled scores of
+    sampled rows must equal the oracle's over every block (each unit's keys come from the key
+    tile written during the unit before it)."""
+    inp = _custom(2, 512, 8, 1, 8, 128, [40000, 65536], 65536, seed=11)
+    p = problem_from_inputs(inp)
+    B, Tq = inp.w.B, inp.w.Tq
+    bs = torch.full((B, Tq, p.nbmax), float("nan"), device="cuda")
+    msa.msa_index(p, bs)
+    torch.cuda.synchronize()
+    assert int(p.status.item()) == 0
+    gbs = bs.cpu().numpy()
+    ik_all = oracle.nvfp4_encode(inp.ik.numpy(), inp.s_ik)
+    for b, L in enumerate(inp.seq_lens):
+        tokens = _sample_tokens(Tq, L, 40, seed=200 + b)
+        pos = [L - Tq + t for t in tokens]
+        ik = oracle.Nvfp4(ik_all.data[b:b + 1], ik_all.scale[b:b + 1], ik_all.tensor_scale)
+        obs = oracle_index_rows(bf16_values(inp.q_idx[b])[tokens], ik, pos)
+        got = gbs[b, tokens]
+        fin = np.isfinite(obs)
+        assert np.array_equal(fin, np.isfinite(got)), "visibility of blocks differs"
+        scale = np.abs(obs[fin]).mean()
+        np.testing.assert_allclose(got[fin], obs[fin], rtol=1e-4, atol=1e-5 * scale)
+
+
 def test_prefill_full_size_sampled_tokens():
     """The full-size chunked-prefill workload in bench.py's launch configuration (one
     msa_decode over both sequences), checked on 128 sampled query tokens of each sequence
