@@ -16,7 +16,7 @@ import oracle
 from block_sparse_attention_10_b200 import configs, msa, synth
 from tests._common import (bf16_values, check_attention, check_selection, oracle_attend_rows,
                            oracle_caches, oracle_index_rows)
-from tests._gpu import problem_from_inputs, run_decode
+from tests._gpu import paged_problem, problem_from_inputs, run_decode
 
 pytestmark = pytest.mark.gpu
 
@@ -111,13 +111,15 @@ def _sample_tokens(Tq, L, n, seed):
     return sorted(toks)
 
 
-def test_prefill_indexer_many_units_per_cta():
+@pytest.mark.parametrize("DI,HI,paged", [(128, 8, False), (64, 4, False), (128, 8, True)])
+def test_prefill_indexer_many_units_per_cta(DI, HI, paged):
     """Every CTA of the tensor-core indexer runs several (sequence, 256-key, query-chunk) units
     here (2 x 256 key tiles x 1 chunk over 148 CTAs), and the shorter sequence's units past its
     length see no token, so live and dead units alternate within a CTA: the pooled scores of
     sampled rows must equal the oracle's over every block (each unit's keys come from the key
-    tile written during the unit before it)."""
-    inp = _custom(2, 512, 8, 1, 8, 128, [40000, 65536], 65536, seed=11)
+    tile written during the unit before it).  Both head dims, and a paged cache (bitwise equal
+    to the contiguous one as well)."""
+    inp = _custom(2, 512, 8, 1, HI, DI, [40000, 65536], 65536, seed=11)
     p = problem_from_inputs(inp)
     B, Tq = inp.w.B, inp.w.Tq
     bs = torch.full((B, Tq, p.nbmax), float("nan"), device="cuda")
@@ -125,6 +127,15 @@ def test_prefill_indexer_many_units_per_cta():
     torch.cuda.synchronize()
     assert int(p.status.item()) == 0
     gbs = bs.cpu().numpy()
+    if paged:
+        pp = paged_problem(p, seed=5)
+        bsp = torch.full((B, Tq, p.nbmax), float("nan"), device="cuda")
+        msa.msa_index(pp, bsp)
+        torch.cuda.synchronize()
+        assert int(pp.status.item()) == 0
+        gbsp = bsp.cpu().numpy()
+        assert np.array_equal(np.nan_to_num(gbs).view(np.uint32), np.nan_to_num(gbsp).view(np.uint32))
+        gbs = gbsp
     ik_all = oracle.nvfp4_encode(inp.ik.numpy(), inp.s_ik)
     for b, L in enumerate(inp.seq_lens):
         tokens = _sample_tokens(Tq, L, 40, seed=200 + b)
