@@ -109,7 +109,7 @@ def test_single_launch_rejects_before_enqueueing(L):
 
 @pytest.mark.parametrize("field,value,code", [
     ("lmax", 4000, 1), ("B", 0, 1), ("Tq", 0, 1), ("seq_lens", None, 1), ("pool_mode", 2, 1),
-    ("D", 64, 2), ("DI", 96, 2), ("HI", 3, 2), ("Hq", 24, 2), ("B", 5000, 2),
+    ("D", 64, 2), ("DI", 96, 2), ("HI", 3, 2), ("Hq", 24, 2), ("B", 4097, 2), ("B", 5000, 2),
     ("q", 0x8001, 3), ("q_idx", 0x9008, 3),
 ])
 def test_decode_rejects_bad_params(L, field, value, code):
