@@ -1,7 +1,7 @@
 """msa_select on crafted pooled scores against the oracle, bit-exact: exact ties (at and
 away from the cutoff), rows where every score is equal, negative scores, and row lengths
 that reach each selection kernel (one warp per row up to 1,024 blocks, a two-level CTA
-up to 4,096, the round-based CTA beyond)."""
+up to 4,096, the round-based CTA beyond), also with thousands of such rows."""
 import ctypes
 
 import numpy as np
@@ -56,6 +56,26 @@ def test_select_crafted_scores_bit_exact(nbmax, kind):
     Tq = 2
     # visible-block counts from 1 up to the whole row; query t of sequence b sits at L - Tq + t
     lens = sorted({2, 129, 130, 16 * 128 + 1, 17 * 128, lmax // 2 + 5, lmax - 1, lmax} & set(range(2, lmax + 1)))
+    B = len(lens)
+    scores = np.full((B, Tq, nbmax), -np.inf, np.float32)
+    for b, L in enumerate(lens):
+        for t in range(Tq):
+            nvis = (L - Tq + t) // 128 + 1
+            scores[b, t, :nvis] = _pattern(kind, rng, nvis)
+    got = _select(scores, lens, Tq)
+    want = oracle.select(scores.astype(np.float64), lens)
+    assert np.array_equal(got, want)
+
+
+@pytest.mark.parametrize("nbmax", [1056, 2048])
+@pytest.mark.parametrize("kind", ["distinct", "few_levels", "tie_at_cutoff"])
+def test_select_many_long_rows_bit_exact(nbmax, kind):
+    """Thousands of rows of more than 1,024 blocks, as in a chunk of prefill tokens (the
+    two-level CTA kernel, one CTA per row)."""
+    rng = np.random.default_rng(nbmax + 3 * len(kind))
+    lmax = nbmax * 128
+    Tq = 1500
+    lens = [lmax, lmax - 1, lmax // 2 + 5, Tq + 1000]
     B = len(lens)
     scores = np.full((B, Tq, nbmax), -np.inf, np.float32)
     for b, L in enumerate(lens):
